@@ -1,0 +1,302 @@
+"""Seeded synthetic inputs for the gated delta-rule layer.
+
+This module is shared by the tests, the benchmark and the oracle harness.  It
+holds no arithmetic of the method itself: it draws random numbers, rounds them
+to bf16 and lays them out.  Every tensor it returns is a numpy array:
+
+* bf16 tensors are ``uint16`` arrays holding the raw bf16 bit patterns,
+* fp32 tensors are ``float32`` arrays,
+* ``cu_seqlens`` is ``int32``.
+
+Distributions follow the workloads the layer is exercised on (16 key heads,
+48 value heads, head dim 128; see the recipe in the repository's design
+notes):
+
+* q, k, v, x, a, b, z  ~ N(0, 1)
+* A_log   = log U(1, 16)                  (one per value head)
+* dt_bias = log(expm1(U(1e-3, 0.1)))     (one per value head)
+* conv weights ~ N(0, 0.5) (std 0.5)
+* initial recurrent states ~ N(0, 0.02) (std 0.02)
+
+The generator is numpy's PCG64 seeded with the workload's seed; draws happen
+in a fixed documented order so that a workload is reproducible bit for bit.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+HK = 16          # key heads
+HV = 48          # value heads
+DK = 128         # key head dim
+DV = 128         # value head dim
+CONV_K = 4       # causal conv width
+CHUNK = 64       # chunk length of the prefill
+
+
+# ---------------------------------------------------------------------------
+# bf16 bit handling (input preparation only)
+# ---------------------------------------------------------------------------
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (round to nearest, ties to even).
+
+    Returns the bf16 bit patterns as uint16.  Inputs are finite.
+    """
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    r = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to float32."""
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    return bf16_bits_to_f32(b).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# primitive draws
+# ---------------------------------------------------------------------------
+
+def _rng(seed: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _normal_bf16(rng, shape, std=1.0) -> np.ndarray:
+    x = rng.standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        x *= np.float32(std)
+    return f32_to_bf16_bits(x)
+
+
+def _unit_rows_bf16(rng, shape) -> np.ndarray:
+    """N(0,1) rows rescaled to unit L2 length along the last axis, then bf16.
+
+    This is the input recipe "q and k L2-normalised per head".
+    """
+    x = rng.standard_normal(size=shape, dtype=np.float32)
+    n = np.sqrt(np.sum(x.astype(np.float64) ** 2, axis=-1, keepdims=True))
+    return f32_to_bf16_bits((x / n).astype(np.float32))
+
+
+def _head_params(rng, hv):
+    """A_log = log U(1,16), dt_bias = log(expm1(U(1e-3, 0.1))), float32."""
+    A_log = np.log(rng.uniform(1.0, 16.0, size=hv)).astype(np.float32)
+    dt = rng.uniform(1e-3, 0.1, size=hv)
+    dt_bias = np.log(np.expm1(dt)).astype(np.float32)
+    return A_log, dt_bias
+
+
+def varlen_lengths(seed: int, n: int, lo: int, hi: int) -> np.ndarray:
+    """n sequence lengths drawn uniformly from the integers [lo, hi]."""
+    rng = _rng(seed)
+    return rng.integers(lo, hi + 1, size=n).astype(np.int64)
+
+
+def cu_seqlens_from_lengths(lengths) -> np.ndarray:
+    cu = np.zeros(len(lengths) + 1, dtype=np.int64)
+    cu[1:] = np.cumsum(np.asarray(lengths, dtype=np.int64))
+    assert cu[-1] < 2 ** 31
+    return cu.astype(np.int32)
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class CoreInputs:
+    """Inputs of the recurrence alone (already convolved / no conv)."""
+    q: np.ndarray            # [T, hk, dk]  bf16 bits
+    k: np.ndarray            # [T, hk, dk]  bf16 bits
+    v: np.ndarray            # [T, hv, dv]  bf16 bits
+    a: np.ndarray            # [T, hv]      bf16 bits
+    b: np.ndarray            # [T, hv]      bf16 bits
+    A_log: np.ndarray        # [hv] f32
+    dt_bias: np.ndarray      # [hv] f32
+    cu_seqlens: np.ndarray   # [N+1] int32
+    h0: Optional[np.ndarray] # [N, hv, dk, dv] f32 or None
+    scale: float = 1.0
+
+    @property
+    def T(self):
+        return int(self.q.shape[0])
+
+    @property
+    def n_seqs(self):
+        return int(self.cu_seqlens.shape[0] - 1)
+
+
+def make_core_inputs(seed: int, lengths, hk=HK, hv=HV, dk=DK, dv=DV,
+                     prenorm_qk=True, h0_std: Optional[float] = None,
+                     scale: float = 1.0) -> CoreInputs:
+    """Draw order: q, k, v, a, b, A_log/dt_bias, h0."""
+    rng = _rng(seed)
+    cu = cu_seqlens_from_lengths(lengths)
+    T = int(cu[-1])
+    if prenorm_qk:
+        q = _unit_rows_bf16(rng, (T, hk, dk))
+        k = _unit_rows_bf16(rng, (T, hk, dk))
+    else:
+        q = _normal_bf16(rng, (T, hk, dk))
+        k = _normal_bf16(rng, (T, hk, dk))
+    v = _normal_bf16(rng, (T, hv, dv))
+    a = _normal_bf16(rng, (T, hv))
+    b = _normal_bf16(rng, (T, hv))
+    A_log, dt_bias = _head_params(rng, hv)
+    h0 = None
+    if h0_std is not None:
+        h0 = (rng.standard_normal(size=(len(lengths), hv, dk, dv), dtype=np.float32)
+              * np.float32(h0_std))
+    return CoreInputs(q, k, v, a, b, A_log, dt_bias, cu, h0, scale)
+
+
+@dataclasses.dataclass
+class FullInputs:
+    """Inputs of the whole prefill path: conv -> recurrence -> gated norm."""
+    x: np.ndarray            # [T, C] bf16 bits, C = hk*dk + hk*dk + hv*dv ([q | k | v])
+    conv_w: np.ndarray       # [C, 4] bf16 bits
+    conv_state: Optional[np.ndarray]  # [N, 3, C] bf16 bits or None (zeros)
+    a: np.ndarray            # [T, hv] bf16 bits
+    b: np.ndarray            # [T, hv] bf16 bits
+    z: np.ndarray            # [T, hv, dv] bf16 bits
+    norm_w: Optional[np.ndarray]  # [dv] f32 or None (ones)
+    A_log: np.ndarray
+    dt_bias: np.ndarray
+    cu_seqlens: np.ndarray
+    h0: Optional[np.ndarray]
+    hk: int = HK
+    hv: int = HV
+    dk: int = DK
+    dv: int = DV
+    scale: float = 1.0
+    eps: float = 1e-6
+
+    @property
+    def T(self):
+        return int(self.x.shape[0])
+
+    @property
+    def n_seqs(self):
+        return int(self.cu_seqlens.shape[0] - 1)
+
+    @property
+    def channels(self):
+        return int(self.x.shape[1])
+
+
+def make_full_inputs(seed: int, lengths, hk=HK, hv=HV, dk=DK, dv=DV,
+                     h0_std: Optional[float] = None, conv_state_std: Optional[float] = None,
+                     norm_w_std: Optional[float] = None, scale: float = 1.0,
+                     eps: float = 1e-6) -> FullInputs:
+    """Draw order: x, conv_w, a, b, z, A_log/dt_bias, h0, conv_state, norm_w."""
+    rng = _rng(seed)
+    cu = cu_seqlens_from_lengths(lengths)
+    T = int(cu[-1])
+    C = hk * dk * 2 + hv * dv
+    x = _normal_bf16(rng, (T, C))
+    conv_w = _normal_bf16(rng, (C, CONV_K), std=0.5)
+    a = _normal_bf16(rng, (T, hv))
+    b = _normal_bf16(rng, (T, hv))
+    z = _normal_bf16(rng, (T, hv, dv))
+    A_log, dt_bias = _head_params(rng, hv)
+    h0 = None
+    if h0_std is not None:
+        h0 = (rng.standard_normal(size=(len(lengths), hv, dk, dv), dtype=np.float32)
+              * np.float32(h0_std))
+    conv_state = None
+    if conv_state_std is not None:
+        conv_state = _normal_bf16(rng, (len(lengths), CONV_K - 1, C), std=conv_state_std)
+    norm_w = None
+    if norm_w_std is not None:
+        norm_w = (1.0 + rng.standard_normal(size=(dv,), dtype=np.float32)
+                  * np.float32(norm_w_std)).astype(np.float32)
+    return FullInputs(x, conv_w, conv_state, a, b, z, norm_w, A_log, dt_bias, cu, h0,
+                      hk, hv, dk, dv, scale, eps)
+
+
+@dataclasses.dataclass
+class DecodeInputs:
+    """B independent sequences advanced by `steps` single-token steps."""
+    x: np.ndarray            # [steps, B, C] bf16 bits (pre-conv)
+    a: np.ndarray            # [steps, B, hv] bf16 bits
+    b: np.ndarray            # [steps, B, hv] bf16 bits
+    conv_w: np.ndarray       # [C, 4] bf16 bits
+    conv_state: np.ndarray   # [B, 3, C] bf16 bits
+    state: np.ndarray        # [B, hv, dk, dv] f32
+    A_log: np.ndarray
+    dt_bias: np.ndarray
+    hk: int = HK
+    hv: int = HV
+    dk: int = DK
+    dv: int = DV
+    scale: float = 1.0
+
+    @property
+    def B(self):
+        return int(self.x.shape[1])
+
+    @property
+    def steps(self):
+        return int(self.x.shape[0])
+
+
+def make_decode_inputs(seed: int, batch: int, steps: int, hk=HK, hv=HV, dk=DK, dv=DV,
+                       state_std=0.02, conv_state_std=1.0, scale: float = 1.0) -> DecodeInputs:
+    """Draw order: state, conv_state, conv_w, A_log/dt_bias, then per step x, a, b."""
+    rng = _rng(seed)
+    C = hk * dk * 2 + hv * dv
+    state = (rng.standard_normal(size=(batch, hv, dk, dv), dtype=np.float32)
+             * np.float32(state_std))
+    conv_state = _normal_bf16(rng, (batch, CONV_K - 1, C), std=conv_state_std)
+    conv_w = _normal_bf16(rng, (C, CONV_K), std=0.5)
+    A_log, dt_bias = _head_params(rng, hv)
+    x = np.empty((steps, batch, C), dtype=np.uint16)
+    a = np.empty((steps, batch, hv), dtype=np.uint16)
+    b = np.empty((steps, batch, hv), dtype=np.uint16)
+    for s in range(steps):
+        x[s] = _normal_bf16(rng, (batch, C))
+        a[s] = _normal_bf16(rng, (batch, hv))
+        b[s] = _normal_bf16(rng, (batch, hv))
+    return DecodeInputs(x, a, b, conv_w, conv_state, state, A_log, dt_bias,
+                        hk, hv, dk, dv, scale)
+
+
+# ---------------------------------------------------------------------------
+# the five workloads of the layer (sizes and seeds)
+# ---------------------------------------------------------------------------
+
+def workload_core_T128(seed=0):
+    """B=1, T=128, pre-normalised q/k, zero initial state, no conv."""
+    return make_core_inputs(seed, [128], prenorm_qk=True)
+
+
+def workload_full_T4096(seed=1):
+    """B=1, T=4096, conv4+SiLU -> recurrence -> gated RMSNorm, zero state."""
+    return make_full_inputs(seed, [4096])
+
+
+def workload_decode_B64(seed=2, steps=1000):
+    """64 sequences, one token per step, fp32 states ~ N(0, 0.02)."""
+    return make_decode_inputs(seed, 64, steps)
+
+
+def workload_core_T262144(seed=3):
+    """B=1, T=262144, pre-normalised q/k, zero initial state, no conv."""
+    return make_core_inputs(seed, [262144], prenorm_qk=True)
+
+
+def varlen8_lengths(seed=4):
+    return varlen_lengths(seed, 8, 1024, 32768)
+
+
+def workload_full_varlen8(seed=4):
+    """8 packed sequences, lengths U{1024..32768}, h0 ~ N(0,0.02), full path."""
+    return make_full_inputs(seed + 1000, varlen8_lengths(seed), h0_std=0.02)

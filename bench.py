@@ -1,0 +1,380 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta-rule layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload full_T4096|decode_B64|core_T262144|varlen8|core_T128]
+
+A step of the default workload is one pass of the prefill path of one layer
+over B=1, T=4096 tokens: causal conv4+SiLU over the 10240 q|k|v channels ->
+chunk-64 gated delta rule (16 key / 48 value heads, dim 128) -> gated RMSNorm.
+The decode path (B=64 sequences, one token each, 1000 consecutive steps) is
+measured in the same run and reported under "decode".  Inputs are seeded
+synthetic tensors (gdr_inputs) with the layer's shapes; there are no weights.
+
+Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs its own
+replica of the workload (the path has no cross-GPU exchange) and the value is
+the sum over ranks divided by the max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gdr_inputs as GI  # noqa: E402
+
+METRIC_PREFILL = "GDR prefill tokens/s/layer"
+METRIC_DECODE = "GDR decode steps/s at B=64"
+L2_BYTES = 126 * 1024 * 1024
+
+# algorithmic HBM bytes per token of each kernel (bf16 tensors, fp32 states)
+CX = 2 * GI.HK * GI.DK + GI.HV * GI.DV                  # 10240 conv channels
+B_CONV = CX * 2 * 2                                      # x read + y write
+B_CORE = (2 * GI.HK * GI.DK + GI.HV * GI.DV) * 2 + 2 * GI.HV * 2 + GI.HV * GI.DV * 2   # q,k,v,a,b + o
+B_NORM = 3 * GI.HV * GI.DV * 2                           # o, z read + y write
+B_FUSED = CX * 2 + 2 * GI.HV * 2 + 2 * GI.HV * GI.DV * 2 # x, a, b, z read + y write
+STATE_BYTES = GI.HV * GI.DK * GI.DV * 4                  # one sequence's fp32 state
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled while the timed region runs
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+def to_dev(torch, bits, device):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+class PrefillRunner:
+    """conv -> chunk prefill -> gated RMSNorm over FullInputs, all on the device."""
+
+    def __init__(self, torch, G, inp, device):
+        self.torch, self.G, self.inp = torch, G, inp
+        f = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+        self.x = to_dev(torch, inp.x, device)
+        self.w = to_dev(torch, inp.conv_w, device)
+        self.a = to_dev(torch, inp.a, device)
+        self.b = to_dev(torch, inp.b, device)
+        self.z = to_dev(torch, inp.z, device).reshape(inp.T, inp.hv, 128)
+        self.A_log, self.dt_bias = f(inp.A_log), f(inp.dt_bias)
+        self.cu_host = inp.cu_seqlens
+        self.cu = torch.from_numpy(inp.cu_seqlens.astype(np.int32)).to(device)
+        self.h0 = f(inp.h0) if inp.h0 is not None else None
+        T, hk, hv = inp.T, inp.hk, inp.hv
+        self.conv_y = torch.empty((T, CX), dtype=torch.bfloat16, device=device)
+        self.q = self.conv_y[:, : hk * 128]
+        self.o = torch.empty((T, hv, 128), dtype=torch.bfloat16, device=device)
+        self.y = torch.empty((T, hv, 128), dtype=torch.bfloat16, device=device)
+        self.hT = torch.empty((inp.n_seqs, hv, 128, 128), dtype=torch.float32, device=device)
+        self.ev = None
+
+    def step(self, prefill_events=None):
+        torch, G, inp = self.torch, self.G, self.inp
+        T, hk, hv = inp.T, inp.hk, inp.hv
+        G.causal_conv(self.x, self.w, self.cu, self.cu_host, None, None, self.conv_y)
+        y = self.conv_y
+        # q, k, v are token-strided views of the [T, q|k|v] conv output, read in place
+        q = y[:, : hk * 128].view(T, hk, 128)
+        k = y[:, hk * 128: 2 * hk * 128].view(T, hk, 128)
+        v = y[:, 2 * hk * 128:].view(T, hv, 128)
+        if prefill_events:
+            prefill_events[0].record()
+        G.chunk_prefill(q, k, v, self.a, self.b, self.A_log, self.dt_bias, self.cu, self.cu_host,
+                        h0=self.h0, hT=self.hT, o=self.o, scale=inp.scale)
+        if prefill_events:
+            prefill_events[1].record()
+        G.gated_rmsnorm(self.o, self.z, None, inp.eps, self.y)
+
+
+def bench_ours(args, rank, world, device):
+    import torch
+    import gated_delta_rule_63_b200 as G
+    G.lib()
+    torch.cuda.set_device(device)
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    inp = GI.workload_full_T4096()
+    T = inp.T
+    run = PrefillRunner(torch, G, inp, device)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+
+    for _ in range(args.warmup):
+        run.step()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    pev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                      else 0) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))                     # evict L2 between timed steps
+            ev[i][0].record()
+            run.step(pev[i])
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        # decode: B=64, 1000 consecutive steps, state updated in place
+        dec_res = bench_decode(torch, G, device, args)
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    pre_ms = [a.elapsed_time(b) for a, b in pev]
+    ms = sum(step_ms) / len(step_ms)
+    pms = sum(pre_ms) / len(pre_ms)
+    if world > 1:
+        t = torch.tensor([ms, pms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, pms = float(t[0]), float(t[1])
+    value = world * T / (ms * 1e-3)
+
+    # end to end through the C ABI with host buffers (pinned), copies inside
+    e2e = bench_e2e(torch, G, inp, device, args)
+
+    prefill_bytes = T * B_CORE + inp.n_seqs * STATE_BYTES
+    achieved = prefill_bytes / (pms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC_PREFILL, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in/out, fp32 state",
+        "data": "synthetic (seeded gdr_inputs, no weights)",
+        "config": {"workload": "full_T4096: B=1 T=4096 conv4+SiLU -> chunk-64 GDR -> gated RMSNorm, "
+                               "hk=16 hv=48 d=128", "global_batch": world, "seq_len": T,
+                   "parallelism": f"replicas x{world}", "l2": "flushed between timed steps (252 MB write)",
+                   "fused": False},
+        "roofline": {"kernel": "gdr_chunk_prefill", "bound": "hbm", "achieved": achieved,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                     "peak_kind": peak_kind, "traffic": None,
+                     "algorithmic_bytes_per_launch": prefill_bytes, "ms_per_launch": pms},
+        "step_roofline": {"bytes_per_token_unfused": B_CONV + B_CORE + B_NORM,
+                          "bytes_per_token_fused": B_FUSED,
+                          "frac_of_fused_hbm_roofline": (T * B_FUSED + STATE_BYTES) / (ms * 1e-3) / 1e9 / hbm_peak},
+        "decode": dec_res,
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps + dec_res["launches"],
+        "clocks": clk.summary(),
+    }
+    return res
+
+
+def bench_decode(torch, G, device, args, steps=1000):
+    hbm_peak, _, _ = measured_peaks()
+    dec = GI.make_decode_inputs(2, 64, 8)       # 8 distinct token batches, reused round robin
+    xs = to_dev(torch, dec.x, device)
+    as_ = to_dev(torch, dec.a, device)
+    bs = to_dev(torch, dec.b, device)
+    cw = to_dev(torch, dec.conv_w, device)
+    cs = to_dev(torch, dec.conv_state, device)
+    st = torch.from_numpy(dec.state).to(device)
+    Al = torch.from_numpy(dec.A_log).to(device)
+    db = torch.from_numpy(dec.dt_bias).to(device)
+    o = torch.empty((64, dec.hv, 128), dtype=torch.bfloat16, device=device)
+    for s in range(5):
+        G.decode_step(xs[s % 8], cw, cs, as_[s % 8], bs[s % 8], Al, db, st, o)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(steps):
+        G.decode_step(xs[s % 8], cw, cs, as_[s % 8], bs[s % 8], Al, db, st, o)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    bytes_step = 64 * STATE_BYTES * 2
+    achieved = bytes_step / (ms * 1e-3) / 1e9
+    return {"metric": METRIC_DECODE, "value": 1e3 / ms, "unit": "steps/s", "ms_per_step": ms,
+            "steps": steps, "launches": steps,
+            "roofline": {"kernel": "gdr_decode_step", "bound": "hbm", "achieved": achieved,
+                         "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                         "algorithmic_bytes_per_launch": bytes_step, "traffic": None}}
+
+
+def bench_e2e(torch, G, inp, device, args):
+    """Same prefill step through the C ABI from pinned host buffers, copies included."""
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()
+    hx, ha, hb, hz = pin(inp.x), pin(inp.a), pin(inp.b), pin(inp.z)
+    run = PrefillRunner(torch, G, inp, device)
+    hy = torch.empty(run.y.shape, dtype=torch.bfloat16).pin_memory()
+    hT = torch.empty(run.hT.shape, dtype=torch.float32).pin_memory()
+
+    def one():
+        run.x.view(torch.int16).copy_(hx, non_blocking=True)
+        run.a.view(torch.int16).copy_(ha, non_blocking=True)
+        run.b.view(torch.int16).copy_(hb, non_blocking=True)
+        run.z.view(torch.int16).view(-1).copy_(hz.view(-1), non_blocking=True)
+        run.step()
+        hy.copy_(run.y, non_blocking=True)
+        hT.copy_(run.hT, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    h2d = (inp.x.nbytes + inp.a.nbytes + inp.b.nbytes + inp.z.nbytes)
+    d2h = hy.numel() * 2 + hT.numel() * 4
+    return {"value": inp.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle as it stands, on the host cores
+# ---------------------------------------------------------------------------
+def oracle_step(O, inp):
+    return O.full_path(inp)
+
+
+def cpu_baseline(inp=None):
+    from oracle import oracle as O
+    inp = inp or GI.workload_full_T4096()
+    t0 = time.perf_counter()
+    oracle_step(O, inp)
+    dt = time.perf_counter() - t0
+    return {"value": inp.T / dt, "unit": "tokens/s", "cores": O.default_threads(), "kind": "oracle",
+            "sample": f"one full_T4096 step (all 48 heads, T={inp.T}), fp64 stepwise, "
+                      f"{dt:.2f} s wall"}
+
+
+def bench_reference(args, rank, world):
+    """The oracle timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    from oracle import oracle as O
+    inp = GI.workload_full_T4096()
+    for _ in range(min(args.warmup, 1)):
+        oracle_step(O, inp)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(O, inp)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    v = inp.T / (ms * 1e-3)
+    return {"impl": "reference", "metric": METRIC_PREFILL, "value": v, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded gdr_inputs, no weights)",
+            "config": {"workload": "full_T4096: B=1 T=4096 conv4+SiLU -> chunk-64 GDR -> gated RMSNorm, "
+                                   "hk=16 hv=48 d=128", "global_batch": 1, "seq_len": inp.T,
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": O.default_threads(),
+                             "kind": "oracle", "sample": "full_T4096 step, every head, fp64 stepwise"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = bench_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    res = bench_ours(args, rank, world, device)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

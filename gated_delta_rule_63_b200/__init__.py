@@ -1,0 +1,234 @@
+"""Gated delta-rule layer on NVIDIA B200 (sm_100a): Python binding of libgdr.so.
+
+A thin ctypes layer over the C ABI declared in ``include/gdr.h``: each function
+checks dtypes and shapes, passes raw device pointers and the current CUDA
+stream, and raises ``GdrError`` on a non-zero status.  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback path.
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+__all__ = [
+    "GdrError", "lib", "status_string", "prepare_chunks", "causal_conv", "chunk_prefill",
+    "decode_step", "gated_rmsnorm", "get_device_error", "HEAD_DIM", "CHUNK",
+]
+
+HEAD_DIM = 128
+CHUNK = 64
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdr.so")
+
+_vp = ctypes.c_void_p
+_ip = ctypes.POINTER(ctypes.c_int32)
+
+
+class GdrError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {status_string(code)} (status {code})")
+        self.code = code
+
+
+class FuseArgs(ctypes.Structure):
+    """Mirror of ``gdr_prefill_fuse_t``."""
+    _fields_ = [("x", _vp), ("conv_w", _vp), ("conv_state_in", _vp), ("conv_state_out", _vp),
+                ("z", _vp), ("norm_w", _vp), ("eps", ctypes.c_float), ("y", _vp)]
+
+
+_lib = None
+
+
+def lib(path: Optional[str] = None):
+    """Load libgdr.so (built in-tree by ``gated_delta_rule_63_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m gated_delta_rule_63_b200.build`")
+    L = ctypes.CDLL(path)
+    L.gdr_status_string.restype = ctypes.c_char_p
+    L.gdr_status_string.argtypes = [ctypes.c_int]
+    L.gdr_abi_version.restype = ctypes.c_int
+    L.gdr_prepare_chunks.argtypes = [_ip, ctypes.c_int, ctypes.c_int, _ip, _ip, _ip, ctypes.c_int,
+                                     ctypes.POINTER(ctypes.c_int)]
+    L.gdr_causal_conv.argtypes = [_vp, _vp, _vp, _vp, _vp, _ip, ctypes.c_int, ctypes.c_int, _vp, _vp]
+    L.gdr_chunk_prefill.argtypes = [_vp, _vp, _vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp,
+                                    _vp, ctypes.c_float, ctypes.c_int,
+                                    ctypes.c_int, _vp, _ip, ctypes.c_int, _vp, _vp, _vp,
+                                    ctypes.POINTER(FuseArgs), _vp]
+    L.gdr_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_int,
+                                  ctypes.c_int, _vp, _vp, ctypes.c_int, _vp]
+    L.gdr_gated_rmsnorm.argtypes = [_vp, _vp, _vp, ctypes.c_float, ctypes.c_int64, ctypes.c_int, _vp,
+                                    _vp]
+    L.gdr_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), _vp]
+    for fn in ("gdr_prepare_chunks", "gdr_causal_conv", "gdr_chunk_prefill", "gdr_decode_step",
+               "gdr_gated_rmsnorm", "gdr_get_device_error"):
+        getattr(L, fn).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().gdr_status_string(int(code)).decode()
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise GdrError(fn, code)
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t, dtype=None, name="tensor", rows=False):
+    """Device pointer of a tensor; with rows=True only the last two dims must be dense."""
+    if t is None:
+        return None
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if rows:
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError(f"{name} must be [T, heads, 128] with dense rows")
+    elif not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _tok_stride(t):
+    return 0 if t is None else int(t.stride(0))
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _host_cu(cu_host):
+    cu = np.ascontiguousarray(np.asarray(cu_host), dtype=np.int32)
+    return cu, cu.ctypes.data_as(_ip)
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+
+def prepare_chunks(cu_seqlens_host, chunk: int = CHUNK):
+    """Chunk table (chunk_seq, chunk_start, chunk_len) of packed sequences."""
+    cu, cup = _host_cu(cu_seqlens_host)
+    n = cu.shape[0] - 1
+    total = int(cu[-1]) if n > 0 else 0
+    cap = max(1, total // max(chunk, 1) + n + 1)
+    seq = np.zeros(cap, np.int32); st = np.zeros(cap, np.int32); ln = np.zeros(cap, np.int32)
+    m = ctypes.c_int(0)
+    _check("gdr_prepare_chunks", lib().gdr_prepare_chunks(
+        cup, n, int(chunk), seq.ctypes.data_as(_ip), st.ctypes.data_as(_ip), ln.ctypes.data_as(_ip),
+        cap, ctypes.byref(m)))
+    k = m.value
+    return seq[:k].copy(), st[:k].copy(), ln[:k].copy()
+
+
+def causal_conv(x, w, cu_seqlens, cu_seqlens_host, conv_state_in=None, conv_state_out=None, y=None,
+                stream=None):
+    """Depthwise causal conv4 + SiLU.  x [T, C] bf16, w [C, 4] bf16 -> y [T, C] bf16."""
+    torch = _torch()
+    bf = torch.bfloat16
+    cu, cup = _host_cu(cu_seqlens_host)
+    if y is None:
+        y = torch.empty_like(x)
+    C = x.shape[1]
+    _check("gdr_causal_conv", lib().gdr_causal_conv(
+        _ptr(x, bf, "x"), _ptr(w, bf, "w"), _ptr(conv_state_in, bf, "conv_state_in"),
+        _ptr(conv_state_out, bf, "conv_state_out"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup,
+        cu.shape[0] - 1, C, _ptr(y, bf, "y"), _stream(stream)))
+    return y
+
+
+def chunk_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_host, h0=None, hT=None,
+                  o=None, scale: float = 1.0, fuse: Optional[dict] = None, stream=None):
+    """Chunk-64 prefill.  q, k [T, hk, 128], v [T, hv, 128], a, b [T, hv] bf16.
+
+    q, k, v may be token-strided views (e.g. slices of the [T, q|k|v] conv output).
+
+    Returns o [T, hv, 128] bf16 (and writes hT [N, hv, 128, 128] fp32 when given).
+    ``fuse`` (optional) maps gdr_prefill_fuse_t field names to tensors.
+    """
+    torch = _torch()
+    bf, f32 = torch.bfloat16, torch.float32
+    cu, cup = _host_cu(cu_seqlens_host)
+    fz = None
+    if fuse is not None:
+        fz = FuseArgs()
+        for name in ("x", "conv_w", "conv_state_in", "conv_state_out", "z", "y"):
+            setattr(fz, name, _ptr(fuse.get(name), bf, name))
+        fz.norm_w = _ptr(fuse.get("norm_w"), f32, "norm_w")
+        fz.eps = float(fuse.get("eps", 1e-6))
+    hk = q.shape[1] if q is not None else int(fuse["hk"])
+    hv = a.shape[1]
+    if q is not None and k.stride(0) != q.stride(0):
+        raise ValueError("q and k must share their token stride")
+    if o is None and (fuse is None or fuse.get("y") is None or fuse.get("keep_o", False)):
+        T = a.shape[0]
+        o = torch.empty((T, hv, HEAD_DIM), dtype=bf, device=a.device)
+    _check("gdr_chunk_prefill", lib().gdr_chunk_prefill(
+        _ptr(q, bf, "q", rows=True), _ptr(k, bf, "k", rows=True), _ptr(v, bf, "v", rows=True),
+        _tok_stride(q), _tok_stride(v), _ptr(a, bf, "a"), _ptr(b, bf, "b"),
+        _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"), float(scale), int(hk), int(hv),
+        _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup, cu.shape[0] - 1,
+        _ptr(h0, f32, "h0"), _ptr(hT, f32, "hT"), _ptr(o, bf, "o"),
+        ctypes.byref(fz) if fz is not None else None, _stream(stream)))
+    return o
+
+
+def decode_step(x, conv_w, conv_state, a, b, A_log, dt_bias, state, o=None, scale: float = 1.0,
+                hk: int = 16, stream=None):
+    """One token for each of B sequences; conv_state and state are updated in place."""
+    torch = _torch()
+    bf, f32 = torch.bfloat16, torch.float32
+    B, hv = a.shape
+    if o is None:
+        o = torch.empty((B, hv, HEAD_DIM), dtype=bf, device=a.device)
+    _check("gdr_decode_step", lib().gdr_decode_step(
+        _ptr(x, bf, "x"), _ptr(conv_w, bf, "conv_w"), _ptr(conv_state, bf, "conv_state"),
+        _ptr(a, bf, "a"), _ptr(b, bf, "b"), _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"),
+        float(scale), int(hk), int(hv), _ptr(state, f32, "state"), _ptr(o, bf, "o"), int(B),
+        _stream(stream)))
+    return o
+
+
+def gated_rmsnorm(o, z, w=None, eps: float = 1e-6, y=None, stream=None):
+    """y = o / sqrt(mean(o^2) + eps) * w * SiLU(z) over rows of 128."""
+    torch = _torch()
+    bf = torch.bfloat16
+    if y is None:
+        y = torch.empty_like(o)
+    d = o.shape[-1]
+    rows = o.numel() // d
+    _check("gdr_gated_rmsnorm", lib().gdr_gated_rmsnorm(
+        _ptr(o, bf, "o"), _ptr(z, bf, "z"), _ptr(w, torch.float32, "w"), float(eps), int(rows), int(d),
+        _ptr(y, bf, "y"), _stream(stream)))
+    return y
+
+
+def get_device_error(stream=None) -> int:
+    """Read and clear the library's device error word (synchronises the stream)."""
+    v = ctypes.c_int(0)
+    _check("gdr_get_device_error", lib().gdr_get_device_error(ctypes.byref(v), _stream(stream)))
+    return v.value

@@ -1,0 +1,186 @@
+// gdr_host.cu -- the C ABI of libgdr.so: argument checks, chunk table, error word.
+//
+// Every entry point validates its arguments on the host and returns a
+// gdr_status_t before anything is launched; the launchers live next to their
+// kernels.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdr_common.cuh"
+#include "gdr_host.h"
+
+#include <atomic>
+
+namespace gdr {
+__device__ int g_device_error = 0;
+
+int *device_error_ptr() {
+  static std::atomic<int *> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  int *p = cache[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_device_error) != cudaSuccess) return nullptr;
+    p = static_cast<int *>(addr);
+    cache[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+}  // namespace gdr
+
+using namespace gdr;
+
+extern "C" {
+
+const char *gdr_status_string(int status) {
+  switch (status) {
+    case GDR_OK: return "GDR_OK";
+    case GDR_ERR_NULL: return "GDR_ERR_NULL: a required pointer is NULL";
+    case GDR_ERR_SHAPE: return "GDR_ERR_SHAPE: invalid or inconsistent size";
+    case GDR_ERR_ALIGN: return "GDR_ERR_ALIGN: tensor pointer not 16-byte aligned";
+    case GDR_ERR_CU_SEQLENS: return "GDR_ERR_CU_SEQLENS: offsets must start at 0 and not decrease";
+    case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED: head dims or grouping not implemented";
+    case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE";
+    case GDR_ERR_CUDA: return "GDR_ERR_CUDA: CUDA launch failed";
+    case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a bounded wait in a kernel ran out";
+    case GDR_ERR_ALIAS: return "GDR_ERR_ALIAS: buffers overlap";
+    default: return "GDR_ERR_UNKNOWN";
+  }
+}
+
+int gdr_abi_version(void) { return 1; }
+
+int gdr_prepare_chunks(const int32_t *cu, int n_seqs, int chunk, int32_t *chunk_seq,
+                       int32_t *chunk_start, int32_t *chunk_len, int max_chunks, int *n_chunks) {
+  if (!cu || !n_chunks) return GDR_ERR_NULL;
+  if (chunk <= 0 || max_chunks < 0) return GDR_ERR_SHAPE;
+  int st = check_cu_seqlens(cu, n_seqs);
+  if (st) return st;
+  if (max_chunks > 0 && (!chunk_seq || !chunk_start || !chunk_len)) return GDR_ERR_NULL;
+  int m = 0;
+  for (int n = 0; n < n_seqs; ++n) {
+    // number of chunks of sequence n, ceil(len / chunk)
+    const int64_t len = static_cast<int64_t>(cu[n + 1]) - cu[n];
+    const int64_t nc = (len + chunk - 1) / chunk;
+    for (int64_t c = 0; c < nc; ++c) {
+      if (m >= max_chunks) {
+        *n_chunks = m;
+        return GDR_ERR_SHAPE;
+      }
+      const int64_t start = cu[n] + c * chunk;
+      const int64_t rest = cu[n + 1] - start;
+      chunk_seq[m] = n;
+      chunk_start[m] = static_cast<int32_t>(start);
+      chunk_len[m] = static_cast<int32_t>(rest < chunk ? rest : chunk);
+      ++m;
+    }
+  }
+  *n_chunks = m;
+  return GDR_OK;
+}
+
+int gdr_get_device_error(int *error_out, void *stream) {
+  if (!error_out) return GDR_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int zero = 0, val = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&val, g_device_error, sizeof(int), 0,
+                                            cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return GDR_ERR_CUDA;
+  *error_out = val;
+  return GDR_OK;
+}
+
+int gdr_causal_conv(const void *x, const void *w, const void *conv_state_in, void *conv_state_out,
+                    const int32_t *cu_dev, const int32_t *cu_host, int n_seqs, int channels, void *y,
+                    void *stream) {
+  if (!cu_host) return GDR_ERR_NULL;
+  int st = check_cu_seqlens(cu_host, n_seqs);
+  if (st) return st;
+  if (channels <= 0 || channels % 8 != 0) return GDR_ERR_SHAPE;
+  const int total = n_seqs > 0 ? cu_host[n_seqs] : 0;
+  if (n_seqs == 0) return GDR_OK;
+  if (!cu_dev || !w) return GDR_ERR_NULL;
+  if (total > 0 && (!x || !y)) return GDR_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) || !aligned16(conv_state_in) ||
+      !aligned16(conv_state_out))
+    return GDR_ERR_ALIGN;
+  const size_t state_bytes = static_cast<size_t>(n_seqs) * 3 * channels * 2;
+  if (overlaps(conv_state_in, state_bytes, conv_state_out, state_bytes)) return GDR_ERR_ALIAS;
+  const size_t act_bytes = static_cast<size_t>(total) * channels * 2;
+  if (overlaps(x, act_bytes, y, act_bytes)) return GDR_ERR_ALIAS;
+  return launch_causal_conv(x, w, conv_state_in, conv_state_out, cu_dev, n_seqs, total, channels, y,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int gdr_gated_rmsnorm(const void *o, const void *z, const float *w, float eps, int64_t rows, int d,
+                      void *y, void *stream) {
+  if (rows < 0) return GDR_ERR_SHAPE;
+  if (d != kHeadDim) return GDR_ERR_UNSUPPORTED;
+  if (rows == 0) return GDR_OK;
+  if (!o || !z || !y) return GDR_ERR_NULL;
+  if (!aligned16(o) || !aligned16(z) || !aligned16(y) || !aligned16(w)) return GDR_ERR_ALIGN;
+  if (!(eps >= 0.0f)) return GDR_ERR_SHAPE;
+  return launch_gated_rmsnorm(o, z, w, eps, rows, y, static_cast<cudaStream_t>(stream));
+}
+
+int gdr_decode_step(const void *x, const void *conv_w, void *conv_state, const void *a, const void *b,
+                    const float *A_log, const float *dt_bias, float scale, int hk, int hv,
+                    float *state, void *o, int batch, void *stream) {
+  int st = check_heads(hk, hv);
+  if (st) return st;
+  if (batch < 0) return GDR_ERR_SHAPE;
+  if (batch == 0) return GDR_OK;
+  if (!x || !conv_w || !conv_state || !a || !b || !A_log || !dt_bias || !state || !o)
+    return GDR_ERR_NULL;
+  if (!aligned16(x) || !aligned16(conv_w) || !aligned16(conv_state) || !aligned16(state) ||
+      !aligned16(o))
+    return GDR_ERR_ALIGN;
+  return launch_decode(x, conv_w, conv_state, a, b, A_log, dt_bias, scale, hk, hv, state, o, batch,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_stride,
+                      int64_t v_stride, const void *a, const void *b, const float *A_log,
+                      const float *dt_bias, float scale, int hk, int hv, const int32_t *cu_dev,
+                      const int32_t *cu_host, int n_seqs, const float *h0, float *hT, void *o,
+                      const gdr_prefill_fuse_t *fuse, void *stream) {
+  int st = check_heads(hk, hv);
+  if (st) return st;
+  if (qk_stride == 0) qk_stride = static_cast<int64_t>(hk) * kHeadDim;
+  if (v_stride == 0) v_stride = static_cast<int64_t>(hv) * kHeadDim;
+  if (qk_stride < static_cast<int64_t>(hk) * kHeadDim || v_stride < static_cast<int64_t>(hv) * kHeadDim)
+    return GDR_ERR_SHAPE;
+  if (qk_stride % 8 != 0 || v_stride % 8 != 0) return GDR_ERR_ALIGN;
+  if (!cu_host) return GDR_ERR_NULL;
+  st = check_cu_seqlens(cu_host, n_seqs);
+  if (st) return st;
+  if (n_seqs == 0) return GDR_OK;
+  const int total = cu_host[n_seqs];
+  int max_len = 0;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int len = cu_host[i + 1] - cu_host[i];
+    if (len > max_len) max_len = len;
+  }
+  if (!cu_dev) return GDR_ERR_NULL;
+  const bool fused_conv = fuse && fuse->x;
+  const bool fused_norm = fuse && fuse->z;
+  if (fused_conv || fused_norm) return GDR_ERR_UNSUPPORTED;   // fusion not built yet
+  if (total > 0) {
+    if (!a || !b || !A_log || !dt_bias) return GDR_ERR_NULL;
+    if (!q || !k || !v || !o) return GDR_ERR_NULL;
+  }
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(h0) ||
+      !aligned16(hT))
+    return GDR_ERR_ALIGN;
+  const size_t state_bytes = static_cast<size_t>(n_seqs) * hv * kHeadDim * kHeadDim * 4;
+  if (h0 != hT && overlaps(h0, state_bytes, hT, state_bytes)) return GDR_ERR_ALIAS;
+  return launch_chunk_prefill(q, k, v, qk_stride, v_stride, a, b, A_log, dt_bias, scale, hk, hv,
+                              cu_dev, n_seqs, max_len,
+                              h0, hT, o, fuse, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

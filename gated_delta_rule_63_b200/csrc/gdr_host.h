@@ -1,0 +1,66 @@
+// gdr_host.h -- host-side argument checks shared by the entry points.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdr.h"
+
+namespace gdr {
+
+constexpr int kHeadDim = 128;
+constexpr int kChunk = 64;
+constexpr int kConvK = 4;
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Ranges [a, a + na) and [b, b + nb) in bytes overlap.
+inline bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const char *pa = static_cast<const char *>(a), *pb = static_cast<const char *>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+// Heads supported by the kernels: dk = dv = 128, hv % hk == 0, group <= 8.
+inline int check_heads(int hk, int hv) {
+  if (hk <= 0 || hv <= 0) return GDR_ERR_SHAPE;
+  if (hv % hk != 0 || hv / hk > 8) return GDR_ERR_UNSUPPORTED;
+  return GDR_OK;
+}
+
+// Host copy of cu_seqlens: starts at 0, non-decreasing, total < 2^31.
+inline int check_cu_seqlens(const int32_t *cu, int n_seqs) {
+  if (!cu) return GDR_ERR_NULL;
+  if (n_seqs < 0) return GDR_ERR_SHAPE;
+  if (cu[0] != 0) return GDR_ERR_CU_SEQLENS;
+  for (int i = 0; i < n_seqs; ++i)
+    if (cu[i + 1] < cu[i]) return GDR_ERR_CU_SEQLENS;
+  return GDR_OK;
+}
+
+// Device address of the library's error word on the current device (cached).
+int *device_error_ptr();
+
+inline int launch_status(cudaError_t e) { return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA; }
+
+inline int last_launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+// Launchers implemented in the kernel files (arguments already checked).
+int launch_causal_conv(const void *x, const void *w, const void *cs_in, void *cs_out,
+                       const int32_t *cu_dev, int n_seqs, int total, int channels, void *y,
+                       cudaStream_t s);
+int launch_gated_rmsnorm(const void *o, const void *z, const float *w, float eps, int64_t rows,
+                         void *y, cudaStream_t s);
+int launch_decode(const void *x, const void *conv_w, void *conv_state, const void *a, const void *b,
+                  const float *A_log, const float *dt_bias, float scale, int hk, int hv,
+                  float *state, void *o, int batch, cudaStream_t s);
+int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_stride,
+                         int64_t v_stride, const void *a, const void *b,
+                         const float *A_log, const float *dt_bias, float scale, int hk, int hv,
+                         const int32_t *cu_dev, int n_seqs, int max_len, const float *h0, float *hT,
+                         void *o, const gdr_prefill_fuse_t *fuse, cudaStream_t s);
+
+}  // namespace gdr

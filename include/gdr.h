@@ -1,0 +1,204 @@
+/*
+ * gdr.h -- C ABI of the gated delta-rule layer library (libgdr.so), sm_100a.
+ *
+ * The layer (one of the 54 recurrent layers of the hybrid decoder described in
+ * "Agnes-3.0-Flash 深度解析：33B 混合注意力多模态模型", section 注意力层的细节):
+ * 16 key heads and 48 value heads of dimension 128, a kernel-4 depthwise
+ * causal conv with SiLU in front, L2-normalised q and k, a decay gate and a
+ * write strength per token and value head, an fp32 recurrent state of
+ * 128 x 128 per value head, and a gated RMSNorm on the output.
+ *
+ * The recurrence ("Sapiens AI 发布 Agnes-3.0-Flash", section
+ * "delta 规则循环层究竟怎么运作", with the forget gate of the gated variant):
+ *     S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = scale * S_t q_t
+ * with ("33B 只做 18 层：Agnes 3.0 Flash ...", §1.2)
+ *     beta_t = sigmoid(b_t),  g_t = -exp(A_log) * softplus(a_t + dt_bias)
+ * computed in fp32, and q, k divided by sqrt(sum x^2 + 1e-6) inside the
+ * kernels.  Value head h reads key head h / (hv / hk).
+ *
+ * Conventions shared by every entry point
+ *  - Tensor pointers are DEVICE memory owned by the caller, except the
+ *    `*_host` arguments, which are host memory.  The library allocates no
+ *    device memory and keeps no per-call state; it writes a device-side error
+ *    word only when a kernel hits a bounded wait (gdr_get_device_error).
+ *  - bf16 tensors are passed as `void *` holding IEEE bfloat16 values; fp32
+ *    tensors as `float *`.  All layouts are dense row-major (C order) with the
+ *    shapes written next to each argument.  Every tensor pointer must be
+ *    16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *    enqueued asynchronously; no call synchronises the device.
+ *  - The recurrent state is stored transposed, H = S^T, as
+ *    [n][hv][dk][dv] fp32 (the dv index is contiguous).
+ *  - Supported dims: dk = dv = 128, hk >= 1, hv % hk == 0, hv / hk <= 8.
+ *  - A non-zero return value is a gdr_status_t; nothing has been launched
+ *    when an argument check fails.  GDR_ERR_CUDA reports a failed launch.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDR_API __attribute__((visibility("default")))
+#else
+#define GDR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdr_status {
+  GDR_OK = 0,
+  GDR_ERR_NULL = 1,        /* a required pointer is NULL */
+  GDR_ERR_SHAPE = 2,       /* a size is negative, zero where it must not be, or inconsistent */
+  GDR_ERR_ALIGN = 3,       /* a tensor pointer is not 16-byte aligned */
+  GDR_ERR_CU_SEQLENS = 4,  /* cu_seqlens does not start at 0 or decreases */
+  GDR_ERR_UNSUPPORTED = 5, /* head dims / grouping outside what the kernels implement */
+  GDR_ERR_WORKSPACE = 6,   /* reserved */
+  GDR_ERR_CUDA = 7,        /* the CUDA launch failed (see cudaGetLastError) */
+  GDR_ERR_TIMEOUT = 8,     /* (device error word) a bounded wait inside a kernel ran out */
+  GDR_ERR_ALIAS = 9        /* two buffers overlap where the call forbids it */
+} gdr_status_t;
+
+/* Human-readable name of a status code.  Never NULL. */
+GDR_API const char *gdr_status_string(int status);
+
+/* ABI version of this header; bumped on any signature change. */
+GDR_API int gdr_abi_version(void);
+
+/*
+ * Chunk table of packed sequences (host only, no device work).
+ * Chunks of `chunk` tokens restart at every sequence start; the last chunk of
+ * a sequence may be shorter; empty sequences have no chunk.  Chunks are listed
+ * sequence by sequence in token order: chunk m covers tokens
+ * [chunk_start[m], chunk_start[m] + chunk_len[m]) of sequence chunk_seq[m].
+ *   cu_seqlens_host: [n_seqs + 1] int32 token offsets, cu[0] = 0, non-decreasing.
+ *   chunk_seq, chunk_start, chunk_len: host arrays of max_chunks entries.
+ * Returns GDR_ERR_CU_SEQLENS for an invalid offset array and GDR_ERR_SHAPE if
+ * the table needs more than max_chunks entries; *n_chunks receives the count.
+ * The prefill kernel walks exactly this table.
+ */
+GDR_API int gdr_prepare_chunks(const int32_t *cu_seqlens_host, int n_seqs, int chunk, int32_t *chunk_seq,
+                       int32_t *chunk_start, int32_t *chunk_len, int max_chunks, int *n_chunks);
+
+/*
+ * gdr_causal_conv -- depthwise causal conv, kernel 4, followed by SiLU,
+ * over packed sequences ("Agnes-3.0-Flash 深度解析", 注意力层的细节: a kernel-4
+ * causal conv in front of the recurrence).
+ *     y[t][c] = SiLU(sum_{j=0..3} w[c][j] * x[t-3+j][c])   (fp32 math, bf16 out)
+ * w[c][3] multiplies the current token.  Inputs before a sequence's first
+ * token come from conv_state_in[n] (oldest first) or are zero when
+ * conv_state_in is NULL; nothing crosses a cu_seqlens boundary.
+ *   x:              bf16 [T][channels]        (T = cu_seqlens_host[n_seqs])
+ *   w:              bf16 [channels][4]
+ *   conv_state_in:  bf16 [n_seqs][3][channels] or NULL
+ *   conv_state_out: bf16 [n_seqs][3][channels] or NULL; receives the last three
+ *                   inputs of each sequence (shifted from conv_state_in when a
+ *                   sequence is shorter than three).  Must not overlap
+ *                   conv_state_in (GDR_ERR_ALIAS).
+ *   cu_seqlens_dev / cu_seqlens_host: the same [n_seqs + 1] int32 offsets on
+ *                   the device and on the host.
+ *   y:              bf16 [T][channels]; channels % 8 == 0.
+ */
+GDR_API int gdr_causal_conv(const void *x, const void *w, const void *conv_state_in, void *conv_state_out,
+                    const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int n_seqs,
+                    int channels, void *y, void *stream);
+
+/*
+ * Optional fusion of the conv in front of and the gated RMSNorm behind the
+ * prefill (pass NULL to gdr_chunk_prefill to run the recurrence alone).
+ * When `x` is set, q, k and v are read as the conv output of x (channels laid
+ * out [q | k | v] = hk*128 + hk*128 + hv*128) and the q/k/v arguments of
+ * gdr_chunk_prefill must be NULL.  When `z` is set, y receives the gated
+ * RMSNorm of o.
+ */
+typedef struct gdr_prefill_fuse {
+  const void *x;             /* bf16 [T][hk*128*2 + hv*128] conv input, or NULL */
+  const void *conv_w;        /* bf16 [channels][4] (required with x) */
+  const void *conv_state_in; /* bf16 [n_seqs][3][channels] or NULL (zeros) */
+  void *conv_state_out;      /* bf16 [n_seqs][3][channels] or NULL; must not overlap conv_state_in */
+  const void *z;             /* bf16 [T][hv][128] gate of the RMSNorm, or NULL */
+  const float *norm_w;       /* fp32 [128] norm weight, or NULL (ones) */
+  float eps;                 /* RMSNorm epsilon */
+  void *y;                   /* bf16 [T][hv][128] (required with z) */
+} gdr_prefill_fuse_t;
+
+/*
+ * gdr_chunk_prefill -- the recurrence over packed sequences, chunk of 64
+ * ("33B 只做 18 层 ...", §1.2: prefill takes the chunk-64 path, said to be
+ * interchangeable with the per-token one).
+ * Per chunk the kernel uses the WY/UT form of the unrolled recurrence; the
+ * dense products run on the tcgen05 tensor cores and the state carried from
+ * chunk to chunk stays fp32.
+ *   q, k:     bf16 [T][hk][128] rows, consecutive tokens qk_token_stride
+ *             elements apart (0 = dense, hk*128)
+ *   v:        bf16 [T][hv][128] rows, consecutive tokens v_token_stride
+ *             elements apart (0 = dense, hv*128).  The strides let q, k, v be
+ *             read in place from the [T][q | k | v] conv output (stride
+ *             2*hk*128 + hv*128); a stride must be a multiple of 8.
+ *   a, b:     bf16 [T][hv]            gate inputs (see the header comment)
+ *   A_log, dt_bias: fp32 [hv]
+ *   scale:    output scale
+ *   cu_seqlens_dev / cu_seqlens_host: [n_seqs + 1] int32, same values.
+ *   h0:       fp32 [n_seqs][hv][128][128] initial state (H = S^T), or NULL = zeros
+ *   hT:       fp32 [n_seqs][hv][128][128] final state, or NULL; may equal h0
+ *             (in place), must not overlap it otherwise.
+ *   o:        bf16 [T][hv][128]; may be NULL only when fuse->y is set.
+ *   fuse:     NULL, or conv / gated-norm fusion (see gdr_prefill_fuse_t).
+ * Empty sequences copy h0 (or zeros) to hT.
+ */
+GDR_API int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_token_stride,
+                              int64_t v_token_stride, const void *a, const void *b,
+                              const float *A_log, const float *dt_bias, float scale, int hk, int hv,
+                              const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                              int n_seqs, const float *h0, float *hT, void *o,
+                              const gdr_prefill_fuse_t *fuse, void *stream);
+
+/*
+ * gdr_decode_step -- one token for each of `batch` independent sequences
+ * ("33B 只做 18 层 ...", §1.2: the single-step recurrent call taken when one
+ * new token resumes from the cached state; "33B 只做 18 层 ..." (mhpq.cn)
+ * §2.1: the single-step form of the causal conv).
+ * Per sequence: conv step y = SiLU(w0 s0 + w1 s1 + w2 s2 + w3 x) over all
+ * channels (rounded to bf16), the conv state rolls to (s1, s2, x); then the
+ * L2 norm of q and k, the gates, and one step of the recurrence on the state,
+ * which is read once and written once in place.
+ *   x:          bf16 [batch][hk*128*2 + hv*128] this step's conv input [q | k | v]
+ *   conv_w:     bf16 [channels][4]
+ *   conv_state: bf16 [batch][3][channels], in/out (updated in place)
+ *   a, b:       bf16 [batch][hv]
+ *   A_log, dt_bias: fp32 [hv]
+ *   state:      fp32 [batch][hv][128][128], in/out (updated in place)
+ *   o:          bf16 [batch][hv][128]
+ */
+GDR_API int gdr_decode_step(const void *x, const void *conv_w, void *conv_state, const void *a, const void *b,
+                    const float *A_log, const float *dt_bias, float scale, int hk, int hv,
+                    float *state, void *o, int batch, void *stream);
+
+/*
+ * gdr_gated_rmsnorm -- gated RMSNorm over rows of d values
+ * ("Agnes-3.0-Flash 深度解析", 注意力层的细节: gated RMS-norm; the z
+ * projection of width 6144 = 48 x 128 in the parameter table of
+ * "33B 只做 18 层 ...", §2):
+ *     y = o / sqrt(mean(o^2) + eps) * w * SiLU(z)    (fp32 math, bf16 out)
+ *   o, z, y: bf16 [rows][d], d == 128;  w: fp32 [d] or NULL (ones).
+ *   y may equal o (in place).
+ */
+GDR_API int gdr_gated_rmsnorm(const void *o, const void *z, const float *w, float eps, int64_t rows, int d,
+                      void *y, void *stream);
+
+/*
+ * Read and clear the device-side error word (0 = none, else a gdr_status_t
+ * such as GDR_ERR_TIMEOUT) after the work queued on `stream` completes.
+ * This call synchronises `stream`.
+ */
+GDR_API int gdr_get_device_error(int *error_out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H_ */

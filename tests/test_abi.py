@@ -1,0 +1,136 @@
+"""The C ABI without a GPU: the library loads, exports what include/gdr.h
+declares, and rejects bad arguments on the host before launching anything."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import gated_delta_rule_63_b200 as G
+from gated_delta_rule_63_b200 import build as B
+from oracle import oracle as O
+import gdr_inputs as GI
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return G.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "gdr.h")).read()
+    return sorted(set(re.findall(r"GDR_API[^;(]*?\b(gdr_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for fn in ("gdr_causal_conv", "gdr_chunk_prefill", "gdr_decode_step", "gdr_gated_rmsnorm",
+               "gdr_prepare_chunks", "gdr_status_string"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    assert G.status_string(0) == "GDR_OK"
+    for code in range(1, 10):
+        assert G.status_string(code).startswith("GDR_ERR_")
+    assert "UNKNOWN" in G.status_string(12345)
+    assert L.gdr_abi_version() == 1
+
+
+@pytest.mark.parametrize("lengths", [[0], [1], [64], [65, 0, 128, 1, 63], [5000, 3, 64 * 7 + 1],
+                                     list(GI.varlen8_lengths())])
+def test_prepare_chunks_is_bit_exact_with_oracle(L, lengths):
+    cu = GI.cu_seqlens_from_lengths(lengths)
+    got = G.prepare_chunks(cu, 64)
+    ref = O.prepare_chunks(cu, 64)
+    for g, r in zip(got, ref):
+        assert g.dtype == np.int32 and np.array_equal(g, r)
+
+
+def test_prepare_chunks_errors(L):
+    with pytest.raises(G.GdrError) as e:
+        G.prepare_chunks(np.array([0, 5, 4], np.int32))
+    assert e.value.code == 4
+    with pytest.raises(G.GdrError) as e:
+        G.prepare_chunks(np.array([2, 5], np.int32))
+    assert e.value.code == 4
+    cu = np.array([0, 200], np.int32)
+    seq = np.zeros(2, np.int32)
+    m = ctypes.c_int(0)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    rc = L.gdr_prepare_chunks(cu.ctypes.data_as(ip), 1, 64, seq.ctypes.data_as(ip),
+                              seq.ctypes.data_as(ip), seq.ctypes.data_as(ip), 2, ctypes.byref(m))
+    assert rc == 2 and m.value == 2   # needs 4 entries, had room for 2
+
+
+FAKE = 0x10000      # an aligned address that is never dereferenced: checks fail first
+ODD = 0x10002
+
+
+def _cu(lengths):
+    cu = GI.cu_seqlens_from_lengths(lengths)
+    return cu, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def test_prefill_rejects_bad_arguments_on_host(L):
+    cu, cup = _cu([10, 5])
+    args = dict(q=FAKE, k=FAKE, v=FAKE, qs=0, vs=0, a=FAKE, b=FAKE, A_log=FAKE, dt_bias=FAKE, scale=1.0, hk=16,
+                hv=48, cu_dev=FAKE, cu_host=cup, n=2, h0=None, hT=FAKE, o=FAKE, fuse=None, s=None)
+
+    def call(**kw):
+        a = dict(args); a.update(kw)
+        return L.gdr_chunk_prefill(a["q"], a["k"], a["v"], a["qs"], a["vs"], a["a"], a["b"],
+                                   a["A_log"], a["dt_bias"],
+                                   a["scale"], a["hk"], a["hv"], a["cu_dev"], a["cu_host"], a["n"],
+                                   a["h0"], a["hT"], a["o"], a["fuse"], a["s"])
+    assert call(hk=16, hv=40) == 5          # grouping not integral
+    assert call(hk=1, hv=48) == 5           # group of 48 > 8
+    assert call(hk=0) == 2
+    assert call(q=None) == 1
+    assert call(cu_dev=None) == 1
+    assert call(cu_host=None) == 1
+    assert call(o=ODD) == 3
+    bad, badp = _cu([3])
+    bad[0] = 1
+    assert call(cu_host=badp, n=1) == 4
+    assert call(h0=FAKE + 64, hT=FAKE) == 9  # partial overlap of h0 and hT
+    assert call(qs=16 * 128 - 8) == 2          # token stride shorter than a row
+    assert call(vs=48 * 128 + 4) == 3          # token stride not a multiple of 8
+
+
+def test_other_entry_points_reject_bad_arguments(L):
+    cu, cup = _cu([4])
+    assert L.gdr_causal_conv(FAKE, FAKE, None, None, FAKE, cup, 1, 10, FAKE, None) == 2   # C % 8
+    assert L.gdr_causal_conv(FAKE, FAKE, FAKE, FAKE, FAKE, cup, 1, 16, FAKE, None) == 9   # state alias
+    assert L.gdr_causal_conv(ODD, FAKE, None, None, FAKE, cup, 1, 16, FAKE, None) == 3
+    assert L.gdr_gated_rmsnorm(FAKE, FAKE, None, ctypes.c_float(1e-6), 10, 64, FAKE, None) == 5
+    assert L.gdr_gated_rmsnorm(None, FAKE, None, ctypes.c_float(1e-6), 10, 128, FAKE, None) == 1
+    assert L.gdr_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(1.0), 16, 50,
+                             FAKE, FAKE, 4, None) == 5
+    assert L.gdr_decode_step(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(1.0), 16, 48,
+                             FAKE, FAKE, 4, None) == 1
+    # zero-sized work is accepted without touching the device
+    assert L.gdr_decode_step(None, None, None, None, None, None, None, ctypes.c_float(1.0), 16, 48,
+                             None, None, 0, None) == 0
+    assert L.gdr_gated_rmsnorm(None, None, None, ctypes.c_float(1e-6), 0, 128, None, None) == 0
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    import importlib
+    import gated_delta_rule_63_b200 as mod
+    saved = mod._lib
+    try:
+        mod._lib = None
+        with pytest.raises(RuntimeError):
+            mod.lib(str(tmp_path / "missing.so"))
+    finally:
+        mod._lib = saved

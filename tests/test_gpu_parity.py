@@ -1,0 +1,234 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on a B200.
+
+Tolerances of the layer: rel-L2 <= 2e-3 on bf16 outputs and <= 1e-4 on the
+fp32 final state; chunk/varlen indexing and copied conv states bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_63_b200 as G
+import gdr_inputs as GI
+from oracle import oracle as O
+from tests.helpers import (TOL_BF16, TOL_STATE, bits_f64, dev_bf16, dev_f32, dev_i32, host_bits,
+                           rel_l2, ulp_diff_bf16)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    G.lib()
+    yield
+    assert G.get_device_error() == 0
+
+
+# ---------------------------------------------------------------------------
+# helpers running the GPU path
+# ---------------------------------------------------------------------------
+
+def gpu_core(inp, h0_inplace=False):
+    """Run gdr_chunk_prefill on CoreInputs; returns (o bits, hT f32)."""
+    cu_d = dev_i32(inp.cu_seqlens)
+    N = inp.n_seqs
+    hv = inp.v.shape[1]
+    h0 = dev_f32(inp.h0) if inp.h0 is not None else None
+    if h0_inplace:
+        hT = h0
+    else:
+        hT = torch.full((N, hv, 128, 128), float("nan"), device="cuda")
+    o = G.chunk_prefill(dev_bf16(inp.q), dev_bf16(inp.k), dev_bf16(inp.v), dev_bf16(inp.a),
+                        dev_bf16(inp.b), dev_f32(inp.A_log), dev_f32(inp.dt_bias), cu_d,
+                        inp.cu_seqlens, h0=h0, hT=hT, scale=inp.scale)
+    torch.cuda.synchronize()
+    return host_bits(o), hT.cpu().numpy()
+
+
+def check_core(inp, heads=None, h0_inplace=False):
+    o_bits, hT = gpu_core(inp, h0_inplace)
+    ref_bits, _, ref_hT = O.core_path(inp, heads=heads)
+    if heads is not None:
+        o_bits = o_bits[:, heads]; ref_bits = ref_bits[:, heads]
+        hT = hT[:, heads]; ref_hT = ref_hT[:, heads]
+    eo = rel_l2(bits_f64(o_bits), bits_f64(ref_bits))
+    eh = rel_l2(hT, ref_hT)
+    assert np.all(np.isfinite(hT))
+    assert eo <= TOL_BF16, f"o rel-L2 {eo:.3e}"
+    assert eh <= TOL_STATE, f"state rel-L2 {eh:.3e}"
+    # per-sequence attribution: every sequence must be right on its own
+    cu = inp.cu_seqlens
+    for n in range(inp.n_seqs):
+        s, e = int(cu[n]), int(cu[n + 1])
+        if e > s:
+            assert rel_l2(bits_f64(o_bits[s:e]), bits_f64(ref_bits[s:e])) <= TOL_BF16
+        assert rel_l2(hT[n], ref_hT[n]) <= TOL_STATE or np.linalg.norm(ref_hT[n]) == 0
+    return eo, eh
+
+
+# ---------------------------------------------------------------------------
+# causal conv
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_conv_varlen_matches_oracle(with_state):
+    lengths = [1, 2, 0, 3, 5, 64, 100, 33]
+    inp = GI.make_full_inputs(50, lengths, conv_state_std=1.0 if with_state else None)
+    C = inp.channels
+    cu_d = dev_i32(inp.cu_seqlens)
+    cs_in = dev_bf16(inp.conv_state) if with_state else None
+    cs_out = torch.zeros((len(lengths), 3, C), dtype=torch.bfloat16, device="cuda")
+    y = G.causal_conv(dev_bf16(inp.x), dev_bf16(inp.conv_w), cu_d, inp.cu_seqlens, cs_in, cs_out)
+    torch.cuda.synchronize()
+    ref_y, ref_cs = O.causal_conv(bits_f64(inp.x), bits_f64(inp.conv_w), inp.cu_seqlens,
+                                  bits_f64(inp.conv_state) if with_state else None, round_y=True)
+    got = host_bits(y)
+    ref = O.round_bf16(ref_y)
+    assert ulp_diff_bf16(got, ref).max() <= 1       # fp32 vs fp64 before the same rounding
+    assert (got != ref).mean() < 1e-3
+    assert np.array_equal(host_bits(cs_out), O.round_bf16(ref_cs))   # raw copies: exact
+
+
+# ---------------------------------------------------------------------------
+# gated RMSNorm
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("with_w", [False, True])
+def test_gated_rmsnorm_matches_oracle(with_w):
+    r = np.random.default_rng(51)
+    rows = 1000
+    o = GI.f32_to_bf16_bits(r.standard_normal((rows, 128)).astype(np.float32) * 3)
+    z = GI.f32_to_bf16_bits(r.standard_normal((rows, 128)).astype(np.float32))
+    w = (1 + 0.1 * r.standard_normal(128)).astype(np.float32) if with_w else None
+    y = G.gated_rmsnorm(dev_bf16(o), dev_bf16(z), dev_f32(w) if with_w else None, eps=1e-6)
+    torch.cuda.synchronize()
+    ref = O.round_bf16(O.gated_rmsnorm(bits_f64(o), bits_f64(z), w, eps=1e-6))
+    got = host_bits(y)
+    assert rel_l2(bits_f64(got), bits_f64(ref)) <= TOL_BF16
+    assert ulp_diff_bf16(got, ref).max() <= 2
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+
+def run_gpu_decode(dec, steps, keep=()):
+    cs = dev_bf16(dec.conv_state)
+    st = dev_f32(dec.state)
+    cw = dev_bf16(dec.conv_w)
+    Al, db = dev_f32(dec.A_log), dev_f32(dec.dt_bias)
+    xs, as_, bs = dev_bf16(dec.x), dev_bf16(dec.a), dev_bf16(dec.b)
+    outs = {}
+    for s in range(steps):
+        o = G.decode_step(xs[s], cw, cs, as_[s], bs[s], Al, db, st, scale=dec.scale, hk=dec.hk)
+        if s in keep:
+            outs[s] = host_bits(o)
+    torch.cuda.synchronize()
+    return outs, st.cpu().numpy(), host_bits(cs)
+
+
+def test_decode_small_batch_several_steps():
+    dec = GI.make_decode_inputs(52, 3, 6)
+    outs, st, cs = run_gpu_decode(dec, 6, keep=range(6))
+    kept, H, ref_cs = O.decode_steps(dec, keep_o=tuple(range(6)))
+    for s in range(6):
+        assert rel_l2(bits_f64(outs[s]), bits_f64(kept[s])) <= TOL_BF16, s
+    assert rel_l2(st, H) <= TOL_STATE
+    assert np.array_equal(cs, O.round_bf16(ref_cs))
+
+
+def test_decode_full_batch_sampled_heads():
+    dec = GI.make_decode_inputs(53, 64, 3)
+    heads = [0, 1, 2, 25, 47]
+    outs, st, cs = run_gpu_decode(dec, 3, keep=(2,))
+    kept, H, ref_cs = O.decode_steps(dec, heads=heads, keep_o=(2,))
+    assert rel_l2(bits_f64(outs[2][:, heads]), bits_f64(kept[2][:, heads])) <= TOL_BF16
+    assert rel_l2(st[:, heads], H[:, heads]) <= TOL_STATE
+    assert np.array_equal(cs, O.round_bf16(ref_cs))
+
+
+# ---------------------------------------------------------------------------
+# chunked prefill
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("lengths", [[1], [63], [64], [65], [200], [1, 64, 65, 0, 130, 3]])
+def test_prefill_lengths_and_varlen(lengths):
+    inp = GI.make_core_inputs(60 + len(lengths), lengths, prenorm_qk=False, h0_std=0.02)
+    check_core(inp)
+
+
+def test_prefill_scale_and_zero_initial_state():
+    inp = GI.make_core_inputs(70, [150, 7], prenorm_qk=True, scale=128 ** -0.5)
+    check_core(inp)
+
+
+def test_prefill_in_place_state():
+    inp = GI.make_core_inputs(71, [90, 40], prenorm_qk=False, h0_std=0.02)
+    check_core(inp, h0_inplace=True)
+
+
+def test_prefill_key_heads_group_contiguously():
+    inp = GI.make_core_inputs(72, [70], hk=16, hv=48, prenorm_qk=False)
+    o1, _ = gpu_core(inp)
+    k2 = inp.k.copy()
+    k2[:, 1] = GI.f32_to_bf16_bits(GI.bf16_bits_to_f32(k2[:, 1]) * np.float32(-1.5) + np.float32(0.3))
+    inp.k = k2
+    o2, _ = gpu_core(inp)
+    moved = [h for h in range(48) if not np.array_equal(o1[:, h], o2[:, h])]
+    assert moved == [3, 4, 5]
+
+
+def test_prefill_workload_T128():
+    eo, eh = check_core(GI.workload_core_T128())
+    print(f"T=128: o rel-L2 {eo:.2e}, state rel-L2 {eh:.2e}")
+
+
+def test_full_path_T4096_unfused():
+    """conv -> prefill -> gated norm as three calls, against the oracle."""
+    inp = GI.workload_full_T4096()
+    cu_d = dev_i32(inp.cu_seqlens)
+    x = dev_bf16(inp.x)
+    y = G.causal_conv(x, dev_bf16(inp.conv_w), cu_d, inp.cu_seqlens)
+    T = inp.T
+    hk, hv = inp.hk, inp.hv
+    q = y[:, : hk * 128].view(T, hk, 128)            # strided views of the conv output
+    k = y[:, hk * 128: 2 * hk * 128].view(T, hk, 128)
+    v = y[:, 2 * hk * 128:].view(T, hv, 128)
+    hT = torch.empty((1, hv, 128, 128), device="cuda")
+    o = G.chunk_prefill(q, k, v, dev_bf16(inp.a), dev_bf16(inp.b), dev_f32(inp.A_log),
+                        dev_f32(inp.dt_bias), cu_d, inp.cu_seqlens, hT=hT, scale=inp.scale)
+    out = G.gated_rmsnorm(o, dev_bf16(inp.z).reshape(T, hv, 128), None, eps=inp.eps)
+    torch.cuda.synchronize()
+    ref = O.full_path(inp)
+    assert rel_l2(bits_f64(host_bits(o)), bits_f64(ref["o"])) <= TOL_BF16
+    assert rel_l2(bits_f64(host_bits(out)), bits_f64(ref["y"])) <= TOL_BF16
+    assert rel_l2(hT.cpu().numpy(), ref["hT"]) <= TOL_STATE
+
+
+def test_prefill_long_context_sampled_heads():
+    """B=1, T=262144: every head on the GPU, three heads through the oracle."""
+    inp = GI.workload_core_T262144()
+    eo, eh = check_core(inp, heads=[0, 23, 47])
+    print(f"T=262144: o rel-L2 {eo:.2e}, state rel-L2 {eh:.2e}")
+
+
+def test_prefill_varlen8_full_path_sampled_heads():
+    inp = GI.workload_full_varlen8()
+    cu_d = dev_i32(inp.cu_seqlens)
+    y = G.causal_conv(dev_bf16(inp.x), dev_bf16(inp.conv_w), cu_d, inp.cu_seqlens)
+    T, hk, hv = inp.T, inp.hk, inp.hv
+    q = y[:, : hk * 128].view(T, hk, 128)            # strided views of the conv output
+    k = y[:, hk * 128: 2 * hk * 128].view(T, hk, 128)
+    v = y[:, 2 * hk * 128:].view(T, hv, 128)
+    hT = torch.empty((inp.n_seqs, hv, 128, 128), device="cuda")
+    o = G.chunk_prefill(q, k, v, dev_bf16(inp.a), dev_bf16(inp.b), dev_f32(inp.A_log),
+                        dev_f32(inp.dt_bias), cu_d, inp.cu_seqlens, h0=dev_f32(inp.h0), hT=hT,
+                        scale=inp.scale)
+    out = G.gated_rmsnorm(o, dev_bf16(inp.z).reshape(T, hv, 128), None, eps=inp.eps)
+    torch.cuda.synchronize()
+    heads = [5, 40]
+    ref = O.full_path(inp, heads=heads)
+    got_y = host_bits(out)[:, heads]
+    assert rel_l2(bits_f64(got_y), bits_f64(ref["y"][:, heads])) <= TOL_BF16
+    assert rel_l2(hT.cpu().numpy()[:, heads], ref["hT"][:, heads]) <= TOL_STATE

@@ -30,7 +30,8 @@ _ip = ctypes.POINTER(ctypes.c_int32)
 
 class GdrError(RuntimeError):
     def __init__(self, fn: str, code: int):
-        super().__init__(f"{fn}: {status_string(code)} (status {code})")
+        detail = lib().gdr_last_error_string().decode() if code == 7 else ""
+        super().__init__(f"{fn}: {status_string(code)} (status {code})" + (f" [{detail}]" if detail else ""))
         self.code = code
 
 
@@ -55,13 +56,18 @@ def lib(path: Optional[str] = None):
     L.gdr_status_string.restype = ctypes.c_char_p
     L.gdr_status_string.argtypes = [ctypes.c_int]
     L.gdr_abi_version.restype = ctypes.c_int
+    L.gdr_last_error_string.restype = ctypes.c_char_p
+    L.gdr_last_error_string.argtypes = []
     L.gdr_prepare_chunks.argtypes = [_ip, ctypes.c_int, ctypes.c_int, _ip, _ip, _ip, ctypes.c_int,
                                      ctypes.POINTER(ctypes.c_int)]
     L.gdr_causal_conv.argtypes = [_vp, _vp, _vp, _vp, _vp, _ip, ctypes.c_int, ctypes.c_int, _vp, _vp]
     L.gdr_chunk_prefill.argtypes = [_vp, _vp, _vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp,
                                     _vp, ctypes.c_float, ctypes.c_int,
                                     ctypes.c_int, _vp, _ip, ctypes.c_int, _vp, _vp, _vp,
-                                    ctypes.POINTER(FuseArgs), _vp]
+                                    ctypes.POINTER(FuseArgs), _vp, ctypes.c_size_t, _vp]
+    L.gdr_chunk_prefill_workspace_size.restype = ctypes.c_size_t
+    L.gdr_chunk_prefill_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int]
     L.gdr_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_int,
                                   ctypes.c_int, _vp, _vp, ctypes.c_int, _vp]
     L.gdr_gated_rmsnorm.argtypes = [_vp, _vp, _vp, ctypes.c_float, ctypes.c_int64, ctypes.c_int, _vp,
@@ -161,8 +167,39 @@ def causal_conv(x, w, cu_seqlens, cu_seqlens_host, conv_state_in=None, conv_stat
     return y
 
 
+DEFAULT_WORKSPACE_BYTES = 512 << 20
+
+
+def prefill_window(cu_seqlens_host, hv: int, max_bytes: int = DEFAULT_WORKSPACE_BYTES,
+                   has_final_state: bool = True) -> int:
+    """Largest chunk window (<= the longest sequence) whose workspace fits max_bytes."""
+    cu = np.asarray(cu_seqlens_host, dtype=np.int64)
+    n = len(cu) - 1
+    if n <= 0:
+        return 1
+    max_chunks = int(max(1, ((np.diff(cu) + CHUNK - 1) // CHUNK).max()))
+    per_chunk = lib().gdr_chunk_prefill_workspace_size(n, hv, 1, 1)
+    carry = lib().gdr_chunk_prefill_workspace_size(n, hv, 1, int(has_final_state)) - per_chunk
+    fit = max(1, (max_bytes - carry) // per_chunk)
+    return int(min(max_chunks, fit))
+
+
+def prefill_workspace(cu_seqlens_host, hv: int, device, window: Optional[int] = None,
+                      has_final_state: bool = True):
+    """A torch uint8 device buffer sized for gdr_chunk_prefill."""
+    torch = _torch()
+    cu = np.asarray(cu_seqlens_host)
+    n = len(cu) - 1
+    if window is None:
+        window = prefill_window(cu_seqlens_host, hv, has_final_state=has_final_state)
+    nbytes = lib().gdr_chunk_prefill_workspace_size(max(n, 1), hv, max(int(window), 1),
+                                                    int(has_final_state))
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
 def chunk_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_host, h0=None, hT=None,
-                  o=None, scale: float = 1.0, fuse: Optional[dict] = None, stream=None):
+                  o=None, scale: float = 1.0, fuse: Optional[dict] = None, workspace=None,
+                  window: Optional[int] = None, stream=None):
     """Chunk-64 prefill.  q, k [T, hk, 128], v [T, hv, 128], a, b [T, hv] bf16.
 
     q, k, v may be token-strided views (e.g. slices of the [T, q|k|v] conv output).
@@ -187,13 +224,16 @@ def chunk_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_host, h0
     if o is None and (fuse is None or fuse.get("y") is None or fuse.get("keep_o", False)):
         T = a.shape[0]
         o = torch.empty((T, hv, HEAD_DIM), dtype=bf, device=a.device)
+    if workspace is None:
+        workspace = prefill_workspace(cu_seqlens_host, hv, a.device, window, hT is not None)
     _check("gdr_chunk_prefill", lib().gdr_chunk_prefill(
         _ptr(q, bf, "q", rows=True), _ptr(k, bf, "k", rows=True), _ptr(v, bf, "v", rows=True),
         _tok_stride(q), _tok_stride(v), _ptr(a, bf, "a"), _ptr(b, bf, "b"),
         _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"), float(scale), int(hk), int(hv),
         _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup, cu.shape[0] - 1,
         _ptr(h0, f32, "h0"), _ptr(hT, f32, "hT"), _ptr(o, bf, "o"),
-        ctypes.byref(fz) if fz is not None else None, _stream(stream)))
+        ctypes.byref(fz) if fz is not None else None, _ptr(workspace, torch.uint8, "workspace"),
+        int(workspace.numel()), _stream(stream)))
     return o
 
 

@@ -10,6 +10,7 @@
 #include "gdr_host.h"
 
 #include <atomic>
+#include <cstdio>
 
 namespace gdr {
 __device__ int g_device_error = 0;
@@ -27,6 +28,16 @@ int *device_error_ptr() {
   }
   return p;
 }
+namespace {
+thread_local char t_last_error[256] = "";
+}
+
+void set_last_error(const char *step, cudaError_t e) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%d)", step,
+           e == cudaSuccess ? "no CUDA error" : cudaGetErrorString(e), static_cast<int>(e));
+}
+void clear_last_error() { t_last_error[0] = 0; }
+const char *t_last_error_ptr() { return t_last_error; }
 }  // namespace gdr
 
 using namespace gdr;
@@ -50,6 +61,8 @@ const char *gdr_status_string(int status) {
 }
 
 int gdr_abi_version(void) { return 1; }
+
+const char *gdr_last_error_string(void) { return gdr::t_last_error_ptr(); }
 
 int gdr_prepare_chunks(const int32_t *cu, int n_seqs, int chunk, int32_t *chunk_seq,
                        int32_t *chunk_start, int32_t *chunk_len, int max_chunks, int *n_chunks) {
@@ -97,6 +110,7 @@ int gdr_get_device_error(int *error_out, void *stream) {
 int gdr_causal_conv(const void *x, const void *w, const void *conv_state_in, void *conv_state_out,
                     const int32_t *cu_dev, const int32_t *cu_host, int n_seqs, int channels, void *y,
                     void *stream) {
+  clear_last_error();
   if (!cu_host) return GDR_ERR_NULL;
   int st = check_cu_seqlens(cu_host, n_seqs);
   if (st) return st;
@@ -118,6 +132,7 @@ int gdr_causal_conv(const void *x, const void *w, const void *conv_state_in, voi
 
 int gdr_gated_rmsnorm(const void *o, const void *z, const float *w, float eps, int64_t rows, int d,
                       void *y, void *stream) {
+  clear_last_error();
   if (rows < 0) return GDR_ERR_SHAPE;
   if (d != kHeadDim) return GDR_ERR_UNSUPPORTED;
   if (rows == 0) return GDR_OK;
@@ -130,6 +145,7 @@ int gdr_gated_rmsnorm(const void *o, const void *z, const float *w, float eps, i
 int gdr_decode_step(const void *x, const void *conv_w, void *conv_state, const void *a, const void *b,
                     const float *A_log, const float *dt_bias, float scale, int hk, int hv,
                     float *state, void *o, int batch, void *stream) {
+  clear_last_error();
   int st = check_heads(hk, hv);
   if (st) return st;
   if (batch < 0) return GDR_ERR_SHAPE;
@@ -143,11 +159,18 @@ int gdr_decode_step(const void *x, const void *conv_w, void *conv_state, const v
                        static_cast<cudaStream_t>(stream));
 }
 
+size_t gdr_chunk_prefill_workspace_size(int n_seqs, int hv, int window_chunks, int has_final_state) {
+  if (n_seqs <= 0 || hv <= 0 || window_chunks <= 0) return 0;
+  return chunk_prefill_workspace_bytes(n_seqs, hv, window_chunks, has_final_state == 0);
+}
+
 int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_stride,
                       int64_t v_stride, const void *a, const void *b, const float *A_log,
                       const float *dt_bias, float scale, int hk, int hv, const int32_t *cu_dev,
                       const int32_t *cu_host, int n_seqs, const float *h0, float *hT, void *o,
-                      const gdr_prefill_fuse_t *fuse, void *stream) {
+                      const gdr_prefill_fuse_t *fuse, void *workspace, size_t workspace_bytes,
+                      void *stream) {
+  clear_last_error();
   int st = check_heads(hk, hv);
   if (st) return st;
   if (qk_stride == 0) qk_stride = static_cast<int64_t>(hk) * kHeadDim;
@@ -160,11 +183,7 @@ int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_st
   if (st) return st;
   if (n_seqs == 0) return GDR_OK;
   const int total = cu_host[n_seqs];
-  int max_len = 0;
-  for (int i = 0; i < n_seqs; ++i) {
-    const int len = cu_host[i + 1] - cu_host[i];
-    if (len > max_len) max_len = len;
-  }
+  if (total == 0 && !hT) return GDR_OK;   // nothing to compute, nothing to write
   if (!cu_dev) return GDR_ERR_NULL;
   const bool fused_conv = fuse && fuse->x;
   const bool fused_norm = fuse && fuse->z;
@@ -174,13 +193,21 @@ int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_st
     if (!q || !k || !v || !o) return GDR_ERR_NULL;
   }
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(h0) ||
-      !aligned16(hT))
+      !aligned16(hT) || !aligned16(workspace))
     return GDR_ERR_ALIGN;
+  int max_chunks = 0;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int nc = (cu_host[i + 1] - cu_host[i] + kChunk - 1) / kChunk;
+    if (nc > max_chunks) max_chunks = nc;
+  }
   const size_t state_bytes = static_cast<size_t>(n_seqs) * hv * kHeadDim * kHeadDim * 4;
   if (h0 != hT && overlaps(h0, state_bytes, hT, state_bytes)) return GDR_ERR_ALIAS;
+  if (max_chunks > 0 &&
+      (!workspace || workspace_bytes < chunk_prefill_workspace_bytes(n_seqs, hv, 1, hT == nullptr)))
+    return GDR_ERR_WORKSPACE;
   return launch_chunk_prefill(q, k, v, qk_stride, v_stride, a, b, A_log, dt_bias, scale, hk, hv,
-                              cu_dev, n_seqs, max_len,
-                              h0, hT, o, fuse, static_cast<cudaStream_t>(stream));
+                              cu_dev, n_seqs, total, max_chunks, h0, hT, o, workspace,
+                              workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -41,11 +41,19 @@ inline int check_cu_seqlens(const int32_t *cu, int n_seqs) {
 // Device address of the library's error word on the current device (cached).
 int *device_error_ptr();
 
-inline int launch_status(cudaError_t e) { return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA; }
+// Record a host-side failure (step name + CUDA error) for gdr_last_error_string.
+void set_last_error(const char *step, cudaError_t e);
+void clear_last_error();
+const char *t_last_error_ptr();
 
-inline int last_launch_status() {
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+inline int launch_status(cudaError_t e, const char *step = "kernel launch") {
+  if (e == cudaSuccess) return GDR_OK;
+  set_last_error(step, e);
+  return GDR_ERR_CUDA;
+}
+
+inline int last_launch_status(const char *step = "kernel launch") {
+  return launch_status(cudaGetLastError(), step);
 }
 
 // Launchers implemented in the kernel files (arguments already checked).
@@ -60,7 +68,9 @@ int launch_decode(const void *x, const void *conv_w, void *conv_state, const voi
 int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_stride,
                          int64_t v_stride, const void *a, const void *b,
                          const float *A_log, const float *dt_bias, float scale, int hk, int hv,
-                         const int32_t *cu_dev, int n_seqs, int max_len, const float *h0, float *hT,
-                         void *o, const gdr_prefill_fuse_t *fuse, cudaStream_t s);
+                         const int32_t *cu_dev, int n_seqs, int total, int max_chunks,
+                         const float *h0, float *hT, void *o, void *workspace, size_t ws_bytes,
+                         cudaStream_t s);
+size_t chunk_prefill_workspace_bytes(int n_seqs, int hv, int window_chunks, bool need_carry);
 
 }  // namespace gdr

@@ -9,27 +9,32 @@
 //     T    = (I + A)^-1
 //     W    = T diag(beta e^gamma) K,      Ut = T diag(beta) V
 //     U    = Ut - W H0
-//     O    = scale (diag(e^gamma) Q H0 + (Q K^T . M) U),  M_ij = e^(gamma_i - gamma_j), j <= i
+//     O    = scale (diag(e^gamma) Q H0 + Mq U),  Mq = (Q K^T) . M,  M_ij = e^(gamma_i - gamma_j), j <= i
 //     H_L  = e^gamma_L H0 + K^T diag(e^(gamma_L - gamma)) U
 // with q, k the L2-normalised rows.
 //
-// Precision plan.  The raw bf16 q, k, v rows are exact MMA operands; the
-// 1/|q|, 1/|k| factors, gates and decays are folded into fp32 row/column
-// scales of the other operand.  Every fp32 operand that feeds the state
-// (T-derived matrices, W, U, H0) is split as hi + lo bf16 and the products
-// are accumulated as hi*hi + hi*lo + lo*hi in fp32 TMEM, which keeps about
-// 16 significant bits.  The state itself never leaves fp32: thread i holds
-// row i of H (its dv slice) in registers from the first chunk to the last.
+// Two kernels.  Everything but the state products is independent of the
+// state, so it is built for every chunk at once:
+//   * prep (one CTA per chunk x value head, fully parallel): norms, gates,
+//     K K^T and Q K^T (tensor cores), A, T = (I + A)^-1 (CUDA cores),
+//     W = T' K and Ut = T'' V (tensor cores), Mq; results go to a workspace
+//     as the exact shared-memory images the chain kernel copies in;
+//   * chain (one CTA per dv slice x value head x sequence): two MMA round
+//     trips per chunk, [Q; W] H0 then K^T U' and Mq U, with the chunk's
+//     operands streamed in by TMA / bulk copies two chunks ahead.
+// Long sequences are cut into windows of chunks so that the workspace stays
+// bounded; the state crosses windows in fp32.
 //
-// Work split.  One CTA of 128 threads per (dv slice of 64 columns, value
-// head, sequence); the value head h reads key head h / (hv / hk).  Thread t
-// owns TMEM lane t; every MMA is M = 128 (cta_group::1) with fp32 TMEM
-// accumulators, operands in shared memory in the 128-byte swizzled layout.
-// The unit lower-triangular inverse runs on CUDA cores (16x16 diagonal
-// blocks by substitution, off-diagonal blocks by block products).
+// Precision.  Raw bf16 q, k, v are exact MMA operands; 1/|q|, 1/|k|, gates
+// and decays are folded into fp32 row/column scales of the other operand.
+// fp32 operands are split hi + lo bf16 and every product keeps the
+// hi*hi + hi*lo + lo*hi terms (two terms when one side is a raw input),
+// about 16 significant bits; the state itself never leaves fp32.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "gdr_common.cuh"
@@ -40,470 +45,588 @@ namespace {
 
 constexpr int C = kChunk;      // 64 tokens per chunk
 constexpr int D = kHeadDim;    // 128
-constexpr int N = 64;          // dv columns per CTA
+constexpr int N = 64;          // dv columns per chain CTA
 constexpr int NS = D / N;      // dv slices
-constexpr int kThreads = 128;
+constexpr uint32_t BLK64 = 64 * 128;     // one [64 x 64] bf16 tile, 128-B swizzled rows
 
-// ---- shared memory plan (byte offsets from a 1024-aligned base) ----------
-// OPA: A/B operand rows, two 64-column k-blocks of 256 rows x 128 B each:
-//      rows   0.. 63  W_lo      rows  64..127  W_hi
-//      rows 128..191  Q (raw)   rows 192..255  K (raw)
-constexpr uint32_t OPA_KB = 256 * 128;
-constexpr uint32_t ROW_WLO = 0, ROW_WHI = 64, ROW_Q = 128, ROW_K = 192;
-constexpr uint32_t OFF_OPA = 0;
-// TB: six [64 x 64] bf16 blocks (one 128-B row per token):
-//      0 T'_hi, 1 T'_lo, 2 T''_hi, 3 T''_lo, 4 Mq_hi, 5 Mq_lo
-//      T' = T diag(beta e^gamma / |k|), T'' = T diag(beta), Mq = (Q K^T . M) / (|q| |k|)
-constexpr uint32_t BLK64 = 64 * 128;
-constexpr uint32_t OFF_TB = OFF_OPA + 2 * OPA_KB;
-constexpr uint32_t OFF_V = OFF_TB + 6 * BLK64;        // V slice [64 tok][64 dv]
-constexpr uint32_t OFF_H = OFF_V + BLK64;             // H_hi, H_lo [128 dk][64 dv]
+// ---- workspace: one record per (sequence, value head, chunk of the window) --
+// Images are laid out exactly as the chain kernel's shared memory expects.
+constexpr uint32_t WS_W_HI = 0;          // W_hi  [kb 2][64 rows][128 B]
+constexpr uint32_t WS_W_LO = 16384;      // W_lo  [kb 2][64 rows][128 B]
+constexpr uint32_t WS_MQ_HI = 32768;     // Mq_hi [64 rows][128 B]
+constexpr uint32_t WS_MQ_LO = 40960;     // Mq_lo [64 rows][128 B]
+constexpr uint32_t WS_UT = 49152;        // Ut fp32 [slice 2][64 rows][64]
+constexpr uint32_t WS_SC = 81920;        // fp32 gamma[64], 1/|q|[64], 1/|k|[64]
+constexpr uint32_t WS_REC = 82944;       // record size (81 KiB)
+
+// ---- prep kernel -------------------------------------------------------------
+constexpr int kPrepThreads = 256;
+constexpr uint32_t P_KQ_KB = 128 * 128;              // [K rows 0..63 | Q rows 64..127] per k-block
+constexpr uint32_t P_OFF_KQ = 0;                     // 2 k-blocks
+constexpr uint32_t P_OFF_V = P_OFF_KQ + 2 * P_KQ_KB; // V [dv block 2][64 rows][128 B]
+constexpr uint32_t P_OFF_T = P_OFF_V + 2 * BLK64;    // T'_hi, T'_lo, T''_hi, T''_lo
+constexpr int LD = 65;                               // fp32 row stride of AT
+constexpr uint32_t P_OFF_AT = P_OFF_T + 4 * BLK64;   // A below / T^T on and above the diagonal
+constexpr uint32_t P_OFF_XF = P_OFF_AT + 64 * LD * 4;
+constexpr uint32_t P_OFF_SC = P_OFF_XF + 3 * 256 * 4;  // gamma, rq, rk, beta, e^gamma, block decay
+constexpr uint32_t P_OFF_BAR = P_OFF_SC + 6 * 64 * 4;
+constexpr uint32_t P_SMEM = P_OFF_BAR + 32 + 1024;
+static_assert((P_OFF_V | P_OFF_T) % 1024 == 0, "swizzled tiles need 1 KB alignment");
+constexpr uint32_t P_TM_COLS = 256;                  // two prep CTAs per SM
+constexpr uint32_t P_COL_S = 0;                      // [K K^T ; Q K^T]
+constexpr uint32_t P_COL_X = 128;                    // W, then Ut (128 cols)
+
+// ---- chain kernel ------------------------------------------------------------
+constexpr int kChainThreads = 128;
+// stage: two k-blocks of [Q 0..63 | W_hi 64..127 | W_lo 128..191 | K 192..255],
+// then Mq_hi, Mq_lo
+constexpr uint32_t C_KB = 256 * 128;
+constexpr uint32_t C_ROW_Q = 0, C_ROW_WHI = 64, C_ROW_WLO = 128, C_ROW_K = 192;
+constexpr uint32_t C_OFF_MQ = 2 * C_KB;
+constexpr uint32_t C_STAGE = C_OFF_MQ + 2 * BLK64;
 constexpr uint32_t BLK128 = 128 * 128;
-constexpr uint32_t OFF_U = OFF_H + 2 * BLK128;        // U_hi, U_lo, U'_hi, U'_lo [64 tok][64 dv]
-constexpr int LD = 65;                                // fp32 row stride of A and T
-constexpr uint32_t OFF_AF = OFF_U + 4 * BLK64;
-constexpr uint32_t OFF_TF = OFF_AF + 64 * LD * 4;
-constexpr uint32_t OFF_XF = OFF_TF + 64 * LD * 4;     // block-product scratch, 3 x 16 x 16
-constexpr uint32_t OFF_VEC = OFF_XF + 3 * 256 * 4;    // gamma, beta, 1/|k|, 1/|q|, e^gamma, decay-to-end
-constexpr uint32_t OFF_BAR = OFF_VEC + 6 * 64 * 4;
-constexpr uint32_t SMEM_USED = OFF_BAR + 16;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;    // slack for aligning the base
-static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
+constexpr uint32_t C_OFF_H = 2 * C_STAGE;            // H_hi, H_lo [128 dk][64 dv]
+constexpr uint32_t C_OFF_U = C_OFF_H + 2 * BLK128;   // U_hi, U_lo, U'_hi, U'_lo [64 tok][64 dv]
+constexpr uint32_t C_OFF_BAR = C_OFF_U + 4 * BLK64;  // full0, full1, mma
+constexpr uint32_t C_SMEM = C_OFF_BAR + 32 + 1024;
+static_assert(C_SMEM <= 232448, "chain shared memory exceeds 227 KB");
+static_assert((C_STAGE | C_OFF_H | C_OFF_U) % 1024 == 0, "swizzled tiles need 1 KB alignment");
+constexpr uint32_t C_TM_COLS = 256;
+constexpr uint32_t C_COL_P = 0;      // [Q H0 ; W_hi H0]
+constexpr uint32_t C_COL_O = 64;     // W_lo H0 (lanes 64..127), then Mq U (lanes 0..63)
+constexpr uint32_t C_COL_H = 128;    // K^T U' (lanes = dk)
 
-// ---- TMEM columns (fp32, lane = row) ---------------------------------------
-constexpr uint32_t TM_COLS = 512;
-constexpr uint32_t COL_S = 0;      // [Q K^T ; K K^T]           64 cols
-constexpr uint32_t COL_W = 64;     // W (rows 0..63)            128 cols
-constexpr uint32_t COL_P = 192;    // [W_hi H ; Q H]            64
-constexpr uint32_t COL_P2 = 256;   // W_lo H_hi (rows 0..63)    64
-constexpr uint32_t COL_UT = 320;   // Ut (rows 0..63)           64
-constexpr uint32_t COL_H = 384;    // K^T U' (rows = dk)        64
-constexpr uint32_t COL_O = 448;    // Mq U (rows 64..127)       64
+#ifdef GDR_PREFILL_TIMING
+// diagnostic build: step timestamps; prep CTA (0,0,0) in row 0, chain CTA
+// (0,0,0) chunk c in row 1 + c (16 slots per row)
+__device__ long long *g_prefill_times;
+#define PTIME(row, step)                                                   \
+  do {                                                                     \
+    if (g_prefill_times && threadIdx.x == 0 && blockIdx.x == 0 &&          \
+        blockIdx.y == 0 && blockIdx.z == 0 && (row) < 64)                  \
+      g_prefill_times[(row) * 16 + (step)] = clock64();                    \
+  } while (0)
+#else
+#define PTIME(row, step) \
+  do {                   \
+  } while (0)
+#endif
 
 struct PrefillParams {
-  const uint16_t *q, *k, *v, *a, *b;
+  const uint16_t *a, *b;
   const float *A_log, *dt_bias;
   float scale;
   int hk, hv, group;
-  int64_t qk_stride, v_stride;   // elements between consecutive tokens
   const int32_t *cu;
-  const float *h0;
-  float *hT;
+  uint8_t *ws;          // workspace records
+  int win0;             // first chunk (per sequence) of this window
+  int win_chunks;       // chunks per window (record stride)
+  const float *state_in;
+  float *state_out;
   uint16_t *o;
   int *err;
-#ifdef GDR_PREFILL_DEBUG
-  float *dbg;   // diagnostic dump of the first chunk of CTA (0, 0, 0)
-#endif
 };
 
-#ifdef GDR_PREFILL_DEBUG
-float *g_dump = nullptr;
-#endif
-
-__device__ __forceinline__ void st_shared16(uint32_t addr, const uint4 &v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
-               "r"(v.w)
-               : "memory");
+// 8 fp32 values -> hi/lo bf16 16-byte chunks at two addresses (shared or global)
+__device__ __forceinline__ void st_split8_shared(uint32_t hi_addr, uint32_t lo_addr, const float *v8) {
+  uint4 hi, lo;
+  split8(v8, hi, lo);
+  st_shared16(hi_addr, hi);
+  st_shared16(lo_addr, lo);
 }
-__device__ __forceinline__ uint4 ld_shared16(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
+__device__ __forceinline__ void st_split8_global(uint8_t *hi_p, uint8_t *lo_p, const float *v8) {
+  uint4 hi, lo;
+  split8(v8, hi, lo);
+  *reinterpret_cast<uint4 *>(hi_p) = hi;
+  *reinterpret_cast<uint4 *>(lo_p) = lo;
 }
 
-// write 64 fp32 values as the hi/lo bf16 row `r` of two 128B-swizzled tiles
-__device__ __forceinline__ void write_row_split(uint32_t hi_base, uint32_t lo_base, uint32_t r,
-                                                const float *vals) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 hi, lo;
-    split8(vals + 8 * c, hi, lo);
-    st_shared16(hi_base + sw128(r, c), hi);
-    st_shared16(lo_base + sw128(r, c), lo);
-  }
-}
-
-// one thread waits for the MMA barrier phase, the CTA agrees on the outcome
-__device__ __forceinline__ bool cta_wait_mma(uint32_t bar, uint32_t &phase, int *err) {
+// one thread waits (bounded), the CTA agrees on the outcome
+__device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity, int *err) {
   bool ok = true;
-  if (threadIdx.x == 0) ok = mbar_wait(bar, phase, err);
-  phase ^= 1u;
+  if (threadIdx.x == 0) ok = mbar_wait(bar, parity, err);
   ok = __syncthreads_and(ok) != 0;
   tc_fence_after();
   return ok;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillParams p) {
+__device__ __forceinline__ uint8_t *ws_record(const PrefillParams &p, int n, int h, int cw) {
+  return p.ws + ((static_cast<size_t>(n) * p.hv + h) * p.win_chunks + cw) * WS_REC;
+}
+
+// =============================================================================
+// prep: one chunk of one value head
+// =============================================================================
+__global__ void __launch_bounds__(kPrepThreads, 2)
+prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+            const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
+  const int cw = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+  const int seq_start = p.cu[n], seq_end = p.cu[n + 1];
+  const int t0 = seq_start + (p.win0 + cw) * C;
+  if (t0 >= seq_end) return;   // the window runs past this sequence (uniform exit)
+  const int L = min(C, seq_end - t0);
+
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
   uint8_t *smem = smem_raw + (sbase - raw_addr);
-
-  const int slice = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kh = h / p.group;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int seq_start = p.cu[n], seq_end = p.cu[n + 1];
-
-  float *s_gam = reinterpret_cast<float *>(smem + OFF_VEC);
-  float *s_beta = s_gam + 64;
-  float *s_rk = s_gam + 128;
-  float *s_rq = s_gam + 192;
-  float *s_eg = s_gam + 256;     // e^gamma_j
-  float *s_ed = s_gam + 320;     // e^(gamma_L - gamma_j) / |k_j|
-  float *AF = reinterpret_cast<float *>(smem + OFF_AF);
-  float *TF = reinterpret_cast<float *>(smem + OFF_TF);
-  float *XF = reinterpret_cast<float *>(smem + OFF_XF);
-  const uint32_t bar = sbase + OFF_BAR;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8);
+  float *AT = reinterpret_cast<float *>(smem + P_OFF_AT);
+  float *XF = reinterpret_cast<float *>(smem + P_OFF_XF);
+  float *s_g = reinterpret_cast<float *>(smem + P_OFF_SC);
+  float *s_rq = s_g + 64, *s_rk = s_g + 128, *s_beta = s_g + 192, *s_eg = s_g + 256, *s_eb = s_g + 320;
+  const uint32_t bar_tma = sbase + P_OFF_BAR, bar_mma = sbase + P_OFF_BAR + 8;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + P_OFF_BAR + 16);
+  uint8_t *rec = ws_record(p, n, h, cw);
 
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_holder), TM_COLS);
+    tmem_alloc(smem_u32(tmem_holder), P_TM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(bar, 1);
+    mbar_init(bar_tma, 1);
+    mbar_init(bar_mma, 1);
     fence_mbar_init();
+    mbar_arrive_expect_tx(bar_tma, 6 * BLK64);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      tma_load_2d(sbase + P_OFF_KQ + kb * P_KQ_KB, &tm_k, kh * D + kb * 64, t0, bar_tma);
+      tma_load_2d(sbase + P_OFF_KQ + kb * P_KQ_KB + 64 * 128, &tm_q, kh * D + kb * 64, t0, bar_tma);
+      tma_load_2d(sbase + P_OFF_V + kb * BLK64, &tm_v, h * D + kb * 64, t0, bar_tma);
+    }
+  }
+  // gates of the chunk's rows; padding rows get no decay and no write
+  float g = 0.0f;
+  if (tid < 64) {
+    float beta = 0.0f;
+    if (tid < L) {
+      const size_t ab = static_cast<size_t>(t0 + tid) * p.hv + h;
+      g = -expf(p.A_log[h]) * softplus_f(bf_bits2f(p.a[ab]) + p.dt_bias[h]);
+      beta = sigmoid_f(bf_bits2f(p.b[ab]));
+    }
+    s_beta[tid] = beta;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);   // this warp's lane quarter
-  uint32_t phase = 0;
+  PTIME(0, 0);
+  bool ok = cta_wait(bar_tma, 0, p.err);
+  PTIME(0, 1);
 
-  // ---- the state: thread tid holds row tid (dk index) of its dv slice ----
+  if (ok && L < C) {   // rows past the sequence end hold other tokens: zero them
+    const uint32_t nz = static_cast<uint32_t>(C - L) * 16;   // rows x 16-B chunks per tile
+    for (uint32_t e = tid; e < 3 * nz; e += kPrepThreads) {
+      const uint32_t tile = e / nz, rem = e % nz, r = L + rem / 16, cc = rem % 16;
+      const uint32_t base = tile == 2 ? P_OFF_V + (cc >> 3) * BLK64
+                                      : P_OFF_KQ + (cc >> 3) * P_KQ_KB + tile * 64 * 128;
+      st_shared16(sbase + base + sw128(r, cc & 7), make_uint4(0, 0, 0, 0));
+    }
+    __syncthreads();
+  }
+  if (ok) {
+    // 1/|k| (rows 0..63 of the KQ tile) and 1/|q| (rows 64..127), two threads per row
+    const int row = tid >> 1, part = tid & 1;
+    float ss = 0.0f;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+      const int c16 = part * 8 + cc;
+      float f[8];
+      unpack8(ld_shared16(sbase + P_OFF_KQ + (c16 >> 3) * P_KQ_KB + sw128(row, c16 & 7)), f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    if (part == 0) (row < 64 ? s_rk : s_rq)[row & 63] = 1.0f / sqrtf(ss + 1e-6f);
+    // inclusive scan of g over the chunk (threads 0..63)
+    float run = g;
+    if (tid < 64) {
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float up = __shfl_up_sync(0xffffffffu, run, off);
+        if (lane >= off) run += up;
+      }
+      if (tid == 31) XF[0] = run;
+    }
+    __syncthreads();
+    if (tid < 64) s_g[tid] = run + (tid >= 32 ? XF[0] : 0.0f);
+    __syncthreads();
+    if (tid < 64) {
+      s_eg[tid] = __expf(s_g[tid]);
+      s_eb[tid] = __expf(s_g[tid | 15] - s_g[tid]);   // decay to the end of the 16-block
+      float *sc = reinterpret_cast<float *>(rec + WS_SC);
+      sc[tid] = s_g[tid];
+      sc[64 + tid] = s_rq[tid];
+      sc[128 + tid] = s_rk[tid];
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+
+    PTIME(0, 2);
+    // ---- [K; Q] K^T ------------------------------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t koff = (kk >> 2) * P_KQ_KB + (kk & 3) * 32;
+        mma_bf16(tmem + P_COL_S, sdesc(sbase + P_OFF_KQ + koff, 16, 1024),
+                 sdesc(sbase + P_OFF_KQ + koff, 16, 1024), id, kk > 0);
+      }
+      mma_commit(bar_mma);
+    }
+    ok = cta_wait(bar_mma, 0, p.err);
+  }
+  if (ok) {
+    PTIME(0, 3);
+    // ---- A (rows 0..63) and Mq (rows 64..127): 2 threads per row, 32 columns each
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int row = 32 * q4 + lane;
+    float sv[32];
+    tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + P_COL_S + 32 * hf, sv);
+    tmem_wait_ld();
+    const int i = row & 63, ib = i >> 4;
+    const float gi = s_g[i];
+    if (row < 64) {
+      const float bi = s_beta[i] * s_rk[i];
+#pragma unroll
+      for (int b2 = 0; b2 < 2; ++b2) {
+        const int blk = 2 * hf + b2;
+        const float fi = __expf(gi - s_g[blk * 16 + 15]);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int j = blk * 16 + e;
+          const float dec = blk < ib ? fi * s_eb[j] : __expf(fminf(gi - s_g[j], 0.0f));
+          if (j < i) AT[i * LD + j] = bi * s_rk[j] * sv[b2 * 16 + e] * dec;
+        }
+      }
+    } else {
+      const float qi = s_rq[i];
+#pragma unroll
+      for (int b2 = 0; b2 < 2; ++b2) {
+        const int blk = 2 * hf + b2;
+        const float fi = __expf(gi - s_g[blk * 16 + 15]);
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          float m[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int j = blk * 16 + h8 * 8 + e;
+            const float dec = blk < ib ? fi * s_eb[j] : (j <= i ? __expf(gi - s_g[j]) : 0.0f);
+            m[e] = sv[b2 * 16 + h8 * 8 + e] * qi * s_rk[j] * dec;
+          }
+          const uint32_t off = sw128(i, blk * 2 + h8);
+          st_split8_global(rec + WS_MQ_HI + off, rec + WS_MQ_LO + off, m);
+        }
+      }
+    }
+    __syncthreads();
+
+    PTIME(0, 4);
+    // ---- T = (I + A)^-1, stored transposed on and above the diagonal ----------
+    if (tid < 64) {   // diagonal 16x16 blocks, one column per thread
+      const int bb = tid >> 4, cc = tid & 15;
+      float x[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        float sacc = (r == cc) ? 1.0f : 0.0f;
+#pragma unroll
+        for (int j = 0; j < r; ++j) sacc -= AT[(16 * bb + r) * LD + 16 * bb + j] * x[j];
+        x[r] = sacc;
+      }
+#pragma unroll
+      for (int r = 0; r < 16; ++r)
+        if (r >= cc) AT[(16 * bb + cc) * LD + 16 * bb + r] = x[r];
+    }
+    __syncthreads();
+    for (int d = 1; d < 4; ++d) {   // T_bc = -T_bb sum_{m=c}^{b-1} A_bm T_mc, b - c = d
+      const int nb = 4 - d;
+      for (int e = tid; e < nb * 256; e += kPrepThreads) {
+        const int blk = e >> 8, bb = d + blk, cb = bb - d, r = (e >> 4) & 15, j = e & 15;
+        float sacc = 0.0f;
+        for (int m = cb; m < bb; ++m) {
+#pragma unroll
+          for (int l = 0; l < 16; ++l) {
+            const float t = (m > cb || l >= j) ? AT[(16 * cb + j) * LD + 16 * m + l] : 0.0f;
+            sacc += AT[(16 * bb + r) * LD + 16 * m + l] * t;
+          }
+        }
+        XF[e] = sacc;
+      }
+      __syncthreads();
+      for (int e = tid; e < nb * 256; e += kPrepThreads) {
+        const int blk = e >> 8, bb = d + blk, cb = bb - d, r = (e >> 4) & 15, j = e & 15;
+        float sacc = 0.0f;
+#pragma unroll
+        for (int l = 0; l < 16; ++l)
+          if (l <= r) sacc -= AT[(16 * bb + l) * LD + 16 * bb + r] * XF[(blk << 8) + l * 16 + j];
+        AT[(16 * cb + j) * LD + 16 * bb + r] = sacc;
+      }
+      __syncthreads();
+    }
+
+    PTIME(0, 5);
+    // ---- T' = T diag(beta e^g / |k|), T'' = T diag(beta), hi/lo tiles --------
+    {
+      const int r = tid >> 2, qc = tid & 3;   // row r, columns 16 qc .. 16 qc + 15
+#pragma unroll
+      for (int h8 = 0; h8 < 2; ++h8) {
+        float t1[8], t2[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int j = 16 * qc + 8 * h8 + e;
+          const float tij = (j <= r) ? AT[j * LD + r] : 0.0f;
+          t2[e] = tij * s_beta[j];
+          t1[e] = t2[e] * s_eg[j] * s_rk[j];
+        }
+        const uint32_t off = sw128(r, 2 * qc + h8);
+        st_split8_shared(sbase + P_OFF_T + off, sbase + P_OFF_T + BLK64 + off, t1);
+        st_split8_shared(sbase + P_OFF_T + 2 * BLK64 + off, sbase + P_OFF_T + 3 * BLK64 + off, t2);
+      }
+    }
+    fence_proxy_async();
+    __syncthreads();
+
+    PTIME(0, 6);
+    // ---- W = T' K  (A rows 64..127 are junk; only lanes 0..63 are read) -------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + P_COL_X, sdesc(sbase + P_OFF_T + part * BLK64 + kk * 32, 16, 1024),
+                   sdesc(sbase + P_OFF_KQ + kk * 2048, P_KQ_KB, 1024), id, (part | kk) != 0);
+      mma_commit(bar_mma);
+    }
+    ok = cta_wait(bar_mma, 1, p.err);
+  }
+  if (ok) {
+    PTIME(0, 7);
+    if ((warp & 2) == 0) {   // warps 0, 1, 4, 5 own lanes 0..63; k-block = warp >> 2
+      const int kb = warp >> 2, r = 32 * (warp & 1) + lane;
+      const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + P_COL_X + 64 * kb;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float w[32];
+        tmem_ld32(tl + 32 * hh, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const uint32_t off = kb * BLK64 + sw128(r, 4 * hh + c4);
+          st_split8_global(rec + WS_W_HI + off, rec + WS_W_LO + off, w + 8 * c4);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    PTIME(0, 8);
+    // ---- Ut = T'' V (N = 128) ---------------------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + P_COL_X, sdesc(sbase + P_OFF_T + (2 + part) * BLK64 + kk * 32, 16, 1024),
+                   sdesc(sbase + P_OFF_V + kk * 2048, BLK64, 1024), id, (part | kk) != 0);
+      mma_commit(bar_mma);
+    }
+    ok = cta_wait(bar_mma, 0, p.err);
+  }
+  PTIME(0, 9);
+  if (ok && (warp & 2) == 0) {   // Ut rows -> fp32 [slice][row][64]
+    const int sl = warp >> 2, r = 32 * (warp & 1) + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + P_COL_X + 64 * sl;
+    float4 *dst = reinterpret_cast<float4 *>(rec + WS_UT + (static_cast<size_t>(sl) * 64 + r) * 256);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float u[32];
+      tmem_ld32(tl + 32 * hh, u);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4)
+        dst[8 * hh + c4] = make_float4(u[4 * c4], u[4 * c4 + 1], u[4 * c4 + 2], u[4 * c4 + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  PTIME(0, 10);
+  if (warp == 0) tmem_dealloc(tmem, P_TM_COLS);
+}
+
+// =============================================================================
+// chain: the state of one dv slice of one value head through one window
+// =============================================================================
+__global__ void __launch_bounds__(kChainThreads, 1)
+chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+             PrefillParams p) {
+  const int slice = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+  const int seq_start = p.cu[n], seq_end = p.cu[n + 1];
+  const int n_all = (seq_end - seq_start + C - 1) / C;
+  const int c_end = min(n_all, p.win0 + p.win_chunks);
+  const int nw = max(0, c_end - p.win0);              // chunks of this window
+  if (nw == 0 && p.win0 > 0) return;                  // state already final
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (sbase - raw_addr);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int kh = h / p.group;
+  const uint32_t bar_full = sbase + C_OFF_BAR, bar_mma = sbase + C_OFF_BAR + 16;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 24);
+
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_holder), C_TM_COLS);
+    tmem_relinquish();
+  }
+  // chunk cw of the window into stage cw & 1
+  auto load_chunk = [&](int cw) {
+    const uint32_t st = sbase + (cw & 1) * C_STAGE;
+    const uint32_t fb = bar_full + 8 * (cw & 1);
+    const int t0 = seq_start + (p.win0 + cw) * C;
+    const uint8_t *rec = ws_record(p, n, h, cw);
+    mbar_arrive_expect_tx(fb, 10 * BLK64);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      tma_load_2d(st + kb * C_KB + C_ROW_Q * 128, &tm_q, kh * D + kb * 64, t0, fb);
+      tma_load_2d(st + kb * C_KB + C_ROW_K * 128, &tm_k, kh * D + kb * 64, t0, fb);
+      bulk_load(st + kb * C_KB + C_ROW_WHI * 128, rec + WS_W_HI + kb * BLK64, BLK64, fb);
+      bulk_load(st + kb * C_KB + C_ROW_WLO * 128, rec + WS_W_LO + kb * BLK64, BLK64, fb);
+    }
+    bulk_load(st + C_OFF_MQ, rec + WS_MQ_HI, BLK64, fb);
+    bulk_load(st + C_OFF_MQ + BLK64, rec + WS_MQ_LO, BLK64, fb);
+  };
+  if (tid == 0) {
+    mbar_init(bar_full, 1);
+    mbar_init(bar_full + 8, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    for (int cw = 0; cw < 2 && cw < nw; ++cw) load_chunk(cw);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+
+  // ---- the state: thread tid holds row tid (dk) of this dv slice ---------------
   float hreg[N];
   const size_t srow = (static_cast<size_t>(n) * p.hv + h) * D * D + static_cast<size_t>(tid) * D + slice * N;
-  if (p.h0) {
+  if (p.state_in) {
 #pragma unroll
     for (int j = 0; j < N; j += 4) {
-      const float4 v4 = *reinterpret_cast<const float4 *>(p.h0 + srow + j);
+      const float4 v4 = *reinterpret_cast<const float4 *>(p.state_in + srow + j);
       hreg[j] = v4.x; hreg[j + 1] = v4.y; hreg[j + 2] = v4.z; hreg[j + 3] = v4.w;
     }
   } else {
 #pragma unroll
     for (int j = 0; j < N; ++j) hreg[j] = 0.0f;
   }
-  write_row_split(sbase + OFF_H, sbase + OFF_H + BLK128, tid, hreg);
+  auto write_h = [&]() {
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc)
+      st_split8_shared(sbase + C_OFF_H + sw128(tid, cc), sbase + C_OFF_H + BLK128 + sw128(tid, cc), hreg + 8 * cc);
+  };
+  write_h();
+  fence_proxy_async();
+  __syncthreads();
 
-  const float A_h = expf(p.A_log[h]);
-  const float dtb = p.dt_bias[h];
+  const bool wrow = tid >= 64;   // lanes 64..127 hold W H0, lanes 0..63 hold Q H0
+  const int r = tid & 63;
+  uint32_t mma_phase = 0;
   bool ok = true;
-#ifdef GDR_PREFILL_DEBUG
-  bool dump = p.dbg && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
-#endif
-
-  for (int t0 = seq_start; t0 < seq_end && ok; t0 += C) {
+  for (int cw = 0; cw < nw && ok; ++cw) {
+    const int s = cw & 1;
+    const uint32_t st = sbase + s * C_STAGE;
+    const int t0 = seq_start + (p.win0 + cw) * C;
     const int L = min(C, seq_end - t0);
-
-    // ---- S0: raw q, k rows (key head kh), v slice, gates -------------------
-    for (int idx = tid; idx < 64 * 16; idx += kThreads) {
-      const int r = idx >> 4, c = idx & 15;
-      const bool valid = r < L;
-      const size_t tok = static_cast<size_t>(t0 + (valid ? r : 0));
-      const uint32_t kb = static_cast<uint32_t>(c >> 3) * OPA_KB;
-      cp_async16(sbase + OFF_OPA + kb + sw128(ROW_Q + r, c & 7),
-                 p.q + tok * p.qk_stride + kh * D + c * 8, valid ? 16u : 0u);
-      cp_async16(sbase + OFF_OPA + kb + sw128(ROW_K + r, c & 7),
-                 p.k + tok * p.qk_stride + kh * D + c * 8, valid ? 16u : 0u);
-    }
-    for (int idx = tid; idx < 64 * 8; idx += kThreads) {
-      const int r = idx >> 3, c = idx & 7;
-      const bool valid = r < L;
-      const size_t tok = static_cast<size_t>(t0 + (valid ? r : 0));
-      cp_async16(sbase + OFF_V + sw128(r, c), p.v + tok * p.v_stride + h * D + slice * N + c * 8,
-                 valid ? 16u : 0u);
-    }
-    cp_async_commit();
-    if (tid < 64) {
-      float g = 0.0f, beta = 0.0f;   // padding rows: no decay, no write
-      if (tid < L) {
-        const size_t ab = static_cast<size_t>(t0 + tid) * p.hv + h;
-        g = -A_h * softplus_f(bf_bits2f(p.a[ab]) + dtb);
-        beta = sigmoid_f(bf_bits2f(p.b[ab]));
+    const uint8_t *rec = ws_record(p, n, h, cw);
+    const float *sc = reinterpret_cast<const float *>(rec + WS_SC);
+    // this thread's Ut row (W lanes) and per-row scalars, fetched ahead of the MMA
+    float ut[N];
+    float scal_a, scal_b;
+    if (wrow) {
+      const float4 *src = reinterpret_cast<const float4 *>(rec + WS_UT + (static_cast<size_t>(slice) * 64 + r) * 256);
+#pragma unroll
+      for (int j = 0; j < N / 4; ++j) {
+        const float4 v4 = src[j];
+        ut[4 * j] = v4.x; ut[4 * j + 1] = v4.y; ut[4 * j + 2] = v4.z; ut[4 * j + 3] = v4.w;
       }
-      s_gam[tid] = g;
-      s_beta[tid] = beta;
+      scal_a = sc[r];          // gamma_r
+      scal_b = sc[128 + r];    // 1/|k_r|
+    } else {
+      scal_a = sc[r];          // gamma_r
+      scal_b = sc[64 + r];     // 1/|q_r|
     }
-    cp_async_wait_all();
-    fence_proxy_async();
-    __syncthreads();
+    const float gL = sc[63];   // padding rows carry gamma_{L-1}
+    PTIME(1 + cw, 0);
+    if (!(ok = cta_wait(bar_full + 8 * s, (cw >> 1) & 1, p.err))) break;
+    PTIME(1 + cw, 1);
 
-    // ---- S1: cumulative gates, 1/|q|, 1/|k| --------------------------------
+    // ---- [Q; W_hi] (H_hi + H_lo) and [*; W_lo] H_hi ---------------------------------
     if (tid == 0) {
-      float run = 0.0f;
-      for (int i = 0; i < 64; ++i) { run += s_gam[i]; s_gam[i] = run; }
-    }
-    {
-      const int r = tid & 63;
-      const uint32_t row = (tid < 64 ? ROW_Q : ROW_K) + r;
-      float ss = 0.0f;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float f[8];
-        unpack8(ld_shared16(sbase + OFF_OPA + (c >> 3) * OPA_KB + sw128(row, c & 7)), f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
-      }
-      (tid < 64 ? s_rq : s_rk)[r] = 1.0f / sqrtf(ss + 1e-6f);
-    }
-    __syncthreads();
-    if (tid < 64) {
-      s_eg[tid] = expf(s_gam[tid]);
-      s_ed[tid] = expf(s_gam[63] - s_gam[tid]) * s_rk[tid];
-    }
-
-    // ---- S2: [Q; K] K^T on the tensor cores --------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t koff = (kk >> 2) * OPA_KB + (kk & 3) * 32;
-        mma_bf16(tmem + COL_S, sdesc(sbase + OFF_OPA + koff + ROW_Q * 128, 16, 1024),
-                 sdesc(sbase + OFF_OPA + koff + ROW_K * 128, 16, 1024), id, kk > 0);
-      }
-      mma_commit(bar);
-    }
-    ok = cta_wait_mma(bar, phase, p.err);
-    if (!ok) break;
-
-    // ---- S3: A (fp32) and the masked, decayed, normalised Q K^T ------------
-    {
-      float sv[64];
-      tmem_ld32(tl + COL_S, sv);
-      tmem_ld32(tl + COL_S + 32, sv + 32);
-      tmem_wait_ld();
-      if (tid < 64) {   // row i of Q K^T
-        const int i = tid;
-        const float gi = s_gam[i], sq = s_rq[i];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float m[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int j = 8 * c + e;
-            m[e] = (j <= i) ? sv[j] * sq * s_rk[j] * expf(gi - s_gam[j]) : 0.0f;
-          }
-          uint4 hi, lo;
-          split8(m, hi, lo);
-          st_shared16(sbase + OFF_TB + 4 * BLK64 + sw128(i, c), hi);
-          st_shared16(sbase + OFF_TB + 5 * BLK64 + sw128(i, c), lo);
-        }
-      } else {          // row i of K K^T
-        const int i = tid - 64;
-        const float gi = s_gam[i], bi = s_beta[i] * s_rk[i];
-#pragma unroll
-        for (int j = 0; j < 64; ++j)
-          AF[i * LD + j] = (j < i) ? bi * s_rk[j] * sv[j] * expf(gi - s_gam[j]) : 0.0f;
-      }
-    }
-#ifdef GDR_PREFILL_DEBUG
-    if (dump && t0 == seq_start) {
-      float sv[64];
-      tmem_ld32(tl + COL_S, sv);
-      tmem_ld32(tl + COL_S + 32, sv + 32);
-      tmem_wait_ld();
-      for (int j = 0; j < 64; ++j) p.dbg[tid * 64 + j] = sv[j];
-    }
-#endif
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- S4: T = (I + A)^-1 ------------------------------------------------
-    if (tid < 64) {   // diagonal 16x16 blocks, one column per thread
-      const int bb = tid >> 4, c = tid & 15;
-      float x[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float s = (i == c) ? 1.0f : 0.0f;
-#pragma unroll
-        for (int j = 0; j < i; ++j) s -= AF[(16 * bb + i) * LD + 16 * bb + j] * x[j];
-        x[i] = s;
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) TF[(16 * bb + i) * LD + 16 * bb + c] = x[i];
-    }
-    __syncthreads();
-    for (int d = 1; d < 4; ++d) {   // block diagonal d: T_bc = -T_bb sum_{m=c}^{b-1} A_bm T_mc
-      const int nb = 4 - d;
-      for (int e = tid; e < nb * 256; e += kThreads) {
-        const int blk = e >> 8, bb = d + blk, c = bb - d, i = (e >> 4) & 15, j = e & 15;
-        float s = 0.0f;
-        for (int m = c; m < bb; ++m)
-#pragma unroll
-          for (int l = 0; l < 16; ++l) s += AF[(16 * bb + i) * LD + 16 * m + l] * TF[(16 * m + l) * LD + 16 * c + j];
-        XF[e] = s;
-      }
-      __syncthreads();
-      for (int e = tid; e < nb * 256; e += kThreads) {
-        const int blk = e >> 8, bb = d + blk, c = bb - d, i = (e >> 4) & 15, j = e & 15;
-        float s = 0.0f;
-#pragma unroll
-        for (int l = 0; l < 16; ++l)
-          if (l <= i) s -= TF[(16 * bb + i) * LD + 16 * bb + l] * XF[(blk << 8) + l * 16 + j];
-        TF[(16 * bb + i) * LD + 16 * c + j] = s;
-      }
-      __syncthreads();
-    }
-
-    // ---- S5: T' = T diag(beta e^gamma / |k|), T'' = T diag(beta), hi/lo ----
-    {
-      const int i = tid & 63, half = tid >> 6;
-#pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        const int c = half * 4 + cb;
-        float t1[8], t2[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int j = 8 * c + e;
-          const float tij = (j <= i) ? TF[i * LD + j] : 0.0f;
-          t2[e] = tij * s_beta[j];
-          t1[e] = t2[e] * s_eg[j] * s_rk[j];
-        }
-        uint4 hi, lo;
-        split8(t1, hi, lo);
-        st_shared16(sbase + OFF_TB + 0 * BLK64 + sw128(i, c), hi);
-        st_shared16(sbase + OFF_TB + 1 * BLK64 + sw128(i, c), lo);
-        split8(t2, hi, lo);
-        st_shared16(sbase + OFF_TB + 2 * BLK64 + sw128(i, c), hi);
-        st_shared16(sbase + OFF_TB + 3 * BLK64 + sw128(i, c), lo);
-      }
-    }
-#ifdef GDR_PREFILL_DEBUG
-    if (dump && t0 == seq_start) {
-      for (int e = tid; e < 64 * 64; e += kThreads) {
-        p.dbg[8192 + e] = AF[(e >> 6) * LD + (e & 63)];
-        p.dbg[8192 + 4096 + e] = ((e & 63) <= (e >> 6)) ? TF[(e >> 6) * LD + (e & 63)] : 0.0f;
-      }
-    }
-#endif
-    fence_proxy_async();
-    __syncthreads();
-
-    // ---- S6: W = T' K and Ut = T'' V -----------------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t idW = idesc_bf16(128, 128, false, true);
-      const uint32_t idU = idesc_bf16(128, 64, false, true);
-#pragma unroll
-      for (int part = 0; part < 2; ++part)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + COL_W, sdesc(sbase + OFF_TB + part * BLK64 + kk * 32, 16, 1024),
-                   sdesc(sbase + OFF_OPA + ROW_K * 128 + kk * 2048, OPA_KB, 1024), idW,
-                   (part | kk) != 0);
-#pragma unroll
-      for (int part = 0; part < 2; ++part)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + COL_UT, sdesc(sbase + OFF_TB + (2 + part) * BLK64 + kk * 32, 16, 1024),
-                   sdesc(sbase + OFF_V + kk * 2048, BLK64, 1024), idU, (part | kk) != 0);
-      mma_commit(bar);
-    }
-    ok = cta_wait_mma(bar, phase, p.err);
-    if (!ok) break;
-
-    // ---- S7: W -> hi/lo operand rows -----------------------------------------
-    if (tid < 64) {
-#pragma unroll
-      for (int kb = 0; kb < 2; ++kb) {
-        float w[64];
-        tmem_ld32(tl + COL_W + kb * 64, w);
-        tmem_ld32(tl + COL_W + kb * 64 + 32, w + 32);
-        tmem_wait_ld();
-        write_row_split(sbase + OFF_OPA + kb * OPA_KB + ROW_WHI * 128,
-                        sbase + OFF_OPA + kb * OPA_KB + ROW_WLO * 128, tid, w);
-#ifdef GDR_PREFILL_DEBUG
-        if (dump && t0 == seq_start)
-          for (int j = 0; j < 64; ++j) p.dbg[16384 + tid * 128 + kb * 64 + j] = w[j];
-#endif
-      }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- S8: [W; Q] H0 (hi/lo) -------------------------------------------------
-    if (tid == 0) {
-      tc_fence_after();
       const uint32_t id = idesc_bf16(128, 64, false, true);
 #pragma unroll
       for (int part = 0; part < 3; ++part) {
-        // part 0: [W_hi; Q] H_hi   part 1: [W_hi; Q] H_lo   part 2: [W_lo; *] H_hi
-        const uint32_t arow = part < 2 ? ROW_WHI : ROW_WLO;
-        const uint32_t hb = part == 1 ? OFF_H + BLK128 : OFF_H;
-        const uint32_t dcol = part < 2 ? COL_P : COL_P2;
+        const uint32_t arow = part < 2 ? C_ROW_Q : C_ROW_WHI;   // part 2: lanes 64..127 get W_lo rows
+        const uint32_t hb = part == 1 ? C_OFF_H + BLK128 : C_OFF_H;
+        const uint32_t dcol = part < 2 ? C_COL_P : C_COL_O;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * OPA_KB + (kk & 3) * 32;
-          mma_bf16(tmem + dcol, sdesc(sbase + OFF_OPA + koff + arow * 128, 16, 1024),
-                   sdesc(sbase + hb + kk * 2048, BLK128, 1024), id, (part == 1 || kk > 0));
+          const uint32_t koff = (kk >> 2) * C_KB + (kk & 3) * 32;
+          mma_bf16(tmem + dcol, sdesc(st + koff + arow * 128, 16, 1024),
+                   sdesc(sbase + hb + kk * 2048, BLK128, 1024), id, (part == 1) || kk > 0);
         }
       }
-      mma_commit(bar);
+      mma_commit(bar_mma);
     }
-    ok = cta_wait_mma(bar, phase, p.err);
-    if (!ok) break;
+    if (!(ok = cta_wait(bar_mma, mma_phase, p.err))) break;
+    mma_phase ^= 1u;
 
-    // ---- S9: U = Ut - W H0 and its scaled copy; O_inter --------------------
+    PTIME(1 + cw, 2);
+    // ---- U = Ut - W H0 and U' = U e^(gL - g) / |k| (W lanes); Q H0 part of o ----
     float oreg[N];
-    if (tid < 64) {
-      const int t = tid;
-      const float ed = s_ed[t];
+    if (wrow) {
+      const float ed = __expf(gL - scal_a) * scal_b;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float ut[32], pw[32], pl[32];
-        tmem_ld32(tl + COL_UT + half * 32, ut);
-        tmem_ld32(tl + COL_P + half * 32, pw);
-        tmem_ld32(tl + COL_P2 + half * 32, pl);
+      for (int hh = 0; hh < 2; ++hh) {
+        float pw[32], pl[32];
+        tmem_ld32(tl + C_COL_P + 32 * hh, pw);
+        tmem_ld32(tl + C_COL_O + 32 * hh, pl);
         tmem_wait_ld();
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int c4 = 0; c4 < 4; ++c4) {
           float u[8], us[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            u[e] = ut[cb * 8 + e] - pw[cb * 8 + e] - pl[cb * 8 + e];
+            u[e] = ut[32 * hh + 8 * c4 + e] - pw[8 * c4 + e] - pl[8 * c4 + e];
             us[e] = u[e] * ed;
           }
-          const int c = half * 4 + cb;
-          uint4 hi, lo;
-          split8(u, hi, lo);
-          st_shared16(sbase + OFF_U + 0 * BLK64 + sw128(t, c), hi);
-          st_shared16(sbase + OFF_U + 1 * BLK64 + sw128(t, c), lo);
-          split8(us, hi, lo);
-          st_shared16(sbase + OFF_U + 2 * BLK64 + sw128(t, c), hi);
-          st_shared16(sbase + OFF_U + 3 * BLK64 + sw128(t, c), lo);
+          const uint32_t off = sw128(r, 4 * hh + c4);
+          st_split8_shared(sbase + C_OFF_U + off, sbase + C_OFF_U + BLK64 + off, u);
+          st_split8_shared(sbase + C_OFF_U + 2 * BLK64 + off, sbase + C_OFF_U + 3 * BLK64 + off, us);
         }
       }
     } else {
-      const int i = tid - 64;
-      const float f = p.scale * s_eg[i] * s_rq[i];
-      tmem_ld32(tl + COL_P, oreg);
-      tmem_ld32(tl + COL_P + 32, oreg + 32);
+      const float f = p.scale * __expf(scal_a) * scal_b;
+      tmem_ld32(tl + C_COL_P, oreg);
+      tmem_ld32(tl + C_COL_P + 32, oreg + 32);
       tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < N; ++j) oreg[j] *= f;
     }
-#ifdef GDR_PREFILL_DEBUG
-    if (dump && t0 == seq_start) {
-      float tmp[64];
-      const uint32_t cols[4] = {COL_UT, COL_P, COL_P2, 0};
-      for (int q4 = 0; q4 < 3; ++q4) {
-        tmem_ld32(tl + cols[q4], tmp);
-        tmem_ld32(tl + cols[q4] + 32, tmp + 32);
-        tmem_wait_ld();
-        for (int j = 0; j < 64; ++j) p.dbg[32768 + q4 * 8192 + tid * 64 + j] = tmp[j];
-      }
-    }
-#endif
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
 
-    // ---- S10: K^T U' (hi/lo) and Mq U (hi/lo) ----------------------------------
+    PTIME(1 + cw, 3);
+    // ---- K^T U' (hi/lo) -> H part;  Mq U (hi/lo x hi/lo) -> o part -------------
     if (tid == 0) {
       tc_fence_after();
       const uint32_t idH = idesc_bf16(128, 64, true, true);
@@ -512,106 +635,161 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillParam
       for (int part = 0; part < 2; ++part)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + COL_H, sdesc(sbase + OFF_OPA + ROW_K * 128 + kk * 2048, OPA_KB, 1024),
-                   sdesc(sbase + OFF_U + (2 + part) * BLK64 + kk * 2048, BLK64, 1024), idH,
+          mma_bf16(tmem + C_COL_H, sdesc(st + C_ROW_K * 128 + kk * 2048, C_KB, 1024),
+                   sdesc(sbase + C_OFF_U + (2 + part) * BLK64 + kk * 2048, BLK64, 1024), idH,
                    (part | kk) != 0);
 #pragma unroll
-      for (int part = 0; part < 3; ++part) {
-        // rows 64..127 of the A tile are Mq: start one block earlier
-        const uint32_t ablk = part < 2 ? 3 : 4;       // Mq_hi, Mq_hi, Mq_lo
-        const uint32_t ub = part == 1 ? 1 : 0;        // U_hi, U_lo, U_hi
+      for (int part = 0; part < 3; ++part) {   // Mq rows land in lanes 0..63
+        const uint32_t aoff = part < 2 ? 0u : BLK64;      // Mq_hi, Mq_hi, Mq_lo
+        const uint32_t ub = part == 1 ? BLK64 : 0u;       // U_hi, U_lo, U_hi
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + COL_O, sdesc(sbase + OFF_TB + ablk * BLK64 + kk * 32, 16, 1024),
-                   sdesc(sbase + OFF_U + ub * BLK64 + kk * 2048, BLK64, 1024), idO,
-                   (part | kk) != 0);
+          mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + aoff + kk * 32, 16, 1024),
+                   sdesc(sbase + C_OFF_U + ub + kk * 2048, BLK64, 1024), idO, (part | kk) != 0);
       }
-      mma_commit(bar);
+      mma_commit(bar_mma);
     }
-    ok = cta_wait_mma(bar, phase, p.err);
-    if (!ok) break;
+    if (!(ok = cta_wait(bar_mma, mma_phase, p.err))) break;
+    mma_phase ^= 1u;
+    if (tid == 0 && cw + 2 < nw) load_chunk(cw + 2);   // stage s is free again
 
-    // ---- S11: state update, output -------------------------------------------
+    PTIME(1 + cw, 4);
+    // ---- H <- e^gamma_L H + K^T U'; o = Q H0 part + Mq U --------------------------
     {
-      const float eL = s_eg[63];   // padding rows carry gamma_{L-1}
+      const float eL = __expf(gL);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int hh = 0; hh < 2; ++hh) {
         float rh[32];
-        tmem_ld32(tl + COL_H + half * 32, rh);
+        tmem_ld32(tl + C_COL_H + 32 * hh, rh);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) hreg[half * 32 + j] = eL * hreg[half * 32 + j] + rh[j];
+        for (int j = 0; j < 32; ++j) hreg[32 * hh + j] = eL * hreg[32 * hh + j] + rh[j];
       }
-      write_row_split(sbase + OFF_H, sbase + OFF_H + BLK128, tid, hreg);
-      if (tid >= 64) {
-        const int t = tid - 64;
+      write_h();
+      if (!wrow) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int hh = 0; hh < 2; ++hh) {
           float ro[32];
-          tmem_ld32(tl + COL_O + half * 32, ro);
+          tmem_ld32(tl + C_COL_O + 32 * hh, ro);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) oreg[half * 32 + j] += p.scale * ro[j];
+          for (int j = 0; j < 32; ++j) oreg[32 * hh + j] += p.scale * ro[j];
         }
-        if (t < L) {
-          uint16_t *dst = p.o + (static_cast<size_t>(t0 + t) * p.hv + h) * D + slice * N;
+        if (r < L) {
+          uint16_t *dst = p.o + (static_cast<size_t>(t0 + r) * p.hv + h) * D + slice * N;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(dst + 8 * c) = pack8(oreg + 8 * c);
+          for (int cc = 0; cc < 8; ++cc) *reinterpret_cast<uint4 *>(dst + 8 * cc) = pack8(oreg + 8 * cc);
         }
       }
-#ifdef GDR_PREFILL_DEBUG
-      if (dump && t0 == seq_start) {
-        float tmp[64];
-        const uint32_t cols[2] = {COL_H, COL_O};
-        for (int q2 = 0; q2 < 2; ++q2) {
-          tmem_ld32(tl + cols[q2], tmp);
-          tmem_ld32(tl + cols[q2] + 32, tmp + 32);
-          tmem_wait_ld();
-          for (int j = 0; j < 64; ++j) p.dbg[57344 + q2 * 8192 + tid * 64 + j] = tmp[j];
-        }
-      }
-#endif
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
+    PTIME(1 + cw, 5);
   }
-
-  if (p.hT && ok) {
+  if (p.state_out && ok) {
 #pragma unroll
     for (int j = 0; j < N; j += 4)
-      *reinterpret_cast<float4 *>(p.hT + srow + j) = make_float4(hreg[j], hreg[j + 1], hreg[j + 2], hreg[j + 3]);
+      *reinterpret_cast<float4 *>(p.state_out + srow + j) = make_float4(hreg[j], hreg[j + 1], hreg[j + 2], hreg[j + 3]);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+  if (warp == 0) tmem_dealloc(tmem, C_TM_COLS);
+}
+
+// ---- host side ---------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (!f) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !ptr)
+      return nullptr;
+    f = reinterpret_cast<EncodeTiledFn>(ptr);
+    fn.store(f, std::memory_order_release);
+  }
+  return f;
+}
+
+// [rows][cols] bf16 with a row stride in elements; 64 x 64 boxes, 128B swizzle;
+// rows past `rows` read as zero
+bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t row_stride) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// per-device one-time opt-in to large dynamic shared memory
+int ensure_smem_attrs() {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return launch_status(e, "prefill: cudaGetDevice");
+  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return GDR_OK;
+  e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
+  if (e != cudaSuccess) return launch_status(e, "prefill: shared memory opt-in");
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return GDR_OK;
 }
 
 }  // namespace
 
+size_t chunk_prefill_workspace_bytes(int n_seqs, int hv, int window_chunks, bool need_carry) {
+  size_t b = static_cast<size_t>(n_seqs) * hv * window_chunks * WS_REC;
+  if (need_carry) b += static_cast<size_t>(n_seqs) * hv * D * D * sizeof(float);
+  return b;
+}
+
 int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_stride,
                          int64_t v_stride, const void *a, const void *b,
                          const float *A_log, const float *dt_bias, float scale, int hk, int hv,
-                         const int32_t *cu_dev, int n_seqs, int max_len, const float *h0, float *hT,
-                         void *o, const gdr_prefill_fuse_t *fuse, cudaStream_t s) {
-  (void)max_len;
-  (void)fuse;
+                         const int32_t *cu_dev, int n_seqs, int total, int max_chunks,
+                         const float *h0, float *hT, void *o, void *workspace, size_t ws_bytes,
+                         cudaStream_t s) {
   if (n_seqs > 65535 || hv > 65535) return GDR_ERR_SHAPE;
-  // the shared-memory opt-in is a per-device function attribute
-  static std::atomic<uint64_t> attr_set{0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GDR_ERR_CUDA;
-  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
-  if (!bit || !(attr_set.load(std::memory_order_acquire) & bit)) {
-    if (cudaFuncSetAttribute(chunk_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return GDR_ERR_CUDA;
-    attr_set.fetch_or(bit, std::memory_order_acq_rel);
-  }
+  int st = ensure_smem_attrs();
+  if (st) return st;
+  // window: as many chunks as the workspace holds (the state crosses windows
+  // in hT, or in the workspace tail when the caller wants no final state)
+  const bool carry_in_ws = hT == nullptr;
+  const size_t rec_per_chunk = static_cast<size_t>(n_seqs) * hv * WS_REC;
+  const size_t carry = carry_in_ws ? chunk_prefill_workspace_bytes(n_seqs, hv, 0, true) : 0;
+  if (max_chunks > 0 && (!workspace || ws_bytes < carry + rec_per_chunk)) return GDR_ERR_WORKSPACE;
+  int win = 1;
+  if (max_chunks > 0)
+    win = static_cast<int>(std::min<size_t>((ws_bytes - carry) / rec_per_chunk, static_cast<size_t>(max_chunks)));
+  if (win > 65535) win = 65535;
+  float *carry_buf = carry_in_ws && max_chunks > 0
+                         ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + rec_per_chunk * win)
+                         : nullptr;
+  CUtensorMap tq, tk, tv;
+  const uint64_t rows = total > 0 ? static_cast<uint64_t>(total) : 1;
+  // with no tokens no tile is ever loaded; any aligned device address serves as a base
+  const void *any = v ? v : (hT ? static_cast<const void *>(hT) : static_cast<const void *>(h0));
+  if (!any) return GDR_OK;
+  if (!encode_fn()) return launch_status(cudaErrorSymbolNotFound, "prefill: cuTensorMapEncodeTiled lookup");
+  if (!make_map(&tq, q ? q : any, static_cast<uint64_t>(hk) * D, rows, static_cast<uint64_t>(qk_stride)) ||
+      !make_map(&tk, k ? k : any, static_cast<uint64_t>(hk) * D, rows, static_cast<uint64_t>(qk_stride)) ||
+      !make_map(&tv, v ? v : any, static_cast<uint64_t>(hv) * D, rows, static_cast<uint64_t>(v_stride)))
+    return launch_status(cudaErrorInvalidValue, "prefill: tensor map encoding");
+
   PrefillParams p;
-  p.q = static_cast<const uint16_t *>(q);
-  p.k = static_cast<const uint16_t *>(k);
-  p.v = static_cast<const uint16_t *>(v);
   p.a = static_cast<const uint16_t *>(a);
   p.b = static_cast<const uint16_t *>(b);
   p.A_log = A_log;
@@ -620,23 +798,34 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   p.hk = hk;
   p.hv = hv;
   p.group = hv / hk;
-  p.qk_stride = qk_stride;
-  p.v_stride = v_stride;
   p.cu = cu_dev;
-  p.h0 = h0;
-  p.hT = hT;
+  p.ws = static_cast<uint8_t *>(workspace);
+  p.win_chunks = win;
   p.o = static_cast<uint16_t *>(o);
   p.err = device_error_ptr();
-#ifdef GDR_PREFILL_DEBUG
-  p.dbg = g_dump;
-#endif
-  dim3 grid(NS, hv, n_seqs);
-  chunk_prefill_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(p);
-  return last_launch_status();
+  const int n_windows = max_chunks > 0 ? (max_chunks + win - 1) / win : 1;
+  for (int w = 0; w < n_windows; ++w) {
+    p.win0 = w * win;
+    const bool first = w == 0, last = w == n_windows - 1;
+    p.state_in = first ? h0 : (carry_in_ws ? carry_buf : hT);
+    p.state_out = last ? hT : (carry_in_ws ? carry_buf : hT);
+    const int nc = std::min(win, max_chunks - p.win0);
+    if (nc > 0) {
+      prep_kernel<<<dim3(nc, hv, n_seqs), kPrepThreads, P_SMEM, s>>>(tq, tk, tv, p);
+      st = last_launch_status("prefill: prep kernel launch");
+      if (st) return st;
+    }
+    chain_kernel<<<dim3(NS, hv, n_seqs), kChainThreads, C_SMEM, s>>>(tq, tk, p);
+    st = last_launch_status("prefill: chain kernel launch");
+    if (st) return st;
+  }
+  return GDR_OK;
 }
 
 }  // namespace gdr
 
-#ifdef GDR_PREFILL_DEBUG
-extern "C" GDR_API void gdr_debug_set_prefill_dump(float *dev_ptr) { gdr::g_dump = dev_ptr; }
+#ifdef GDR_PREFILL_TIMING
+extern "C" GDR_API int gdr_debug_set_prefill_times(long long *dev_ptr) {
+  return cudaMemcpyToSymbol(gdr::g_prefill_times, &dev_ptr, sizeof(dev_ptr)) == cudaSuccess ? 0 : 7;
+}
 #endif

@@ -148,6 +148,10 @@ typedef struct gdr_prefill_fuse {
  *             (in place), must not overlap it otherwise.
  *   o:        bf16 [T][hv][128]; may be NULL only when fuse->y is set.
  *   fuse:     NULL, or conv / gated-norm fusion (see gdr_prefill_fuse_t).
+ *   workspace, workspace_bytes: device scratch, 16-byte aligned, at least
+ *             gdr_chunk_prefill_workspace_size(n_seqs, hv, 1, hT != NULL)
+ *             bytes (GDR_ERR_WORKSPACE otherwise); the window is the largest
+ *             number of chunks that fits.
  * Empty sequences copy h0 (or zeros) to hT.
  */
 GDR_API int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_token_stride,
@@ -155,7 +159,22 @@ GDR_API int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64
                               const float *A_log, const float *dt_bias, float scale, int hk, int hv,
                               const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
                               int n_seqs, const float *h0, float *hT, void *o,
-                              const gdr_prefill_fuse_t *fuse, void *stream);
+                              const gdr_prefill_fuse_t *fuse, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+/*
+ * Bytes of device workspace gdr_chunk_prefill needs to build the
+ * state-independent operands of `window_chunks` chunks of every sequence at a
+ * time (81 KiB per sequence, value head and chunk), plus room to carry the
+ * state between windows when hT is NULL (has_final_state == 0).  Any
+ * window_chunks >= 1 is valid; a window of ceil(max sequence length / 64)
+ * chunks processes everything in one pass, smaller windows use less memory
+ * and more kernel launches.  The workspace is caller-owned scratch: its
+ * contents need no initialisation and are meaningless after the call, and
+ * two calls in flight at the same time must not share it.
+ */
+GDR_API size_t gdr_chunk_prefill_workspace_size(int n_seqs, int hv, int window_chunks,
+                                                int has_final_state);
 
 /*
  * gdr_decode_step -- one token for each of `batch` independent sequences
@@ -189,6 +208,13 @@ GDR_API int gdr_decode_step(const void *x, const void *conv_w, void *conv_state,
  */
 GDR_API int gdr_gated_rmsnorm(const void *o, const void *z, const float *w, float eps, int64_t rows, int d,
                       void *y, void *stream);
+
+/*
+ * Text of the last host-side failure of a call made from this thread: which
+ * step failed and the CUDA error string (empty when the last call succeeded).
+ * The pointer stays valid until the next call from the same thread.
+ */
+GDR_API const char *gdr_last_error_string(void);
 
 /*
  * Read and clear the device-side error word (0 = none, else a gdr_status_t

@@ -84,14 +84,15 @@ def _cu(lengths):
 def test_prefill_rejects_bad_arguments_on_host(L):
     cu, cup = _cu([10, 5])
     args = dict(q=FAKE, k=FAKE, v=FAKE, qs=0, vs=0, a=FAKE, b=FAKE, A_log=FAKE, dt_bias=FAKE, scale=1.0, hk=16,
-                hv=48, cu_dev=FAKE, cu_host=cup, n=2, h0=None, hT=FAKE, o=FAKE, fuse=None, s=None)
+                hv=48, cu_dev=FAKE, cu_host=cup, n=2, h0=None, hT=FAKE, o=FAKE, fuse=None, ws=FAKE,
+                wsb=1 << 30, s=None)
 
     def call(**kw):
         a = dict(args); a.update(kw)
         return L.gdr_chunk_prefill(a["q"], a["k"], a["v"], a["qs"], a["vs"], a["a"], a["b"],
                                    a["A_log"], a["dt_bias"],
                                    a["scale"], a["hk"], a["hv"], a["cu_dev"], a["cu_host"], a["n"],
-                                   a["h0"], a["hT"], a["o"], a["fuse"], a["s"])
+                                   a["h0"], a["hT"], a["o"], a["fuse"], a["ws"], a["wsb"], a["s"])
     assert call(hk=16, hv=40) == 5          # grouping not integral
     assert call(hk=1, hv=48) == 5           # group of 48 > 8
     assert call(hk=0) == 2
@@ -105,6 +106,18 @@ def test_prefill_rejects_bad_arguments_on_host(L):
     assert call(h0=FAKE + 64, hT=FAKE) == 9  # partial overlap of h0 and hT
     assert call(qs=16 * 128 - 8) == 2          # token stride shorter than a row
     assert call(vs=48 * 128 + 4) == 3          # token stride not a multiple of 8
+    assert call(ws=None) == 6                  # no workspace
+    assert call(wsb=1000) == 6                 # too small for one chunk window
+    assert call(ws=FAKE + 8) == 3
+
+
+def test_prefill_workspace_size(L):
+    L.gdr_chunk_prefill_workspace_size.restype = ctypes.c_size_t
+    one = L.gdr_chunk_prefill_workspace_size(2, 48, 1, 1)
+    assert one == 2 * 48 * 82944
+    assert L.gdr_chunk_prefill_workspace_size(2, 48, 5, 1) == 5 * one
+    assert L.gdr_chunk_prefill_workspace_size(2, 48, 5, 0) == 5 * one + 2 * 48 * 128 * 128 * 4
+    assert L.gdr_chunk_prefill_workspace_size(0, 48, 5, 1) == 0
 
 
 def test_other_entry_points_reject_bad_arguments(L):

@@ -16,6 +16,7 @@ import numpy as np
 
 __all__ = [
     "GdrError", "lib", "status_string", "prepare_chunks", "causal_conv", "chunk_prefill",
+    "chunk_prefill_noalloc", "prefill_workspace", "prefill_window",
     "decode_step", "gated_rmsnorm", "get_device_error", "HEAD_DIM", "CHUNK",
 ]
 
@@ -65,6 +66,12 @@ def lib(path: Optional[str] = None):
                                     _vp, ctypes.c_float, ctypes.c_int,
                                     ctypes.c_int, _vp, _ip, ctypes.c_int, _vp, _vp, _vp,
                                     ctypes.POINTER(FuseArgs), _vp, ctypes.c_size_t, _vp]
+    L.gdr_chunk_prefill_noalloc.argtypes = [_vp, _vp, _vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp,
+                                            _vp, _vp, ctypes.c_float, ctypes.c_int, ctypes.c_int,
+                                            _vp, _ip, ctypes.c_int, _vp, _vp, _vp, _vp]
+    L.gdr_chunk_prefill_noalloc.restype = ctypes.c_int
+    L.gdr_chunk_prefill_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    L.gdr_chunk_prefill_noalloc_scratch_bytes.argtypes = []
     L.gdr_chunk_prefill_workspace_size.restype = ctypes.c_size_t
     L.gdr_chunk_prefill_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int]
@@ -234,6 +241,28 @@ def chunk_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_host, h0
         _ptr(h0, f32, "h0"), _ptr(hT, f32, "hT"), _ptr(o, bf, "o"),
         ctypes.byref(fz) if fz is not None else None, _ptr(workspace, torch.uint8, "workspace"),
         int(workspace.numel()), _stream(stream)))
+    return o
+
+
+def chunk_prefill_noalloc(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_host, h0=None,
+                          hT=None, o=None, scale: float = 1.0, stream=None):
+    """gdr_chunk_prefill on the library's own scratch array (no workspace argument).
+
+    For callers that cannot allocate device memory; see gdr_chunk_prefill_noalloc
+    in include/gdr.h for the size limit and the rule that calls must not overlap.
+    """
+    torch = _torch()
+    bf, f32 = torch.bfloat16, torch.float32
+    cu, cup = _host_cu(cu_seqlens_host)
+    hv = a.shape[1]
+    if o is None:
+        o = torch.empty((a.shape[0], hv, HEAD_DIM), dtype=bf, device=a.device)
+    _check("gdr_chunk_prefill_noalloc", lib().gdr_chunk_prefill_noalloc(
+        _ptr(q, bf, "q", rows=True), _ptr(k, bf, "k", rows=True), _ptr(v, bf, "v", rows=True),
+        _tok_stride(q), _tok_stride(v), _ptr(a, bf, "a"), _ptr(b, bf, "b"),
+        _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"), float(scale), int(q.shape[1]),
+        int(hv), _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup, cu.shape[0] - 1,
+        _ptr(h0, f32, "h0"), _ptr(hT, f32, "hT"), _ptr(o, bf, "o"), _stream(stream)))
     return o
 
 

@@ -177,6 +177,43 @@ GDR_API size_t gdr_chunk_prefill_workspace_size(int n_seqs, int hv, int window_c
                                                 int has_final_state);
 
 /*
+ * gdr_chunk_prefill_noalloc -- gdr_chunk_prefill without a caller workspace.
+ * (No counterpart in the pages that describe the layer: this is an interface
+ * convenience of this library.)
+ * For callers that cannot allocate device memory: a plugin whose host
+ * framework owns all device memory and hands out no scratch buffers, a
+ * fixed-budget deployment that must not grow at run time, or code running
+ * where CUDA API calls such as cudaMalloc are not allowed.  The kernels run on
+ * a 32 MiB scratch array that is part of the library itself; every GPU that
+ * loads the library holds it until the process exits.  Arguments and results
+ * are those of gdr_chunk_prefill (no fusion).  The call allocates nothing.
+ *  - The scratch holds a window of at least one chunk for every sequence:
+ *    gdr_chunk_prefill_workspace_size(n_seqs, hv, 1, hT != NULL) must not
+ *    exceed gdr_chunk_prefill_noalloc_scratch_bytes(), otherwise the call
+ *    returns GDR_ERR_WORKSPACE and launches nothing (for 48 value heads:
+ *    up to 8 sequences with hT given).  Longer sequences are processed in
+ *    more windows, i.e. more kernel launches.
+ *  - The first call on a device looks up the scratch's device address with
+ *    cudaGetSymbolAddress (once per device, with that device current); make
+ *    that first call before any stream capture.
+ *  - All calls share the one scratch array, which keeps whatever the last
+ *    call left in it (no call relies on its contents: every part is written
+ *    before it is read).  Calls whose work overlaps on the GPU -- on two
+ *    streams, or from two threads -- race on the scratch and corrupt each
+ *    other's results: serialise them.
+ */
+GDR_API int gdr_chunk_prefill_noalloc(const void *q, const void *k, const void *v,
+                                      int64_t qk_token_stride, int64_t v_token_stride,
+                                      const void *a, const void *b, const float *A_log,
+                                      const float *dt_bias, float scale, int hk, int hv,
+                                      const int32_t *cu_seqlens_dev,
+                                      const int32_t *cu_seqlens_host, int n_seqs,
+                                      const float *h0, float *hT, void *o, void *stream);
+
+/* Size in bytes of the scratch array gdr_chunk_prefill_noalloc runs on. */
+GDR_API size_t gdr_chunk_prefill_noalloc_scratch_bytes(void);
+
+/*
  * gdr_decode_step -- one token for each of `batch` independent sequences
  * ("33B 只做 18 层 ...", §1.2: the single-step recurrent call taken when one
  * new token resumes from the cached state; "33B 只做 18 层 ..." (mhpq.cn)

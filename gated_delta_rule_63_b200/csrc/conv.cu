@@ -5,10 +5,11 @@
 // SiLU(sum_j w[c][j] x[t-3+j][c]), fp32 math, bf16 output; inputs before a
 // sequence start come from the conv state (oldest first) or are zero.
 //
-// Memory-bound: each thread owns 8 adjacent channels (one 16-byte vector) and
-// walks a run of kTokens tokens with a 3-deep sliding window in registers, so
-// x is read once (plus a 3-token halo per run) and y written once, both with
-// coalesced 16-byte accesses.
+// Memory-bound: each thread owns 8 adjacent channels (one 16-byte vector) of
+// a run of kTokens tokens; the run's rows and its 3-row halo are loaded up
+// front so that all its loads are in flight together.  x is read once (plus
+// the halo, mostly from L2) and y written once, with coalesced 16-byte
+// accesses.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -19,7 +20,7 @@ namespace gdr {
 namespace {
 
 constexpr int kThreads = 128;   // threads per block; 8 channels each
-constexpr int kTokens = 32;     // tokens per run
+constexpr int kTokens = 8;      // tokens per run
 
 struct ConvParams {
   const uint16_t *x;
@@ -43,28 +44,15 @@ __device__ int seq_of(const int32_t *cu, int n_seqs, int t) {
   return lo;
 }
 
-__device__ __forceinline__ void load8(const uint16_t *p, float *f) {
-  unpack8(*reinterpret_cast<const uint4 *>(p), f);
-}
-
+// Each thread: 8 channels x kTokens tokens.  All kTokens + 3 input rows are
+// loaded up front (independent 16-byte loads in flight), then each output
+// takes its taps from the rows of its own sequence, from the conv state or
+// zero before the sequence start.
 __global__ void __launch_bounds__(kThreads) causal_conv_kernel(ConvParams p) {
   const int C = p.channels;
   const int c0 = (blockIdx.x * kThreads + threadIdx.x) * 8;   // first channel of this thread
   if (c0 >= C) return;
   const int t_begin = blockIdx.y * kTokens;
-
-  float w[4][8];
-  {
-    // w is [C][4]: channels c0..c0+7 occupy 32 contiguous bf16
-    const uint4 *wp = reinterpret_cast<const uint4 *>(p.w + static_cast<size_t>(c0) * 4);
-    float tmp[32];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) unpack8(__ldg(wp + i), tmp + 8 * i);
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) w[j][ch] = tmp[ch * 4 + j];
-  }
 
   // empty sequences: their conv state passes through unchanged (run once)
   if (blockIdx.y == 0 && p.cs_out) {
@@ -80,57 +68,70 @@ __global__ void __launch_bounds__(kThreads) causal_conv_kernel(ConvParams p) {
   if (t_begin >= p.total) return;
   const int t_end = min(t_begin + kTokens, p.total);
 
-  int n = seq_of(p.cu, p.n_seqs, t_begin);
-  int seq_start = __ldg(p.cu + n);
-  int seq_end = __ldg(p.cu + n + 1);
-
-  // window: win[0] = x[t-3], win[1] = x[t-2], win[2] = x[t-1]
-  float win[3][8];
-  auto fill_window = [&](int t) {
+  uint4 raw[kTokens + 3];   // rows t_begin - 3 .. t_begin + kTokens - 1
 #pragma unroll
-    for (int s = 0; s < 3; ++s) {
-      const int pos = t - 3 + s;
+  for (int i = 0; i < kTokens + 3; ++i) {
+    const int pos = t_begin - 3 + i;
+    raw[i] = (pos >= 0 && pos < t_end) ? __ldg(reinterpret_cast<const uint4 *>(p.x + static_cast<size_t>(pos) * C + c0))
+                                       : make_uint4(0, 0, 0, 0);
+  }
+  float w[4][8];
+  {
+    // w is [C][4]: channels c0..c0+7 occupy 32 contiguous bf16
+    const uint4 *wp = reinterpret_cast<const uint4 *>(p.w + static_cast<size_t>(c0) * 4);
+    float tmp[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) unpack8(__ldg(wp + i), tmp + 8 * i);
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) w[j][ch] = tmp[ch * 4 + j];
+  }
+  int n = seq_of(p.cu, p.n_seqs, t_begin);
+  int seq_start = __ldg(p.cu + n), seq_end = __ldg(p.cu + n + 1);
+
+#pragma unroll
+  for (int i = 0; i < kTokens; ++i) {
+    const int t = t_begin + i;
+    if (t >= t_end) break;
+    while (t >= seq_end) {   // next non-empty sequence
+      ++n;
+      seq_start = __ldg(p.cu + n);
+      seq_end = __ldg(p.cu + n + 1);
+    }
+    float acc[8];
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) acc[ch] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int pos = t - 3 + j;
+      float xv[8];
       if (pos >= seq_start) {
-        load8(p.x + static_cast<size_t>(pos) * C + c0, win[s]);
-      } else if (p.cs_in) {
-        const int back = seq_start - pos;   // 1..3 positions before the start
-        load8(p.cs_in + (static_cast<size_t>(n) * 3 + (3 - back)) * C + c0, win[s]);
+        unpack8(raw[i + j], xv);
+      } else if (p.cs_in) {   // before the sequence start: the conv state, oldest first
+        const int slot = 3 - (seq_start - pos);   // 1..3 positions before the start
+        unpack8(*reinterpret_cast<const uint4 *>(p.cs_in + (static_cast<size_t>(n) * 3 + slot) * C + c0), xv);
       } else {
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) win[s][ch] = 0.0f;
+        for (int ch = 0; ch < 8; ++ch) xv[ch] = 0.0f;
       }
-    }
-  };
-  fill_window(t_begin);
-
-  for (int t = t_begin; t < t_end; ++t) {
-    if (t >= seq_end) {   // crossed into the next non-empty sequence
-      do {
-        ++n;
-        seq_start = __ldg(p.cu + n);
-        seq_end = __ldg(p.cu + n + 1);
-      } while (seq_end <= t);
-      fill_window(t);
-    }
-    float xt[8], out[8];
-    load8(p.x + static_cast<size_t>(t) * C + c0, xt);
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      const float acc = w[0][ch] * win[0][ch] + w[1][ch] * win[1][ch] + w[2][ch] * win[2][ch] +
-                        w[3][ch] * xt[ch];
-      out[ch] = silu_f(acc);
+      for (int ch = 0; ch < 8; ++ch) acc[ch] += w[j][ch] * xv[ch];
     }
+    float out[8];
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) out[ch] = silu_f(acc[ch]);
     *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(t) * C + c0) = pack8(out);
+    if (t == seq_end - 1 && p.cs_out) {   // last token: the last three inputs are the new conv state
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      win[0][ch] = win[1][ch];
-      win[1][ch] = win[2][ch];
-      win[2][ch] = xt[ch];
-    }
-    if (t == seq_end - 1 && p.cs_out) {   // last token: the window is the new conv state
-#pragma unroll
-      for (int s = 0; s < 3; ++s)
-        *reinterpret_cast<uint4 *>(p.cs_out + (static_cast<size_t>(n) * 3 + s) * C + c0) = pack8(win[s]);
+      for (int s = 0; s < 3; ++s) {
+        const int pos = t - 2 + s;
+        uint4 v;
+        if (pos >= seq_start) v = raw[i + 1 + s];
+        else if (p.cs_in) v = *reinterpret_cast<const uint4 *>(p.cs_in + (static_cast<size_t>(n) * 3 + (3 - (seq_start - pos))) * C + c0);
+        else v = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(p.cs_out + (static_cast<size_t>(n) * 3 + s) * C + c0) = v;
+      }
     }
   }
 }

@@ -307,3 +307,50 @@ __device__ __forceinline__ uint4 ld_shared16(uint32_t addr) {
 }
 
 }  // namespace gdr
+
+namespace gdr {
+
+// hi = bf16(x) and lo = bf16(x - hi) for 8 values, with packed bf16x2 conversions
+__device__ __forceinline__ void split8x2(const float *f, uint4 &hi, uint4 &lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 hb = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    const __nv_bfloat162 lb =
+        __floats2bfloat162_rn(f[2 * i] - __low2float(hb), f[2 * i + 1] - __high2float(hb));
+    h[i] = *reinterpret_cast<const uint32_t *>(&hb);
+    l[i] = *reinterpret_cast<const uint32_t *>(&lb);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// 8 fp32 -> 8 bf16 (round to nearest even), packed bf16x2
+__device__ __forceinline__ uint4 pack8x2(const float *f) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t *>(&b);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+}  // namespace gdr
+
+namespace gdr {
+
+// 1D bulk copy shared -> global (16-byte aligned, size a multiple of 16)
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst), "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// the shared-memory sources of this thread's bulk stores may be overwritten
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+}
+// this thread's bulk stores are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+
+}  // namespace gdr

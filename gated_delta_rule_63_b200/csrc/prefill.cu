@@ -55,7 +55,7 @@ constexpr uint32_t WS_W_HI = 0;          // W_hi  [kb 2][64 rows][128 B]
 constexpr uint32_t WS_W_LO = 16384;      // W_lo  [kb 2][64 rows][128 B]
 constexpr uint32_t WS_MQ_HI = 32768;     // Mq_hi [64 rows][128 B]
 constexpr uint32_t WS_MQ_LO = 40960;     // Mq_lo [64 rows][128 B]
-constexpr uint32_t WS_UT = 49152;        // Ut fp32 [slice 2][64 rows][64]
+constexpr uint32_t WS_UT = 49152;        // Ut fp32 [slice 2][64 rows][64], 16-B chunk j of row r at j ^ (r & 7)
 constexpr uint32_t WS_SC = 81920;        // fp32 gamma[64], 1/|q|[64], 1/|k|[64]
 constexpr uint32_t WS_REC = 82944;       // record size (81 KiB)
 
@@ -77,7 +77,7 @@ constexpr uint32_t P_COL_S = 0;                      // [K K^T ; Q K^T]
 constexpr uint32_t P_COL_X = 128;                    // W, then Ut (128 cols)
 
 // ---- chain kernel ------------------------------------------------------------
-constexpr int kChainThreads = 128;
+constexpr int kChainThreads = 256;
 // stage: two k-blocks of [Q 0..63 | W_hi 64..127 | W_lo 128..191 | K 192..255],
 // then Mq_hi, Mq_lo
 constexpr uint32_t C_KB = 256 * 128;
@@ -87,14 +87,15 @@ constexpr uint32_t C_STAGE = C_OFF_MQ + 2 * BLK64;
 constexpr uint32_t BLK128 = 128 * 128;
 constexpr uint32_t C_OFF_H = 2 * C_STAGE;            // H_hi, H_lo [128 dk][64 dv]
 constexpr uint32_t C_OFF_U = C_OFF_H + 2 * BLK128;   // U_hi, U_lo, U'_hi, U'_lo [64 tok][64 dv]
-constexpr uint32_t C_OFF_BAR = C_OFF_U + 4 * BLK64;  // full0, full1, mma
-constexpr uint32_t C_SMEM = C_OFF_BAR + 32 + 1024;
+constexpr uint32_t C_OFF_BAR = C_OFF_U + 4 * BLK64;  // full0, full1, p, h, o; tmem base
+constexpr uint32_t C_SMEM = C_OFF_BAR + 48 + 1024;
 static_assert(C_SMEM <= 232448, "chain shared memory exceeds 227 KB");
 static_assert((C_STAGE | C_OFF_H | C_OFF_U) % 1024 == 0, "swizzled tiles need 1 KB alignment");
 constexpr uint32_t C_TM_COLS = 256;
 constexpr uint32_t C_COL_P = 0;      // [Q H0 ; W_hi H0]
-constexpr uint32_t C_COL_O = 64;     // W_lo H0 (lanes 64..127), then Mq U (lanes 0..63)
+constexpr uint32_t C_COL_P2 = 64;    // W_lo H0 (lanes 64..127)
 constexpr uint32_t C_COL_H = 128;    // K^T U' (lanes = dk)
+constexpr uint32_t C_COL_O = 192;    // Mq U (lanes 0..63)
 
 #ifdef GDR_PREFILL_TIMING
 // diagnostic build: step timestamps; prep CTA (0,0,0) in row 0, chain CTA
@@ -317,12 +318,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float dec = blk < ib ? fi * s_eb[j] : (j <= i ? __expf(gi - s_g[j]) : 0.0f);
             m[e] = sv[b2 * 16 + h8 * 8 + e] * qi * s_rk[j] * dec;
           }
-          const uint32_t off = sw128(i, blk * 2 + h8);
-          st_split8_global(rec + WS_MQ_HI + off, rec + WS_MQ_LO + off, m);
+          const uint32_t off = sw128(i, blk * 2 + h8);   // staged in the T region, stored in bulk
+          st_split8_shared(sbase + P_OFF_T + off, sbase + P_OFF_T + BLK64 + off, m);
         }
       }
     }
+    fence_proxy_async();
     __syncthreads();
+    if (tid == 0) {   // Mq_hi | Mq_lo, contiguous in shared memory and in the record
+      bulk_store(rec + WS_MQ_HI, sbase + P_OFF_T, 2 * BLK64);
+      bulk_commit();
+    }
 
     PTIME(0, 4);
     // ---- T = (I + A)^-1, stored transposed on and above the diagonal ----------
@@ -369,6 +375,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     PTIME(0, 5);
     // ---- T' = T diag(beta e^g / |k|), T'' = T diag(beta), hi/lo tiles --------
+    if (tid == 0) bulk_wait_read();   // the Mq staging is about to be overwritten
+    __syncthreads();
     {
       const int r = tid >> 2, qc = tid & 3;   // row r, columns 16 qc .. 16 qc + 15
 #pragma unroll
@@ -415,17 +423,20 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tmem_ld32(tl + 32 * hh, w);
         tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
+        for (int c4 = 0; c4 < 4; ++c4) {   // [W_hi kb0 | W_hi kb1 | W_lo kb0 | W_lo kb1] over the dead K/Q tiles
           const uint32_t off = kb * BLK64 + sw128(r, 4 * hh + c4);
-          st_split8_global(rec + WS_W_HI + off, rec + WS_W_LO + off, w + 8 * c4);
+          st_split8_shared(sbase + P_OFF_KQ + off, sbase + P_OFF_KQ + 2 * BLK64 + off, w + 8 * c4);
         }
       }
     }
+    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     PTIME(0, 8);
     // ---- Ut = T'' V (N = 128) ---------------------------------------------------
     if (tid == 0) {
+      bulk_store(rec + WS_W_HI, sbase + P_OFF_KQ, 4 * BLK64);
+      bulk_commit();
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 128, false, true);
 #pragma unroll
@@ -439,22 +450,33 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     ok = cta_wait(bar_mma, 0, p.err);
   }
   PTIME(0, 9);
-  if (ok && (warp & 2) == 0) {   // Ut rows -> fp32 [slice][row][64]
+  if (ok && (warp & 2) == 0) {   // Ut rows -> fp32 [slice][row][64] staged over the T'' tiles
     const int sl = warp >> 2, r = 32 * (warp & 1) + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + P_COL_X + 64 * sl;
-    float4 *dst = reinterpret_cast<float4 *>(rec + WS_UT + (static_cast<size_t>(sl) * 64 + r) * 256);
+    const uint32_t dst = sbase + P_OFF_T + (static_cast<uint32_t>(sl) * 64 + r) * 256;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       float u[32];
       tmem_ld32(tl + 32 * hh, u);
       tmem_wait_ld();
 #pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4)
-        dst[8 * hh + c4] = make_float4(u[4 * c4], u[4 * c4 + 1], u[4 * c4 + 2], u[4 * c4 + 3]);
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const uint32_t j = (8 * hh + c4) ^ (r & 7);
+        st_shared16(dst + 16 * j, make_uint4(__float_as_uint(u[4 * c4]), __float_as_uint(u[4 * c4 + 1]),
+                                             __float_as_uint(u[4 * c4 + 2]), __float_as_uint(u[4 * c4 + 3])));
+      }
     }
   }
+  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
+  if (tid == 0) {
+    if (ok) {
+      bulk_store(rec + WS_UT, sbase + P_OFF_T, 4 * BLK64);
+      bulk_commit();
+    }
+    bulk_wait_all();   // the stores must finish before the shared memory goes away
+  }
   PTIME(0, 10);
   if (warp == 0) tmem_dealloc(tmem, P_TM_COLS);
 }
@@ -462,6 +484,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // =============================================================================
 // chain: the state of one dv slice of one value head through one window
 // =============================================================================
+// 8 warps: warp w reads TMEM lanes 32 (w & 3) .. + 31 (rows) and columns
+// 32 (w >> 2) .. + 31 of the 64-column slice, so every row of a product is
+// shared by two threads.  Rows 0..63 of [Q; W] H0 are the Q H0 rows (output),
+// rows 64..127 the W H0 rows (state); the K^T U' product has one row per dk.
+// The output product Mq U of chunk c is finished while the tensor core runs
+// the first product of chunk c+1, off the state's critical path.
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              PrefillParams p) {
@@ -476,10 +504,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
   uint8_t *smem = smem_raw + (sbase - raw_addr);
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kh = h / p.group;
-  const uint32_t bar_full = sbase + C_OFF_BAR, bar_mma = sbase + C_OFF_BAR + 16;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 24);
+  const uint32_t bar_full = sbase + C_OFF_BAR;                 // 2 stages
+  const uint32_t bar_p = bar_full + 16, bar_h = bar_full + 24, bar_o = bar_full + 32;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 40);
 
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_holder), C_TM_COLS);
@@ -503,9 +532,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     bulk_load(st + C_OFF_MQ + BLK64, rec + WS_MQ_LO, BLK64, fb);
   };
   if (tid == 0) {
-    mbar_init(bar_full, 1);
-    mbar_init(bar_full + 8, 1);
-    mbar_init(bar_mma, 1);
+    for (int i = 0; i < 5; ++i) mbar_init(bar_full + 8 * i, 1);
     fence_mbar_init();
     for (int cw = 0; cw < 2 && cw < nw; ++cw) load_chunk(cw);
   }
@@ -513,183 +540,200 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const int q4 = warp & 3, ch = warp >> 2;           // lane quarter, column half
+  const int row = 32 * q4 + lane;                    // TMEM lane / dk row
+  const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16) + 32 * ch;
+  const bool wrow = row >= 64;                       // W H0 rows (state) vs Q H0 rows (output)
+  const int r = row & 63;
 
-  // ---- the state: thread tid holds row tid (dk) of this dv slice ---------------
-  float hreg[N];
-  const size_t srow = (static_cast<size_t>(n) * p.hv + h) * D * D + static_cast<size_t>(tid) * D + slice * N;
+  // ---- the state: row `row` (dk), columns 32 ch .. 32 ch + 31 of this dv slice --
+  float hreg[32];
+  const size_t srow = (static_cast<size_t>(n) * p.hv + h) * D * D + static_cast<size_t>(row) * D + slice * N + 32 * ch;
   if (p.state_in) {
 #pragma unroll
-    for (int j = 0; j < N; j += 4) {
+    for (int j = 0; j < 32; j += 4) {
       const float4 v4 = *reinterpret_cast<const float4 *>(p.state_in + srow + j);
       hreg[j] = v4.x; hreg[j + 1] = v4.y; hreg[j + 2] = v4.z; hreg[j + 3] = v4.w;
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < N; ++j) hreg[j] = 0.0f;
+    for (int j = 0; j < 32; ++j) hreg[j] = 0.0f;
   }
   auto write_h = [&]() {
 #pragma unroll
-    for (int cc = 0; cc < 8; ++cc)
-      st_split8_shared(sbase + C_OFF_H + sw128(tid, cc), sbase + C_OFF_H + BLK128 + sw128(tid, cc), hreg + 8 * cc);
+    for (int c4 = 0; c4 < 4; ++c4) {
+      uint4 hi, lo;
+      split8x2(hreg + 8 * c4, hi, lo);
+      const uint32_t off = sw128(row, 4 * ch + c4);
+      st_shared16(sbase + C_OFF_H + off, hi);
+      st_shared16(sbase + C_OFF_H + BLK128 + off, lo);
+    }
   };
   write_h();
   fence_proxy_async();
   __syncthreads();
 
-  const bool wrow = tid >= 64;   // lanes 64..127 hold W H0, lanes 0..63 hold Q H0
-  const int r = tid & 63;
-  uint32_t mma_phase = 0;
+  float oreg[32];            // Q H0 part of o for the chunk whose output is pending
+  int prev_t0 = 0, prev_L = 0;
   bool ok = true;
-  for (int cw = 0; cw < nw && ok; ++cw) {
+  auto finish_output = [&](int cprev) {   // o = Q H0 part + scale Mq U, rows of chunk cprev
+    if (!wrow) {
+      float ro[32];
+      tmem_ld32(tl + C_COL_O, ro);
+      tmem_wait_ld();
+      if (r < prev_L) {
+        uint16_t *dst = p.o + (static_cast<size_t>(prev_t0 + r) * p.hv + h) * D + slice * N + 32 * ch;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float v8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v8[e] = oreg[8 * c4 + e] + p.scale * ro[8 * c4 + e];
+          *reinterpret_cast<uint4 *>(dst + 8 * c4) = pack8x2(v8);
+        }
+      }
+    }
+    (void)cprev;
+  };
+
+  for (int cw = 0; cw < nw; ++cw) {
     const int s = cw & 1;
     const uint32_t st = sbase + s * C_STAGE;
     const int t0 = seq_start + (p.win0 + cw) * C;
     const int L = min(C, seq_end - t0);
     const uint8_t *rec = ws_record(p, n, h, cw);
     const float *sc = reinterpret_cast<const float *>(rec + WS_SC);
-    // this thread's Ut row (W lanes) and per-row scalars, fetched ahead of the MMA
-    float ut[N];
-    float scal_a, scal_b;
+    // this thread's Ut columns (state rows) and per-row scalars, fetched early
+    float ut[32];
     if (wrow) {
       const float4 *src = reinterpret_cast<const float4 *>(rec + WS_UT + (static_cast<size_t>(slice) * 64 + r) * 256);
 #pragma unroll
-      for (int j = 0; j < N / 4; ++j) {
-        const float4 v4 = src[j];
+      for (int j = 0; j < 8; ++j) {
+        const float4 v4 = src[(8 * ch + j) ^ (r & 7)];
         ut[4 * j] = v4.x; ut[4 * j + 1] = v4.y; ut[4 * j + 2] = v4.z; ut[4 * j + 3] = v4.w;
       }
-      scal_a = sc[r];          // gamma_r
-      scal_b = sc[128 + r];    // 1/|k_r|
-    } else {
-      scal_a = sc[r];          // gamma_r
-      scal_b = sc[64 + r];     // 1/|q_r|
     }
-    const float gL = sc[63];   // padding rows carry gamma_{L-1}
+    const float g_r = sc[r];
+    const float scal_b = wrow ? sc[128 + r] : sc[64 + r];   // 1/|k_r| or 1/|q_r|
+    const float gL = sc[63];                                // padding rows carry gamma_{L-1}
     PTIME(1 + cw, 0);
     if (!(ok = cta_wait(bar_full + 8 * s, (cw >> 1) & 1, p.err))) break;
     PTIME(1 + cw, 1);
 
-    // ---- [Q; W_hi] (H_hi + H_lo) and [*; W_lo] H_hi ---------------------------------
+    // ---- [Q; W_hi] (H_hi + H_lo) -> P ;  [*; W_lo] H_hi -> P2 (lanes 64..127) -------
     if (tid == 0) {
       const uint32_t id = idesc_bf16(128, 64, false, true);
+      const uint64_t aq = sdesc(st + C_ROW_Q * 128, 16, 1024);
+      const uint64_t aw = sdesc(st + C_ROW_WHI * 128, 16, 1024);
+      const uint64_t bh = sdesc(sbase + C_OFF_H, BLK128, 1024);
 #pragma unroll
       for (int part = 0; part < 3; ++part) {
-        const uint32_t arow = part < 2 ? C_ROW_Q : C_ROW_WHI;   // part 2: lanes 64..127 get W_lo rows
-        const uint32_t hb = part == 1 ? C_OFF_H + BLK128 : C_OFF_H;
-        const uint32_t dcol = part < 2 ? C_COL_P : C_COL_O;
+        const uint64_t a0 = part < 2 ? aq : aw;
+        const uint64_t b0 = bh + (part == 1 ? (BLK128 >> 4) : 0);
+        const uint32_t dcol = part < 2 ? C_COL_P : C_COL_P2;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t koff = (kk >> 2) * C_KB + (kk & 3) * 32;
-          mma_bf16(tmem + dcol, sdesc(st + koff + arow * 128, 16, 1024),
-                   sdesc(sbase + hb + kk * 2048, BLK128, 1024), id, (part == 1) || kk > 0);
+          mma_bf16(tmem + dcol, a0 + (koff >> 4), b0 + ((kk * 2048) >> 4), id, (part == 1) || kk > 0);
         }
       }
-      mma_commit(bar_mma);
+      mma_commit(bar_p);
     }
-    if (!(ok = cta_wait(bar_mma, mma_phase, p.err))) break;
-    mma_phase ^= 1u;
-
+    // ---- meanwhile: the output of the previous chunk; its stage is free after that
+    if (cw > 0) {
+      if (!(ok = cta_wait(bar_o, (cw - 1) & 1, p.err))) break;
+      finish_output(cw - 1);
+      if (tid == 32 && cw + 1 < nw) load_chunk(cw + 1);   // not the MMA-issuing thread
+    }
     PTIME(1 + cw, 2);
-    // ---- U = Ut - W H0 and U' = U e^(gL - g) / |k| (W lanes); Q H0 part of o ----
-    float oreg[N];
+    if (!(ok = cta_wait(bar_p, cw & 1, p.err))) break;
+    PTIME(1 + cw, 3);
+
+    // ---- U = Ut - W H0 and U' = U e^(gL - g) / |k| (state rows); Q H0 part of o --
     if (wrow) {
-      const float ed = __expf(gL - scal_a) * scal_b;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float pw[32], pl[32];
-        tmem_ld32(tl + C_COL_P + 32 * hh, pw);
-        tmem_ld32(tl + C_COL_O + 32 * hh, pl);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float u[8], us[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            u[e] = ut[32 * hh + 8 * c4 + e] - pw[8 * c4 + e] - pl[8 * c4 + e];
-            us[e] = u[e] * ed;
-          }
-          const uint32_t off = sw128(r, 4 * hh + c4);
-          st_split8_shared(sbase + C_OFF_U + off, sbase + C_OFF_U + BLK64 + off, u);
-          st_split8_shared(sbase + C_OFF_U + 2 * BLK64 + off, sbase + C_OFF_U + 3 * BLK64 + off, us);
-        }
-      }
-    } else {
-      const float f = p.scale * __expf(scal_a) * scal_b;
-      tmem_ld32(tl + C_COL_P, oreg);
-      tmem_ld32(tl + C_COL_P + 32, oreg + 32);
+      const float ed = __expf(gL - g_r) * scal_b;
+      float pw[32], pl[32];
+      tmem_ld32(tl + C_COL_P, pw);
+      tmem_ld32(tl + C_COL_P2, pl);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < N; ++j) oreg[j] *= f;
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float u[8], us[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          u[e] = ut[8 * c4 + e] - pw[8 * c4 + e] - pl[8 * c4 + e];
+          us[e] = u[e] * ed;
+        }
+        const uint32_t off = sw128(r, 4 * ch + c4);
+        uint4 hi, lo;
+        split8x2(u, hi, lo);
+        st_shared16(sbase + C_OFF_U + off, hi);
+        st_shared16(sbase + C_OFF_U + BLK64 + off, lo);
+        split8x2(us, hi, lo);
+        st_shared16(sbase + C_OFF_U + 2 * BLK64 + off, hi);
+        st_shared16(sbase + C_OFF_U + 3 * BLK64 + off, lo);
+      }
+    } else {
+      const float f = p.scale * __expf(g_r) * scal_b;
+      tmem_ld32(tl + C_COL_P, oreg);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) oreg[j] *= f;
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
 
-    PTIME(1 + cw, 3);
-    // ---- K^T U' (hi/lo) -> H part;  Mq U (hi/lo x hi/lo) -> o part -------------
+    PTIME(1 + cw, 4);
+    // ---- K^T U' (hi/lo) -> H part (commit);  Mq U (hi/lo x hi/lo) -> o part (commit)
     if (tid == 0) {
       tc_fence_after();
       const uint32_t idH = idesc_bf16(128, 64, true, true);
       const uint32_t idO = idesc_bf16(128, 64, false, true);
+      const uint64_t ak = sdesc(st + C_ROW_K * 128, C_KB, 1024);
+      const uint64_t bu = sdesc(sbase + C_OFF_U, BLK64, 1024);
 #pragma unroll
       for (int part = 0; part < 2; ++part)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + C_COL_H, sdesc(st + C_ROW_K * 128 + kk * 2048, C_KB, 1024),
-                   sdesc(sbase + C_OFF_U + (2 + part) * BLK64 + kk * 2048, BLK64, 1024), idH,
-                   (part | kk) != 0);
+          mma_bf16(tmem + C_COL_H, ak + ((kk * 2048) >> 4), bu + (((2 + part) * BLK64 + kk * 2048) >> 4),
+                   idH, (part | kk) != 0);
+      mma_commit(bar_h);
+      const uint64_t am = sdesc(st + C_OFF_MQ, 16, 1024);
 #pragma unroll
       for (int part = 0; part < 3; ++part) {   // Mq rows land in lanes 0..63
         const uint32_t aoff = part < 2 ? 0u : BLK64;      // Mq_hi, Mq_hi, Mq_lo
         const uint32_t ub = part == 1 ? BLK64 : 0u;       // U_hi, U_lo, U_hi
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + aoff + kk * 32, 16, 1024),
-                   sdesc(sbase + C_OFF_U + ub + kk * 2048, BLK64, 1024), idO, (part | kk) != 0);
+          mma_bf16(tmem + C_COL_O, am + ((aoff + kk * 32) >> 4), bu + ((ub + kk * 2048) >> 4), idO,
+                   (part | kk) != 0);
       }
-      mma_commit(bar_mma);
+      mma_commit(bar_o);
     }
-    if (!(ok = cta_wait(bar_mma, mma_phase, p.err))) break;
-    mma_phase ^= 1u;
-    if (tid == 0 && cw + 2 < nw) load_chunk(cw + 2);   // stage s is free again
+    prev_t0 = t0;
+    prev_L = L;
+    if (!(ok = cta_wait(bar_h, cw & 1, p.err))) break;
+    PTIME(1 + cw, 5);
 
-    PTIME(1 + cw, 4);
-    // ---- H <- e^gamma_L H + K^T U'; o = Q H0 part + Mq U --------------------------
+    // ---- H <- e^gamma_L H + K^T U' ------------------------------------------------
     {
       const float eL = __expf(gL);
+      float rh[32];
+      tmem_ld32(tl + C_COL_H, rh);
+      tmem_wait_ld();
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float rh[32];
-        tmem_ld32(tl + C_COL_H + 32 * hh, rh);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) hreg[32 * hh + j] = eL * hreg[32 * hh + j] + rh[j];
-      }
+      for (int j = 0; j < 32; ++j) hreg[j] = eL * hreg[j] + rh[j];
       write_h();
-      if (!wrow) {
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float ro[32];
-          tmem_ld32(tl + C_COL_O + 32 * hh, ro);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) oreg[32 * hh + j] += p.scale * ro[j];
-        }
-        if (r < L) {
-          uint16_t *dst = p.o + (static_cast<size_t>(t0 + r) * p.hv + h) * D + slice * N;
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc) *reinterpret_cast<uint4 *>(dst + 8 * cc) = pack8(oreg + 8 * cc);
-        }
-      }
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
-    PTIME(1 + cw, 5);
+    PTIME(1 + cw, 6);
   }
+  if (ok && nw > 0 && cta_wait(bar_o, (nw - 1) & 1, p.err)) finish_output(nw - 1);
   if (p.state_out && ok) {
 #pragma unroll
-    for (int j = 0; j < N; j += 4)
+    for (int j = 0; j < 32; j += 4)
       *reinterpret_cast<float4 *>(p.state_out + srow + j) = make_float4(hreg[j], hreg[j + 1], hreg[j + 2], hreg[j + 3]);
   }
   tc_fence_before();

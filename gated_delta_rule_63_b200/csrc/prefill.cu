@@ -78,6 +78,7 @@ constexpr uint32_t P_COL_X = 128;                    // W, then Ut (128 cols)
 
 // ---- chain kernel ------------------------------------------------------------
 constexpr int kChainThreads = 256;
+constexpr uint32_t BAR_WROWS = 1, BAR_QROWS = 2;      // named barriers of the two chain roles
 // stage: two k-blocks of [Q 0..63 | W_hi 64..127 | W_lo 128..191 | K 192..255],
 // then Mq_hi, Mq_lo
 constexpr uint32_t C_KB = 256 * 128;
@@ -107,7 +108,16 @@ __device__ long long *g_prefill_times;
         blockIdx.y == 0 && blockIdx.z == 0 && (row) < 64)                  \
       g_prefill_times[(row) * 16 + (step)] = clock64();                    \
   } while (0)
+#define PTIME_T(row, step, thread)                                         \
+  do {                                                                     \
+    if (g_prefill_times && threadIdx.x == (thread) && blockIdx.x == 0 &&   \
+        blockIdx.y == 0 && blockIdx.z == 0 && (row) < 64)                  \
+      g_prefill_times[(row) * 16 + (step)] = clock64();                    \
+  } while (0)
 #else
+#define PTIME_T(row, step, thread) \
+  do {                             \
+  } while (0)
 #define PTIME(row, step) \
   do {                   \
   } while (0)
@@ -131,21 +141,15 @@ struct PrefillParams {
 // 8 fp32 values -> hi/lo bf16 16-byte chunks at two addresses (shared or global)
 __device__ __forceinline__ void st_split8_shared(uint32_t hi_addr, uint32_t lo_addr, const float *v8) {
   uint4 hi, lo;
-  split8(v8, hi, lo);
+  split8x2(v8, hi, lo);
   st_shared16(hi_addr, hi);
   st_shared16(lo_addr, lo);
 }
-__device__ __forceinline__ void st_split8_global(uint8_t *hi_p, uint8_t *lo_p, const float *v8) {
-  uint4 hi, lo;
-  split8(v8, hi, lo);
-  *reinterpret_cast<uint4 *>(hi_p) = hi;
-  *reinterpret_cast<uint4 *>(lo_p) = lo;
-}
 
 // one thread waits (bounded), the CTA agrees on the outcome
-__device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity, int *err) {
-  bool ok = true;
-  if (threadIdx.x == 0) ok = mbar_wait(bar, parity, err);
+__device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity, int *err, bool also = true) {
+  bool ok = also;
+  if (threadIdx.x == 0 && ok) ok = mbar_wait(bar, parity, err);
   ok = __syncthreads_and(ok) != 0;
   tc_fence_after();
   return ok;
@@ -287,40 +291,50 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int row = 32 * q4 + lane;
     float sv[32];
     tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + P_COL_S + 32 * hf, sv);
-    tmem_wait_ld();
+    // per-column factors of this thread's 32 columns: 1/|k_j| and the decay e^(g_i - g_j)
     const int i = row & 63, ib = i >> 4;
     const float gi = s_g[i];
-    if (row < 64) {
-      const float bi = s_beta[i] * s_rk[i];
+    float colf[32];
 #pragma unroll
-      for (int b2 = 0; b2 < 2; ++b2) {
-        const int blk = 2 * hf + b2;
-        const float fi = __expf(gi - s_g[blk * 16 + 15]);
+    for (int b2 = 0; b2 < 2; ++b2) {
+      const int blk = 2 * hf + b2;
+      const float fi = __expf(gi - s_g[blk * 16 + 15]);   // used for whole earlier blocks only
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int j = blk * 16 + e;
-          const float dec = blk < ib ? fi * s_eb[j] : __expf(fminf(gi - s_g[j], 0.0f));
-          if (j < i) AT[i * LD + j] = bi * s_rk[j] * sv[b2 * 16 + e] * dec;
+      for (int e4 = 0; e4 < 4; ++e4) {
+        const int j0 = blk * 16 + 4 * e4;
+        const float4 rk4 = *reinterpret_cast<const float4 *>(s_rk + j0);
+        const float4 g4 = *reinterpret_cast<const float4 *>(s_g + j0);
+        const float4 eb4 = *reinterpret_cast<const float4 *>(s_eb + j0);
+        const float rkv[4] = {rk4.x, rk4.y, rk4.z, rk4.w};
+        const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+        const float ebv[4] = {eb4.x, eb4.y, eb4.z, eb4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = j0 + e;
+          float dec;
+          if (blk < ib) dec = fi * ebv[e];
+          else dec = j <= i ? __expf(gi - gv[e]) : 0.0f;
+          colf[b2 * 16 + 4 * e4 + e] = rkv[e] * dec;
         }
       }
-    } else {
+    }
+    tmem_wait_ld();
+    if (row < 64) {   // A_ij = beta_i / |k_i| * (k_i.k_j) / |k_j| * e^(g_i - g_j), j < i
+      const float bi = s_beta[i] * s_rk[i];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int j = 32 * hf + e;
+        if (j < i) AT[i * LD + j] = bi * sv[e] * colf[e];
+      }
+    } else {          // Mq_ij = (q_i.k_j) / (|q_i| |k_j|) * e^(g_i - g_j), j <= i
       const float qi = s_rq[i];
 #pragma unroll
-      for (int b2 = 0; b2 < 2; ++b2) {
-        const int blk = 2 * hf + b2;
-        const float fi = __expf(gi - s_g[blk * 16 + 15]);
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float m[8];
 #pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-          float m[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int j = blk * 16 + h8 * 8 + e;
-            const float dec = blk < ib ? fi * s_eb[j] : (j <= i ? __expf(gi - s_g[j]) : 0.0f);
-            m[e] = sv[b2 * 16 + h8 * 8 + e] * qi * s_rk[j] * dec;
-          }
-          const uint32_t off = sw128(i, blk * 2 + h8);   // staged in the T region, stored in bulk
-          st_split8_shared(sbase + P_OFF_T + off, sbase + P_OFF_T + BLK64 + off, m);
-        }
+        for (int e = 0; e < 8; ++e) m[e] = sv[8 * c4 + e] * qi * colf[8 * c4 + e];
+        const uint32_t off = sw128(i, 4 * hf + c4);   // staged in the T region, stored in bulk
+        st_split8_shared(sbase + P_OFF_T + off, sbase + P_OFF_T + BLK64 + off, m);
       }
     }
     fence_proxy_async();
@@ -488,8 +502,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // 32 (w >> 2) .. + 31 of the 64-column slice, so every row of a product is
 // shared by two threads.  Rows 0..63 of [Q; W] H0 are the Q H0 rows (output),
 // rows 64..127 the W H0 rows (state); the K^T U' product has one row per dk.
-// The output product Mq U of chunk c is finished while the tensor core runs
-// the first product of chunk c+1, off the state's critical path.
+// The warps split by role: the state-row warps (TMEM lanes 64..127) compute U
+// and issue the tensor-core products, while the output-row warps (lanes
+// 0..63) finish the previous chunk's output (Mq U, issued after U) and stream
+// in the next chunk; the two roles meet only at the state update.
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              PrefillParams p) {
@@ -595,6 +611,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     (void)cprev;
   };
 
+  // bounded wait shared by one role's 128 threads (its leader polls)
+  auto role_wait = [&](uint32_t bar, uint32_t parity, bool is_leader, uint32_t id) {
+    bool fine = true;
+    if (is_leader) fine = mbar_wait(bar, parity, p.err);
+    fine = !named_sync_or(id, 128, !fine);
+    tc_fence_after();
+    return fine;
+  };
+
   for (int cw = 0; cw < nw; ++cw) {
     const int s = cw & 1;
     const uint32_t st = sbase + s * C_STAGE;
@@ -620,7 +645,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     PTIME(1 + cw, 1);
 
     // ---- [Q; W_hi] (H_hi + H_lo) -> P ;  [*; W_lo] H_hi -> P2 (lanes 64..127) -------
-    if (tid == 0) {
+    if (tid == 64) {   // a state-row thread issues the state products
       const uint32_t id = idesc_bf16(128, 64, false, true);
       const uint64_t aq = sdesc(st + C_ROW_Q * 128, 16, 1024);
       const uint64_t aw = sdesc(st + C_ROW_WHI * 128, 16, 1024);
@@ -637,58 +662,72 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
       }
       mma_commit(bar_p);
+      PTIME_T(1 + cw, 10, 64);
     }
-    // ---- meanwhile: the output of the previous chunk; its stage is free after that
-    if (cw > 0) {
-      if (!(ok = cta_wait(bar_o, (cw - 1) & 1, p.err))) break;
-      finish_output(cw - 1);
-      if (tid == 32 && cw + 1 < nw) load_chunk(cw + 1);   // not the MMA-issuing thread
-    }
-    PTIME(1 + cw, 2);
-    if (!(ok = cta_wait(bar_p, cw & 1, p.err))) break;
-    PTIME(1 + cw, 3);
-
-    // ---- U = Ut - W H0 and U' = U e^(gL - g) / |k| (state rows); Q H0 part of o --
-    if (wrow) {
-      const float ed = __expf(gL - g_r) * scal_b;
-      float pw[32], pl[32];
-      tmem_ld32(tl + C_COL_P, pw);
-      tmem_ld32(tl + C_COL_P2, pl);
-      tmem_wait_ld();
+    PTIME(1 + cw, 7);
+    bool good = true;   // this thread's waits succeeded
+    if (!wrow) {
+      // output rows: the previous chunk's output, then its stage takes chunk cw + 1
+      if (cw > 0) {
+        good = role_wait(bar_o, (cw - 1) & 1, tid == 0, BAR_QROWS);
+        if (good && tid == 0 && cw + 1 < nw) load_chunk(cw + 1);
+        PTIME(1 + cw, 8);
+        if (good) finish_output(cw - 1);
+        PTIME(1 + cw, 9);
+      }
+      PTIME(1 + cw, 2);
+      good = role_wait(bar_p, cw & 1, tid == 0, BAR_QROWS) && good;
+      if (good) {   // Q H0 part of o
+        const float f = p.scale * __expf(g_r) * scal_b;
+        tmem_ld32(tl + C_COL_P, oreg);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float u[8], us[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          u[e] = ut[8 * c4 + e] - pw[8 * c4 + e] - pl[8 * c4 + e];
-          us[e] = u[e] * ed;
-        }
-        const uint32_t off = sw128(r, 4 * ch + c4);
-        uint4 hi, lo;
-        split8x2(u, hi, lo);
-        st_shared16(sbase + C_OFF_U + off, hi);
-        st_shared16(sbase + C_OFF_U + BLK64 + off, lo);
-        split8x2(us, hi, lo);
-        st_shared16(sbase + C_OFF_U + 2 * BLK64 + off, hi);
-        st_shared16(sbase + C_OFF_U + 3 * BLK64 + off, lo);
+        for (int j = 0; j < 32; ++j) oreg[j] *= f;
       }
     } else {
-      const float f = p.scale * __expf(g_r) * scal_b;
-      tmem_ld32(tl + C_COL_P, oreg);
-      tmem_wait_ld();
+      // the previous output product must be done reading the U tiles
+      if (cw > 0) good = role_wait(bar_o, (cw - 1) & 1, tid == 64, BAR_WROWS);
+      good = role_wait(bar_p, cw & 1, tid == 64, BAR_WROWS) && good;
+      PTIME_T(1 + cw, 11, 64);
+      // ---- U = Ut - W H0 and U' = U e^(gL - g) / |k| ---------------------------------
+      if (good) {
+        const float ed = __expf(gL - g_r) * scal_b;
+        float pw[32], pl[32];
+        tmem_ld32(tl + C_COL_P, pw);
+        tmem_ld32(tl + C_COL_P2, pl);
+        tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) oreg[j] *= f;
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float u[8], us[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            u[e] = ut[8 * c4 + e] - pw[8 * c4 + e] - pl[8 * c4 + e];
+            us[e] = u[e] * ed;
+          }
+          const uint32_t off = sw128(r, 4 * ch + c4);
+          uint4 hi, lo;
+          split8x2(u, hi, lo);
+          st_shared16(sbase + C_OFF_U + off, hi);
+          st_shared16(sbase + C_OFF_U + BLK64 + off, lo);
+          split8x2(us, hi, lo);
+          st_shared16(sbase + C_OFF_U + 2 * BLK64 + off, hi);
+          st_shared16(sbase + C_OFF_U + 3 * BLK64 + off, lo);
+        }
+      }
+      PTIME_T(1 + cw, 12, 64);
+      // the U tiles are complete among the state-row warps
+      fence_proxy_async();
+      tc_fence_before();
+      named_sync(BAR_WROWS, 128);
+      PTIME_T(1 + cw, 13, 64);
     }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
 
     PTIME(1 + cw, 4);
-    // ---- K^T U' (hi/lo) -> H part (commit);  Mq U (hi/lo x hi/lo) -> o part (commit)
-    if (tid == 0) {
+    // ---- K^T U' (hi/lo) -> H part, issued by thread 64 and waited on;
+    //      Mq U (hi/lo x hi/lo) -> o part, issued by thread 96, waited on next chunk
+    if (tid == 64) {
       tc_fence_after();
       const uint32_t idH = idesc_bf16(128, 64, true, true);
-      const uint32_t idO = idesc_bf16(128, 64, false, true);
       const uint64_t ak = sdesc(st + C_ROW_K * 128, C_KB, 1024);
       const uint64_t bu = sdesc(sbase + C_OFF_U, BLK64, 1024);
 #pragma unroll
@@ -698,6 +737,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           mma_bf16(tmem + C_COL_H, ak + ((kk * 2048) >> 4), bu + (((2 + part) * BLK64 + kk * 2048) >> 4),
                    idH, (part | kk) != 0);
       mma_commit(bar_h);
+      PTIME_T(1 + cw, 14, 64);
+    } else if (tid == 96) {
+      tc_fence_after();
+      const uint32_t idO = idesc_bf16(128, 64, false, true);
+      const uint64_t bu = sdesc(sbase + C_OFF_U, BLK64, 1024);
       const uint64_t am = sdesc(st + C_OFF_MQ, 16, 1024);
 #pragma unroll
       for (int part = 0; part < 3; ++part) {   // Mq rows land in lanes 0..63
@@ -712,7 +756,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
     prev_t0 = t0;
     prev_L = L;
-    if (!(ok = cta_wait(bar_h, cw & 1, p.err))) break;
+    if (!(ok = cta_wait(bar_h, cw & 1, p.err, good))) break;
     PTIME(1 + cw, 5);
 
     // ---- H <- e^gamma_L H + K^T U' ------------------------------------------------
@@ -730,7 +774,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     __syncthreads();
     PTIME(1 + cw, 6);
   }
-  if (ok && nw > 0 && cta_wait(bar_o, (nw - 1) & 1, p.err)) finish_output(nw - 1);
+  if (ok && nw > 0 && cta_wait(bar_o, (nw - 1) & 1, p.err, true)) finish_output(nw - 1);
   if (p.state_out && ok) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4)

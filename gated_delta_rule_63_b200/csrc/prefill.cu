@@ -58,6 +58,7 @@ constexpr uint32_t WS_MQ_LO = 40960;     // Mq_lo [64 rows][128 B]
 constexpr uint32_t WS_UT = 49152;        // Ut fp32 [slice 2][64 rows][64], 16-B chunk j of row r at j ^ (r & 7)
 constexpr uint32_t WS_SC = 81920;        // fp32 gamma[64], 1/|q|[64], 1/|k|[64]
 constexpr uint32_t WS_REC = 82944;       // record size (81 KiB)
+static_assert(WS_MQ_LO == WS_MQ_HI + 64 * 128, "Mq_hi and Mq_lo are copied as one block");
 
 // ---- prep kernel -------------------------------------------------------------
 constexpr int kPrepThreads = 256;
@@ -77,44 +78,45 @@ constexpr uint32_t P_COL_S = 0;                      // [K K^T ; Q K^T]
 constexpr uint32_t P_COL_X = 128;                    // W, then Ut (128 cols)
 
 // ---- chain kernel ------------------------------------------------------------
-constexpr int kChainThreads = 256;
-constexpr uint32_t BAR_WROWS = 1, BAR_QROWS = 2;      // named barriers of the two chain roles
-// stage: two k-blocks of [Q 0..63 | W_hi 64..127 | W_lo 128..191 | K 192..255],
-// then Mq_hi, Mq_lo
-constexpr uint32_t C_KB = 256 * 128;
-constexpr uint32_t C_ROW_Q = 0, C_ROW_WHI = 64, C_ROW_WLO = 128, C_ROW_K = 192;
-constexpr uint32_t C_OFF_MQ = 2 * C_KB;
-constexpr uint32_t C_STAGE = C_OFF_MQ + 2 * BLK64;
+constexpr int kChainThreads = 288;                    // warps 0..7 state and output, warp 8 control
+constexpr int kCtrlWarp = 8;
+// stage: per k-block the rows [Q 0..63 | W_hi 64..127 | W_lo 128..191] (A operands
+// [Q; W_hi] and [W_hi; W_lo]), then K (two dk blocks), then [Mq_hi; Mq_lo]
+constexpr uint32_t C_QW_KB = 192 * 128;
+constexpr uint32_t C_OFF_K = 2 * C_QW_KB;
+constexpr uint32_t C_OFF_MQ = C_OFF_K + 2 * BLK64;
+constexpr uint32_t C_STAGE = C_OFF_MQ + 2 * BLK64;   // 80 KiB
 constexpr uint32_t BLK128 = 128 * 128;
-constexpr uint32_t C_OFF_H = 2 * C_STAGE;            // H_hi, H_lo [128 dk][64 dv]
-constexpr uint32_t C_OFF_U = C_OFF_H + 2 * BLK128;   // U_hi, U_lo, U'_hi, U'_lo [64 tok][64 dv]
-constexpr uint32_t C_OFF_BAR = C_OFF_U + 4 * BLK64;  // full0, full1, p, h, o; tmem base
-constexpr uint32_t C_SMEM = C_OFF_BAR + 48 + 1024;
+constexpr uint32_t C_OFF_H = 2 * C_STAGE;            // [H_hi | H_lo], each [128 dk][64 dv]
+constexpr uint32_t C_OFF_U = C_OFF_H + 2 * BLK128;   // [U_hi | U_lo | U'_hi | U'_lo], each [64 tok][64 dv]
+constexpr uint32_t C_OFF_BAR = C_OFF_U + 4 * BLK64;  // 13 mbarriers, tmem base, abort flag
+constexpr uint32_t C_SMEM = C_OFF_BAR + 128 + 1024;
 static_assert(C_SMEM <= 232448, "chain shared memory exceeds 227 KB");
-static_assert((C_STAGE | C_OFF_H | C_OFF_U) % 1024 == 0, "swizzled tiles need 1 KB alignment");
-constexpr uint32_t C_TM_COLS = 256;
-constexpr uint32_t C_COL_P = 0;      // [Q H0 ; W_hi H0]
-constexpr uint32_t C_COL_P2 = 64;    // W_lo H0 (lanes 64..127)
-constexpr uint32_t C_COL_H = 128;    // K^T U' (lanes = dk)
-constexpr uint32_t C_COL_O = 192;    // Mq U (lanes 0..63)
+static_assert((C_QW_KB | C_OFF_K | C_OFF_MQ | C_STAGE | C_OFF_H | C_OFF_U) % 1024 == 0,
+              "swizzled tiles need 1 KB alignment");
+constexpr uint32_t C_TM_COLS = 512;
+constexpr uint32_t C_COL_P = 0;      // [Q; W_hi] [H_hi | H_lo]: lanes 0..63 Q rows, 64..127 W rows
+constexpr uint32_t C_COL_P2 = 128;   // [W_hi; W_lo] H_hi: lanes 64..127 hold W_lo H_hi
+constexpr uint32_t C_COL_H = 256;    // K^T [U'_hi | U'_lo], lanes = dk
+constexpr uint32_t C_COL_O = 384;    // [Mq_hi; Mq_lo] [U_hi | U_lo] + Mq_lo U_hi, lanes 0..63
 
 #ifdef GDR_PREFILL_TIMING
 // diagnostic build: step timestamps; prep CTA (0,0,0) in row 0, chain CTA
-// (0,0,0) chunk c in row 1 + c (16 slots per row)
+// (0,0,0) chunk c in row 1 + c (32 slots per row).  Kernels read the buffer
+// pointer once (PTIME_INIT) so that a marker costs no memory round trip.
 __device__ long long *g_prefill_times;
-#define PTIME(row, step)                                                   \
-  do {                                                                     \
-    if (g_prefill_times && threadIdx.x == 0 && blockIdx.x == 0 &&          \
-        blockIdx.y == 0 && blockIdx.z == 0 && (row) < 64)                  \
-      g_prefill_times[(row) * 16 + (step)] = clock64();                    \
-  } while (0)
+#define PTIME_INIT() long long *const ptime_buf_ = g_prefill_times
 #define PTIME_T(row, step, thread)                                         \
   do {                                                                     \
-    if (g_prefill_times && threadIdx.x == (thread) && blockIdx.x == 0 &&   \
+    if (ptime_buf_ && threadIdx.x == (thread) && blockIdx.x == 0 &&        \
         blockIdx.y == 0 && blockIdx.z == 0 && (row) < 64)                  \
-      g_prefill_times[(row) * 16 + (step)] = clock64();                    \
+      ptime_buf_[(row) * 32 + (step)] = clock64();                         \
   } while (0)
+#define PTIME(row, step) PTIME_T(row, step, 0)
 #else
+#define PTIME_INIT() \
+  do {               \
+  } while (0)
 #define PTIME_T(row, step, thread) \
   do {                             \
   } while (0)
@@ -165,6 +167,7 @@ __device__ __forceinline__ uint8_t *ws_record(const PrefillParams &p, int n, int
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
+  PTIME_INIT();
   const int cw = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
   const int seq_start = p.cu[n], seq_end = p.cu[n + 1];
   const int t0 = seq_start + (p.win0 + cw) * C;
@@ -290,7 +293,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int q4 = warp & 3, hf = warp >> 2;
     const int row = 32 * q4 + lane;
     float sv[32];
-    tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + P_COL_S + 32 * hf, sv);
+    PTIME(0, 17);
     // per-column factors of this thread's 32 columns: 1/|k_j| and the decay e^(g_i - g_j)
     const int i = row & 63, ib = i >> 4;
     const float gi = s_g[i];
@@ -318,6 +321,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
       }
     }
+    PTIME(0, 11);
+    tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + P_COL_S + 32 * hf, sv);
     tmem_wait_ld();
     if (row < 64) {   // A_ij = beta_i / |k_i| * (k_i.k_j) / |k_j| * e^(g_i - g_j), j < i
       const float bi = s_beta[i] * s_rk[i];
@@ -337,6 +342,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         st_split8_shared(sbase + P_OFF_T + off, sbase + P_OFF_T + BLK64 + off, m);
       }
     }
+    PTIME(0, 12);
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {   // Mq_hi | Mq_lo, contiguous in shared memory and in the record
@@ -360,6 +366,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       for (int r = 0; r < 16; ++r)
         if (r >= cc) AT[(16 * bb + cc) * LD + 16 * bb + r] = x[r];
     }
+    PTIME(0, 13);
     __syncthreads();
     for (int d = 1; d < 4; ++d) {   // T_bc = -T_bb sum_{m=c}^{b-1} A_bm T_mc, b - c = d
       const int nb = 4 - d;
@@ -385,6 +392,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         AT[(16 * cb + j) * LD + 16 * bb + r] = sacc;
       }
       __syncthreads();
+      PTIME(0, 13 + d);
     }
 
     PTIME(0, 5);
@@ -498,17 +506,46 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // =============================================================================
 // chain: the state of one dv slice of one value head through one window
 // =============================================================================
-// 8 warps: warp w reads TMEM lanes 32 (w & 3) .. + 31 (rows) and columns
-// 32 (w >> 2) .. + 31 of the 64-column slice, so every row of a product is
-// shared by two threads.  Rows 0..63 of [Q; W] H0 are the Q H0 rows (output),
-// rows 64..127 the W H0 rows (state); the K^T U' product has one row per dk.
-// The warps split by role: the state-row warps (TMEM lanes 64..127) compute U
-// and issue the tensor-core products, while the output-row warps (lanes
-// 0..63) finish the previous chunk's output (Mq U, issued after U) and stream
-// in the next chunk; the two roles meet only at the state update.
+// One CTA per (64-column dv slice, value head, sequence).  The fp32 state slice
+// H (128 dk rows x 64 dv columns) stays in registers of warps 0..7: warp w
+// holds rows 32 (w & 3) .. + 31 (its TMEM lane quarter), columns
+// 32 (w >> 2) .. + 31.  Per chunk:
+//   P  = [Q; W_hi] [H_hi | H_lo],  P2 = [W_hi; W_lo] H_hi          tensor cores
+//   U  = Ut - W H0,  U' = U e^(gamma_L - gamma) / |k|                warps 2, 3, 6, 7 (lanes 64..127)
+//   H' = K^T [U'_hi | U'_lo]                                         tensor cores
+//   H  = e^gamma_L H + H'                                            warps 0..7
+//   O  = [Mq_hi; Mq_lo] [U_hi | U_lo] + Mq_lo U_hi                   tensor cores
+//   o  = scale (e^gamma / |q| Q H0 + O)                              warps 0, 1, 4, 5 (lanes 0..63)
+// N = 128 products stack the hi and lo parts of one operand side by side, so
+// each fp32 product takes two MMA groups instead of three.  Warp 8 issues every
+// product and every copy and does nothing else; the roles meet only on
+// mbarriers (no CTA-wide barrier inside the chunk loop).  Operands arrive two
+// chunks ahead in three groups ([Q | W_hi | W_lo], K, Mq), each refilled as
+// soon as the products reading it are complete; Ut and the chunk scalars are
+// read into registers a chunk ahead; the output of a chunk is finished while
+// the next chunk's first products run.
+
+// Bounded mbarrier wait that gives up at once after a timeout anywhere in the
+// CTA.  The waiting thread sleeps in try_wait (it takes no issue slots from
+// the warps that share its scheduler) and gives up after about 2^32 cycles.
+__device__ __forceinline__ bool chain_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort, int *err) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const long long start = clock64();
+  while (!*abort) {
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (clock64() - start > (1LL << 32)) {
+      *abort = 1u;
+      raise_device_error(err, GDR_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return false;
+}
+
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              PrefillParams p) {
+  PTIME_INIT();
   const int slice = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
   const int seq_start = p.cu[n], seq_end = p.cu[n + 1];
   const int n_all = (seq_end - seq_start + C - 1) / C;
@@ -522,58 +559,79 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   uint8_t *smem = smem_raw + (sbase - raw_addr);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kh = h / p.group;
-  const uint32_t bar_full = sbase + C_OFF_BAR;                 // 2 stages
-  const uint32_t bar_p = bar_full + 16, bar_h = bar_full + 24, bar_o = bar_full + 32;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 40);
+  const uint32_t bars = sbase + C_OFF_BAR;
+  const uint32_t full_qw = bars, full_k = bars + 16, full_mq = bars + 32;   // + 8 * stage
+  const uint32_t bar_p = bars + 48, bar_h = bars + 56, bar_o = bars + 64;  // products complete
+  const uint32_t o_free = bars + 72, h_ready = bars + 80, u_ready = bars + 88, bar_drain = bars + 96;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 104);
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C_OFF_BAR + 108);
+  const bool ctrl = warp == kCtrlWarp;
 
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_holder), C_TM_COLS);
     tmem_relinquish();
   }
-  // chunk cw of the window into stage cw & 1
-  auto load_chunk = [&](int cw) {
-    const uint32_t st = sbase + (cw & 1) * C_STAGE;
-    const uint32_t fb = bar_full + 8 * (cw & 1);
-    const int t0 = seq_start + (p.win0 + cw) * C;
+  auto t0_of = [&](int cw) { return seq_start + (p.win0 + cw) * C; };
+  // copies of chunk cw into stage cw & 1 (lane 0 of the control warp); issued counts per group
+  int iss_qw = 0, iss_k = 0, iss_mq = 0, wt_qw = 0, wt_k = 0, wt_mq = 0;
+  auto load_qw = [&](int cw) {
+    const uint32_t st = sbase + (cw & 1) * C_STAGE, fb = full_qw + 8 * (cw & 1);
     const uint8_t *rec = ws_record(p, n, h, cw);
-    mbar_arrive_expect_tx(fb, 10 * BLK64);
+    mbar_arrive_expect_tx(fb, 6 * BLK64);
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb) {
-      tma_load_2d(st + kb * C_KB + C_ROW_Q * 128, &tm_q, kh * D + kb * 64, t0, fb);
-      tma_load_2d(st + kb * C_KB + C_ROW_K * 128, &tm_k, kh * D + kb * 64, t0, fb);
-      bulk_load(st + kb * C_KB + C_ROW_WHI * 128, rec + WS_W_HI + kb * BLK64, BLK64, fb);
-      bulk_load(st + kb * C_KB + C_ROW_WLO * 128, rec + WS_W_LO + kb * BLK64, BLK64, fb);
+      tma_load_2d(st + kb * C_QW_KB, &tm_q, kh * D + kb * 64, t0_of(cw), fb);
+      bulk_load(st + kb * C_QW_KB + 64 * 128, rec + WS_W_HI + kb * BLK64, BLK64, fb);
+      bulk_load(st + kb * C_QW_KB + 128 * 128, rec + WS_W_LO + kb * BLK64, BLK64, fb);
     }
-    bulk_load(st + C_OFF_MQ, rec + WS_MQ_HI, BLK64, fb);
-    bulk_load(st + C_OFF_MQ + BLK64, rec + WS_MQ_LO, BLK64, fb);
+    iss_qw = cw + 1;
   };
-  if (tid == 0) {
-    for (int i = 0; i < 5; ++i) mbar_init(bar_full + 8 * i, 1);
+  auto load_k = [&](int cw) {
+    const uint32_t st = sbase + (cw & 1) * C_STAGE, fb = full_k + 8 * (cw & 1);
+    mbar_arrive_expect_tx(fb, 2 * BLK64);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) tma_load_2d(st + C_OFF_K + kb * BLK64, &tm_k, kh * D + kb * 64, t0_of(cw), fb);
+    iss_k = cw + 1;
+  };
+  auto load_mq = [&](int cw) {   // Mq_hi | Mq_lo are contiguous in the record
+    const uint32_t st = sbase + (cw & 1) * C_STAGE, fb = full_mq + 8 * (cw & 1);
+    mbar_arrive_expect_tx(fb, 2 * BLK64);
+    bulk_load(st + C_OFF_MQ, ws_record(p, n, h, cw) + WS_MQ_HI, 2 * BLK64, fb);
+    iss_mq = cw + 1;
+  };
+  if (ctrl && lane == 0) {
+    // full x 6, products x 3, o_free (4 output warps), h_ready (8 warps), u_ready (4 state warps), drain
+    const uint32_t counts[13] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 8, 4, 1};
+    for (int i = 0; i < 13; ++i) mbar_init(bars + 8 * i, counts[i]);
+    *abort_flag = 0u;
     fence_mbar_init();
-    for (int cw = 0; cw < 2 && cw < nw; ++cw) load_chunk(cw);
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    for (int cw = 0; cw < 2 && cw < nw; ++cw) {
+      load_qw(cw);
+      load_k(cw);
+      load_mq(cw);
+    }
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  const int q4 = warp & 3, ch = warp >> 2;           // lane quarter, column half
-  const int row = 32 * q4 + lane;                    // TMEM lane / dk row
-  const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16) + 32 * ch;
-  const bool wrow = row >= 64;                       // W H0 rows (state) vs Q H0 rows (output)
-  const int r = row & 63;
+  const int q4 = warp & 3, ch = (warp >> 2) & 1;     // lane quarter, column half
+  const int row = 32 * q4 + lane;                    // TMEM lane / dk row of the state
+  const bool wrow = row >= 64;                       // W rows (state side) vs Q rows (output side)
+  const int r = row & 63;                            // chunk row
 
-  // ---- the state: row `row` (dk), columns 32 ch .. 32 ch + 31 of this dv slice --
+  // ---- the state: row `row`, columns 32 ch .. 32 ch + 31 of this dv slice --------------
   float hreg[32];
   const size_t srow = (static_cast<size_t>(n) * p.hv + h) * D * D + static_cast<size_t>(row) * D + slice * N + 32 * ch;
-  if (p.state_in) {
+  if (!ctrl) {
+    if (p.state_in) {
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      const float4 v4 = *reinterpret_cast<const float4 *>(p.state_in + srow + j);
-      hreg[j] = v4.x; hreg[j + 1] = v4.y; hreg[j + 2] = v4.z; hreg[j + 3] = v4.w;
+      for (int j = 0; j < 32; j += 4) {
+        const float4 v4 = *reinterpret_cast<const float4 *>(p.state_in + srow + j);
+        hreg[j] = v4.x; hreg[j + 1] = v4.y; hreg[j + 2] = v4.z; hreg[j + 3] = v4.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) hreg[j] = 0.0f;
     }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) hreg[j] = 0.0f;
   }
   auto write_h = [&]() {
 #pragma unroll
@@ -585,203 +643,260 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       st_shared16(sbase + C_OFF_H + BLK128 + off, lo);
     }
   };
-  write_h();
-  fence_proxy_async();
-  __syncthreads();
+  tc_fence_before();
+  __syncthreads();   // barriers initialised, tensor memory allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
 
-  float oreg[32];            // Q H0 part of o for the chunk whose output is pending
-  int prev_t0 = 0, prev_L = 0;
-  bool ok = true;
-  auto finish_output = [&](int cprev) {   // o = Q H0 part + scale Mq U, rows of chunk cprev
-    if (!wrow) {
-      float ro[32];
-      tmem_ld32(tl + C_COL_O, ro);
-      tmem_wait_ld();
-      if (r < prev_L) {
-        uint16_t *dst = p.o + (static_cast<size_t>(prev_t0 + r) * p.hv + h) * D + slice * N + 32 * ch;
+  if (ctrl) {
+    // =========================== control warp ===========================
+    for (int cw = 0; cw < nw; ++cw) {
+      const int s = cw & 1;
+      const uint32_t par = (cw >> 1) & 1, ph = cw & 1;
+      const uint32_t st = sbase + s * C_STAGE;
+      // ---- P = [Q; W_hi] [H_hi | H_lo] (N = 128), P2 = [W_hi; W_lo] H_hi (N = 64) ----------
+      PTIME_T(1 + cw, 25, 32 * kCtrlWarp);
+      if (chain_wait(full_qw + 8 * s, par, abort_flag, p.err)) wt_qw = cw + 1;
+      PTIME_T(1 + cw, 28, 32 * kCtrlWarp);
+      chain_wait(h_ready, ph, abort_flag, p.err);    // H tiles of this chunk; P of the last one read
+      PTIME_T(1 + cw, 11, 32 * kCtrlWarp);
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t id1 = idesc_bf16(128, 128, false, true), id2 = idesc_bf16(128, 64, false, true);
+        const uint64_t bh = sdesc(sbase + C_OFF_H, BLK128, 1024);
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float v8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v8[e] = oreg[8 * c4 + e] + p.scale * ro[8 * c4 + e];
-          *reinterpret_cast<uint4 *>(dst + 8 * c4) = pack8x2(v8);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * C_QW_KB + (kk & 3) * 32;
+          mma_bf16(tmem + C_COL_P, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id1, kk > 0);
         }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * C_QW_KB + 64 * 128 + (kk & 3) * 32;
+          mma_bf16(tmem + C_COL_P2, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id2, kk > 0);
+        }
+        mma_commit(bar_p);
       }
+      __syncwarp();
+      PTIME_T(1 + cw, 1, 32 * kCtrlWarp);
+      chain_wait(bar_p, ph, abort_flag, p.err);
+      PTIME_T(1 + cw, 2, 32 * kCtrlWarp);
+      if (lane == 0 && cw + 2 < nw) load_qw(cw + 2);   // P has read this stage's [Q | W]
+      __syncwarp();
+      // ---- H' = K^T [U'_hi | U'_lo] ----------------------------------------------------------
+      chain_wait(u_ready, ph, abort_flag, p.err);
+      PTIME_T(1 + cw, 3, 32 * kCtrlWarp);
+      if (chain_wait(full_k + 8 * s, par, abort_flag, p.err)) wt_k = cw + 1;
+      PTIME_T(1 + cw, 8, 32 * kCtrlWarp);
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t idH = idesc_bf16(128, 128, true, true);
+        const uint64_t ak = sdesc(st + C_OFF_K, BLK64, 1024);
+        const uint64_t bu = sdesc(sbase + C_OFF_U + 2 * BLK64, BLK64, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + C_COL_H, ak + ((kk * 2048) >> 4), bu + ((kk * 2048) >> 4), idH, kk > 0);
+        mma_commit(bar_h);
+      }
+      __syncwarp();
+      PTIME_T(1 + cw, 4, 32 * kCtrlWarp);
+      // ---- O = [Mq_hi; Mq_lo] [U_hi | U_lo] + Mq_lo U_hi (rows in lanes 0..63) ----------------
+      if (cw > 0) {
+        chain_wait(o_free, ph ^ 1, abort_flag, p.err);   // the previous O is read ...
+        PTIME_T(1 + cw, 13, 32 * kCtrlWarp);
+        if (lane == 0 && cw + 1 < nw) load_mq(cw + 1);   // ... and its Mq stage is free
+        __syncwarp();
+      }
+      if (chain_wait(full_mq + 8 * s, par, abort_flag, p.err)) wt_mq = cw + 1;
+      PTIME_T(1 + cw, 14, 32 * kCtrlWarp);
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t idO1 = idesc_bf16(128, 128, false, true), idO2 = idesc_bf16(128, 64, false, true);
+        const uint64_t bo = sdesc(sbase + C_OFF_U, BLK64, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO1, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + BLK64 + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO2, 1);
+        mma_commit(bar_o);
+      }
+      __syncwarp();
+      PTIME_T(1 + cw, 9, 32 * kCtrlWarp);
+      chain_wait(bar_h, ph, abort_flag, p.err);
+      PTIME_T(1 + cw, 10, 32 * kCtrlWarp);
+      if (lane == 0 && cw + 2 < nw) load_k(cw + 2);    // K^T U' has read this stage's K
+      __syncwarp();
     }
-    (void)cprev;
-  };
+    if (lane == 0) {
+      // every product completes before tensor memory is released; after a
+      // timeout, copies may still be landing in shared memory: let them finish
+      mma_commit(bar_drain);
+      mbar_wait(bar_drain, 0, p.err, 1u << 20);
+      for (int c = wt_qw; c < iss_qw; ++c) mbar_wait(full_qw + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
+      for (int c = wt_k; c < iss_k; ++c) mbar_wait(full_k + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
+      for (int c = wt_mq; c < iss_mq; ++c) mbar_wait(full_mq + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
+    }
+    __syncwarp();
+  } else {
+    // ======================== state and output warps ========================
+    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q4) << 16) + 32 * ch;
+    write_h();
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(h_ready);
 
-  // bounded wait shared by one role's 128 threads (its leader polls)
-  auto role_wait = [&](uint32_t bar, uint32_t parity, bool is_leader, uint32_t id) {
-    bool fine = true;
-    if (is_leader) fine = mbar_wait(bar, parity, p.err);
-    fine = !named_sync_or(id, 128, !fine);
-    tc_fence_after();
-    return fine;
-  };
-
-  for (int cw = 0; cw < nw; ++cw) {
-    const int s = cw & 1;
-    const uint32_t st = sbase + s * C_STAGE;
-    const int t0 = seq_start + (p.win0 + cw) * C;
-    const int L = min(C, seq_end - t0);
-    const uint8_t *rec = ws_record(p, n, h, cw);
-    const float *sc = reinterpret_cast<const float *>(rec + WS_SC);
-    // this thread's Ut columns (state rows) and per-row scalars, fetched early
+    // per-chunk data read into registers one chunk ahead: Ut (state rows) and scalars
     float ut[32];
-    if (wrow) {
-      const float4 *src = reinterpret_cast<const float4 *>(rec + WS_UT + (static_cast<size_t>(slice) * 64 + r) * 256);
+    auto load_ut = [&](int cw) {
+      const float4 *src = reinterpret_cast<const float4 *>(ws_record(p, n, h, cw) + WS_UT +
+                                                           (static_cast<size_t>(slice) * 64 + r) * 256);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const float4 v4 = src[(8 * ch + j) ^ (r & 7)];
         ut[4 * j] = v4.x; ut[4 * j + 1] = v4.y; ut[4 * j + 2] = v4.z; ut[4 * j + 3] = v4.w;
       }
+    };
+    float nx_g = 0.0f, nx_s = 0.0f, nx_gL = 0.0f;   // gamma_r, 1/|k_r| or 1/|q_r|, gamma_(L-1)
+    auto load_sc = [&](int cw) {
+      const float *sc = reinterpret_cast<const float *>(ws_record(p, n, h, cw) + WS_SC);
+      nx_g = sc[r];
+      nx_s = wrow ? sc[128 + r] : sc[64 + r];
+      nx_gL = sc[63];
+    };
+    if (nw > 0) {
+      load_sc(0);
+      if (wrow) load_ut(0);
     }
-    const float g_r = sc[r];
-    const float scal_b = wrow ? sc[128 + r] : sc[64 + r];   // 1/|k_r| or 1/|q_r|
-    const float gL = sc[63];                                // padding rows carry gamma_{L-1}
-    PTIME(1 + cw, 0);
-    if (!(ok = cta_wait(bar_full + 8 * s, (cw >> 1) & 1, p.err))) break;
-    PTIME(1 + cw, 1);
 
-    // ---- [Q; W_hi] (H_hi + H_lo) -> P ;  [*; W_lo] H_hi -> P2 (lanes 64..127) -------
-    if (tid == 64) {   // a state-row thread issues the state products
-      const uint32_t id = idesc_bf16(128, 64, false, true);
-      const uint64_t aq = sdesc(st + C_ROW_Q * 128, 16, 1024);
-      const uint64_t aw = sdesc(st + C_ROW_WHI * 128, 16, 1024);
-      const uint64_t bh = sdesc(sbase + C_OFF_H, BLK128, 1024);
+    float oreg[32];   // e^gamma / |q| Q H0 part of o (output rows)
+    for (int cw = 0; cw < nw; ++cw) {
+      const uint32_t ph = cw & 1;
+      const int t0 = t0_of(cw), L = min(C, seq_end - t0);
+      const float g_r = nx_g, sb = nx_s, gL = nx_gL;
+      if (cw + 1 < nw) load_sc(cw + 1);
+      PTIME(1 + cw, 0);
+      if (wrow) {
+        // ---- U = Ut - W H0 and U' = U e^(gamma_L - gamma) / |k| (state rows) ----------------
+        chain_wait(bar_p, ph, abort_flag, p.err);
+        PTIME_T(1 + cw, 22, 64);
+        if (cw > 0) chain_wait(bar_o, ph ^ 1, abort_flag, p.err);   // the last O product read U
+        __syncwarp();
+        tc_fence_after();
+        PTIME_T(1 + cw, 23, 64);
+        const float ed = __expf(gL - g_r) * sb;
 #pragma unroll
-      for (int part = 0; part < 3; ++part) {
-        const uint64_t a0 = part < 2 ? aq : aw;
-        const uint64_t b0 = bh + (part == 1 ? (BLK128 >> 4) : 0);
-        const uint32_t dcol = part < 2 ? C_COL_P : C_COL_P2;
+        for (int hh = 0; hh < 2; ++hh) {
+          float pa[16], pb[16], pc[16];
+          tmem_ld16(tl + C_COL_P + 16 * hh, pa);
+          tmem_ld16(tl + C_COL_P + 64 + 16 * hh, pb);
+          tmem_ld16(tl + C_COL_P2 + 16 * hh, pc);
+          tmem_wait_ld();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * C_KB + (kk & 3) * 32;
-          mma_bf16(tmem + dcol, a0 + (koff >> 4), b0 + ((kk * 2048) >> 4), id, (part == 1) || kk > 0);
-        }
-      }
-      mma_commit(bar_p);
-      PTIME_T(1 + cw, 10, 64);
-    }
-    PTIME(1 + cw, 7);
-    bool good = true;   // this thread's waits succeeded
-    if (!wrow) {
-      // output rows: the previous chunk's output, then its stage takes chunk cw + 1
-      if (cw > 0) {
-        good = role_wait(bar_o, (cw - 1) & 1, tid == 0, BAR_QROWS);
-        if (good && tid == 0 && cw + 1 < nw) load_chunk(cw + 1);
-        PTIME(1 + cw, 8);
-        if (good) finish_output(cw - 1);
-        PTIME(1 + cw, 9);
-      }
-      PTIME(1 + cw, 2);
-      good = role_wait(bar_p, cw & 1, tid == 0, BAR_QROWS) && good;
-      if (good) {   // Q H0 part of o
-        const float f = p.scale * __expf(g_r) * scal_b;
-        tmem_ld32(tl + C_COL_P, oreg);
-        tmem_wait_ld();
+          for (int c4 = 0; c4 < 2; ++c4) {
+            float u[8], us[8];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) oreg[j] *= f;
-      }
-    } else {
-      // the previous output product must be done reading the U tiles
-      if (cw > 0) good = role_wait(bar_o, (cw - 1) & 1, tid == 64, BAR_WROWS);
-      good = role_wait(bar_p, cw & 1, tid == 64, BAR_WROWS) && good;
-      PTIME_T(1 + cw, 11, 64);
-      // ---- U = Ut - W H0 and U' = U e^(gL - g) / |k| ---------------------------------
-      if (good) {
-        const float ed = __expf(gL - g_r) * scal_b;
-        float pw[32], pl[32];
-        tmem_ld32(tl + C_COL_P, pw);
-        tmem_ld32(tl + C_COL_P2, pl);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float u[8], us[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            u[e] = ut[8 * c4 + e] - pw[8 * c4 + e] - pl[8 * c4 + e];
-            us[e] = u[e] * ed;
+            for (int e = 0; e < 8; ++e) {
+              const int j = 8 * c4 + e;
+              u[e] = ((ut[16 * hh + j] - pa[j]) - pb[j]) - pc[j];
+              us[e] = u[e] * ed;
+            }
+            const uint32_t off = sw128(r, 4 * ch + 2 * hh + c4);
+            uint4 hi, lo;
+            split8x2(u, hi, lo);
+            st_shared16(sbase + C_OFF_U + off, hi);
+            st_shared16(sbase + C_OFF_U + BLK64 + off, lo);
+            split8x2(us, hi, lo);
+            st_shared16(sbase + C_OFF_U + 2 * BLK64 + off, hi);
+            st_shared16(sbase + C_OFF_U + 3 * BLK64 + off, lo);
           }
-          const uint32_t off = sw128(r, 4 * ch + c4);
-          uint4 hi, lo;
-          split8x2(u, hi, lo);
-          st_shared16(sbase + C_OFF_U + off, hi);
-          st_shared16(sbase + C_OFF_U + BLK64 + off, lo);
-          split8x2(us, hi, lo);
-          st_shared16(sbase + C_OFF_U + 2 * BLK64 + off, hi);
-          st_shared16(sbase + C_OFF_U + 3 * BLK64 + off, lo);
+        }
+        PTIME_T(1 + cw, 24, 64);
+        fence_proxy_async();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(u_ready);
+        PTIME_T(1 + cw, 12, 64);
+        if (cw + 1 < nw) load_ut(cw + 1);
+      } else {
+        // ---- Q H0 part of the output (output rows) ------------------------------------------
+        chain_wait(bar_p, ph, abort_flag, p.err);
+        __syncwarp();
+        tc_fence_after();
+        const float f = p.scale * __expf(g_r) * sb;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float pa[16], pb[16];
+          tmem_ld16(tl + C_COL_P + 16 * hh, pa);
+          tmem_ld16(tl + C_COL_P + 64 + 16 * hh, pb);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) oreg[16 * hh + j] = (pa[j] + pb[j]) * f;
         }
       }
-      PTIME_T(1 + cw, 12, 64);
-      // the U tiles are complete among the state-row warps
+
+      // ---- H <- e^gamma_L H + K^T U' ------------------------------------------------------------
+      chain_wait(bar_h, ph, abort_flag, p.err);
+      __syncwarp();
+      tc_fence_after();
+      PTIME(1 + cw, 5);
+      PTIME_T(1 + cw, 16, 64);
+      PTIME_T(1 + cw, 17, 224);
+      {
+        const float eL = __expf(gL);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float ha[16], hb[16];
+          tmem_ld16(tl + C_COL_H + 16 * hh, ha);
+          tmem_ld16(tl + C_COL_H + 64 + 16 * hh, hb);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) hreg[16 * hh + j] = eL * hreg[16 * hh + j] + (ha[j] + hb[j]);
+        }
+        write_h();
+      }
+      PTIME(1 + cw, 18);
+      PTIME_T(1 + cw, 19, 64);
       fence_proxy_async();
       tc_fence_before();
-      named_sync(BAR_WROWS, 128);
-      PTIME_T(1 + cw, 13, 64);
-    }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(h_ready);
+      PTIME(1 + cw, 6);
+      PTIME_T(1 + cw, 20, 64);
+      PTIME_T(1 + cw, 21, 224);
 
-    PTIME(1 + cw, 4);
-    // ---- K^T U' (hi/lo) -> H part, issued by thread 64 and waited on;
-    //      Mq U (hi/lo x hi/lo) -> o part, issued by thread 96, waited on next chunk
-    if (tid == 64) {
-      tc_fence_after();
-      const uint32_t idH = idesc_bf16(128, 64, true, true);
-      const uint64_t ak = sdesc(st + C_ROW_K * 128, C_KB, 1024);
-      const uint64_t bu = sdesc(sbase + C_OFF_U, BLK64, 1024);
+      // ---- output rows: o = scale (e^gamma / |q| Q H0 + O), overlapping the next chunk ---------
+      if (!wrow) {
+        chain_wait(bar_o, ph, abort_flag, p.err);
+        __syncwarp();
+        tc_fence_after();
 #pragma unroll
-      for (int part = 0; part < 2; ++part)
+        for (int hh = 0; hh < 2; ++hh) {
+          float oa[16], ob[16];
+          tmem_ld16(tl + C_COL_O + 16 * hh, oa);
+          tmem_ld16(tl + C_COL_O + 64 + 16 * hh, ob);
+          tmem_wait_ld();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + C_COL_H, ak + ((kk * 2048) >> 4), bu + (((2 + part) * BLK64 + kk * 2048) >> 4),
-                   idH, (part | kk) != 0);
-      mma_commit(bar_h);
-      PTIME_T(1 + cw, 14, 64);
-    } else if (tid == 96) {
-      tc_fence_after();
-      const uint32_t idO = idesc_bf16(128, 64, false, true);
-      const uint64_t bu = sdesc(sbase + C_OFF_U, BLK64, 1024);
-      const uint64_t am = sdesc(st + C_OFF_MQ, 16, 1024);
+          for (int j = 0; j < 16; ++j) oreg[16 * hh + j] += p.scale * (oa[j] + ob[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_free);
+        if (r < L) {
+          uint16_t *dst = p.o + (static_cast<size_t>(t0 + r) * p.hv + h) * D + slice * N + 32 * ch;
 #pragma unroll
-      for (int part = 0; part < 3; ++part) {   // Mq rows land in lanes 0..63
-        const uint32_t aoff = part < 2 ? 0u : BLK64;      // Mq_hi, Mq_hi, Mq_lo
-        const uint32_t ub = part == 1 ? BLK64 : 0u;       // U_hi, U_lo, U_hi
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + C_COL_O, am + ((aoff + kk * 32) >> 4), bu + ((ub + kk * 2048) >> 4), idO,
-                   (part | kk) != 0);
+          for (int c4 = 0; c4 < 4; ++c4) *reinterpret_cast<uint4 *>(dst + 8 * c4) = pack8x2(oreg + 8 * c4);
+        }
+        PTIME(1 + cw, 7);
       }
-      mma_commit(bar_o);
     }
-    prev_t0 = t0;
-    prev_L = L;
-    if (!(ok = cta_wait(bar_h, cw & 1, p.err, good))) break;
-    PTIME(1 + cw, 5);
-
-    // ---- H <- e^gamma_L H + K^T U' ------------------------------------------------
-    {
-      const float eL = __expf(gL);
-      float rh[32];
-      tmem_ld32(tl + C_COL_H, rh);
-      tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) hreg[j] = eL * hreg[j] + rh[j];
-      write_h();
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    PTIME(1 + cw, 6);
   }
-  if (ok && nw > 0 && cta_wait(bar_o, (nw - 1) & 1, p.err, true)) finish_output(nw - 1);
-  if (p.state_out && ok) {
+  tc_fence_before();
+  __syncthreads();
+  if (!ctrl && p.state_out && *abort_flag == 0u) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4)
       *reinterpret_cast<float4 *>(p.state_out + srow + j) = make_float4(hreg[j], hreg[j + 1], hreg[j + 2], hreg[j + 3]);
   }
-  tc_fence_before();
-  __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, C_TM_COLS);
 }
 

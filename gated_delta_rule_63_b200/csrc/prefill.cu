@@ -53,12 +53,10 @@ constexpr uint32_t BLK64 = 64 * 128;     // one [64 x 64] bf16 tile, 128-B swizz
 // Images are laid out exactly as the chain kernel's shared memory expects.
 constexpr uint32_t WS_W_HI = 0;          // W_hi  [kb 2][64 rows][128 B]
 constexpr uint32_t WS_W_LO = 16384;      // W_lo  [kb 2][64 rows][128 B]
-constexpr uint32_t WS_MQ_HI = 32768;     // Mq_hi [64 rows][128 B]
-constexpr uint32_t WS_MQ_LO = 40960;     // Mq_lo [64 rows][128 B]
+constexpr uint32_t WS_MQ = 32768;        // Mq_lo, Mq_hi: 2 x [64 rows][128 B]
 constexpr uint32_t WS_UT = 49152;        // Ut fp32 [slice 2][64 rows][64], 16-B chunk j of row r at j ^ (r & 7)
 constexpr uint32_t WS_SC = 81920;        // fp32 gamma[64], 1/|q|[64], 1/|k|[64]
 constexpr uint32_t WS_REC = 82944;       // record size (81 KiB)
-static_assert(WS_MQ_LO == WS_MQ_HI + 64 * 128, "Mq_hi and Mq_lo are copied as one block");
 
 // ---- prep kernel -------------------------------------------------------------
 constexpr int kPrepThreads = 256;
@@ -66,11 +64,12 @@ constexpr uint32_t P_KQ_KB = 128 * 128;              // [K rows 0..63 | Q rows 6
 constexpr uint32_t P_OFF_KQ = 0;                     // 2 k-blocks
 constexpr uint32_t P_OFF_V = P_OFF_KQ + 2 * P_KQ_KB; // V [dv block 2][64 rows][128 B]
 constexpr uint32_t P_OFF_T = P_OFF_V + 2 * BLK64;    // T'_hi, T'_lo, T''_hi, T''_lo
-constexpr int LD = 65;                               // fp32 row stride of AT
+constexpr int LD = 68;                               // fp32 row stride of AT (rows 16-byte aligned)
+constexpr int XLD = 20;                              // fp32 row stride of the X^T blocks
 constexpr uint32_t P_OFF_AT = P_OFF_T + 4 * BLK64;   // A below / T^T on and above the diagonal
 constexpr uint32_t P_OFF_XF = P_OFF_AT + 64 * LD * 4;
-constexpr uint32_t P_OFF_SC = P_OFF_XF + 3 * 256 * 4;  // gamma, rq, rk, beta, e^gamma, block decay
-constexpr uint32_t P_OFF_BAR = P_OFF_SC + 6 * 64 * 4;
+constexpr uint32_t P_OFF_SC = P_OFF_XF + 3 * 16 * XLD * 4;  // gamma, rq, rk, beta, e^gamma, block decay, e^g
+constexpr uint32_t P_OFF_BAR = P_OFF_SC + 7 * 64 * 4;
 constexpr uint32_t P_SMEM = P_OFF_BAR + 32 + 1024;
 static_assert((P_OFF_V | P_OFF_T) % 1024 == 0, "swizzled tiles need 1 KB alignment");
 constexpr uint32_t P_TM_COLS = 256;                  // two prep CTAs per SM
@@ -80,8 +79,8 @@ constexpr uint32_t P_COL_X = 128;                    // W, then Ut (128 cols)
 // ---- chain kernel ------------------------------------------------------------
 constexpr int kChainThreads = 288;                    // warps 0..7 state and output, warp 8 control
 constexpr int kCtrlWarp = 8;
-// stage: per k-block the rows [Q 0..63 | W_hi 64..127 | W_lo 128..191] (A operands
-// [Q; W_hi] and [W_hi; W_lo]), then K (two dk blocks), then [Mq_hi; Mq_lo]
+// stage: per k-block the rows [W_lo 0..63 | W_hi 64..127 | Q 128..191] (A operands
+// [W_lo; W_hi] and [W_hi; Q]), then K (two dk blocks), then [Mq_lo; Mq_hi]
 constexpr uint32_t C_QW_KB = 192 * 128;
 constexpr uint32_t C_OFF_K = 2 * C_QW_KB;
 constexpr uint32_t C_OFF_MQ = C_OFF_K + 2 * BLK64;
@@ -95,10 +94,10 @@ static_assert(C_SMEM <= 232448, "chain shared memory exceeds 227 KB");
 static_assert((C_QW_KB | C_OFF_K | C_OFF_MQ | C_STAGE | C_OFF_H | C_OFF_U) % 1024 == 0,
               "swizzled tiles need 1 KB alignment");
 constexpr uint32_t C_TM_COLS = 512;
-constexpr uint32_t C_COL_P = 0;      // [Q; W_hi] [H_hi | H_lo]: lanes 0..63 Q rows, 64..127 W rows
-constexpr uint32_t C_COL_P2 = 128;   // [W_hi; W_lo] H_hi: lanes 64..127 hold W_lo H_hi
+constexpr uint32_t C_COL_P = 0;      // [W_hi; Q] [H_hi | H_lo]: lanes 0..63 W rows, 64..127 Q rows
+constexpr uint32_t C_COL_P2 = 128;   // [W_lo; W_hi] H_hi: lanes 0..63 hold W_lo H_hi
 constexpr uint32_t C_COL_H = 256;    // K^T [U'_hi | U'_lo], lanes = dk
-constexpr uint32_t C_COL_O = 384;    // [Mq_hi; Mq_lo] [U_hi | U_lo] + Mq_lo U_hi, lanes 0..63
+constexpr uint32_t C_COL_O = 384;    // [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi, lanes 64..127
 
 #ifdef GDR_PREFILL_TIMING
 // diagnostic build: step timestamps; prep CTA (0,0,0) in row 0, chain CTA
@@ -184,6 +183,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   float *XF = reinterpret_cast<float *>(smem + P_OFF_XF);
   float *s_g = reinterpret_cast<float *>(smem + P_OFF_SC);
   float *s_rq = s_g + 64, *s_rk = s_g + 128, *s_beta = s_g + 192, *s_eg = s_g + 256, *s_eb = s_g + 320;
+  float *s_e1 = s_g + 384;   // e^(g_t): one step of decay
   const uint32_t bar_tma = sbase + P_OFF_BAR, bar_mma = sbase + P_OFF_BAR + 8;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + P_OFF_BAR + 16);
   uint8_t *rec = ws_record(p, n, h, cw);
@@ -263,6 +263,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (tid < 64) {
       s_eg[tid] = __expf(s_g[tid]);
       s_eb[tid] = __expf(s_g[tid | 15] - s_g[tid]);   // decay to the end of the 16-block
+      s_e1[tid] = __expf(g);
       float *sc = reinterpret_cast<float *>(rec + WS_SC);
       sc[tid] = s_g[tid];
       sc[64 + tid] = s_rq[tid];
@@ -297,26 +298,31 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // per-column factors of this thread's 32 columns: 1/|k_j| and the decay e^(g_i - g_j)
     const int i = row & 63, ib = i >> 4;
     const float gi = s_g[i];
+    // e^(g_i - g_j): for a whole earlier 16-block as e^(g_i - g_end) e^(g_end - g_j) (both <= 1);
+    // inside the row's own block as a backward running product of one-step decays e^(g_t)
     float colf[32];
 #pragma unroll
     for (int b2 = 0; b2 < 2; ++b2) {
       const int blk = 2 * hf + b2;
-      const float fi = __expf(gi - s_g[blk * 16 + 15]);   // used for whole earlier blocks only
+      const float fi = __expf(gi - s_g[blk * 16 + 15]);   // used for blocks before the row's own only
+      float dg[16];
+      float run = 0.0f;
+#pragma unroll
+      for (int e = 15; e >= 0; --e) {
+        const int j = blk * 16 + e;
+        run = (j == i) ? 1.0f : (e == 15 ? 0.0f : run * s_e1[j + 1]);   // zero above the diagonal
+        dg[e] = run;
+      }
 #pragma unroll
       for (int e4 = 0; e4 < 4; ++e4) {
         const int j0 = blk * 16 + 4 * e4;
         const float4 rk4 = *reinterpret_cast<const float4 *>(s_rk + j0);
-        const float4 g4 = *reinterpret_cast<const float4 *>(s_g + j0);
         const float4 eb4 = *reinterpret_cast<const float4 *>(s_eb + j0);
         const float rkv[4] = {rk4.x, rk4.y, rk4.z, rk4.w};
-        const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
         const float ebv[4] = {eb4.x, eb4.y, eb4.z, eb4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int j = j0 + e;
-          float dec;
-          if (blk < ib) dec = fi * ebv[e];
-          else dec = j <= i ? __expf(gi - gv[e]) : 0.0f;
+          const float dec = blk < ib ? fi * ebv[e] : dg[4 * e4 + e];
           colf[b2 * 16 + 4 * e4 + e] = rkv[e] * dec;
         }
       }
@@ -325,12 +331,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + P_COL_S + 32 * hf, sv);
     tmem_wait_ld();
     if (row < 64) {   // A_ij = beta_i / |k_i| * (k_i.k_j) / |k_j| * e^(g_i - g_j), j < i
+      // (columns j >= i hold junk until T^T overwrites them)
       const float bi = s_beta[i] * s_rk[i];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int j = 32 * hf + e;
-        if (j < i) AT[i * LD + j] = bi * sv[e] * colf[e];
-      }
+      for (int c4 = 0; c4 < 8; ++c4)
+        *reinterpret_cast<float4 *>(AT + i * LD + 32 * hf + 4 * c4) =
+            make_float4(bi * sv[4 * c4] * colf[4 * c4], bi * sv[4 * c4 + 1] * colf[4 * c4 + 1],
+                        bi * sv[4 * c4 + 2] * colf[4 * c4 + 2], bi * sv[4 * c4 + 3] * colf[4 * c4 + 3]);
     } else {          // Mq_ij = (q_i.k_j) / (|q_i| |k_j|) * e^(g_i - g_j), j <= i
       const float qi = s_rq[i];
 #pragma unroll
@@ -339,14 +346,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
         for (int e = 0; e < 8; ++e) m[e] = sv[8 * c4 + e] * qi * colf[8 * c4 + e];
         const uint32_t off = sw128(i, 4 * hf + c4);   // staged in the T region, stored in bulk
-        st_split8_shared(sbase + P_OFF_T + off, sbase + P_OFF_T + BLK64 + off, m);
+        st_split8_shared(sbase + P_OFF_T + BLK64 + off, sbase + P_OFF_T + off, m);   // [Mq_lo | Mq_hi]
       }
     }
     PTIME(0, 12);
     fence_proxy_async();
     __syncthreads();
-    if (tid == 0) {   // Mq_hi | Mq_lo, contiguous in shared memory and in the record
-      bulk_store(rec + WS_MQ_HI, sbase + P_OFF_T, 2 * BLK64);
+    if (tid == 0) {   // Mq_lo | Mq_hi, contiguous in shared memory and in the record
+      bulk_store(rec + WS_MQ, sbase + P_OFF_T, 2 * BLK64);
       bulk_commit();
     }
 
@@ -368,28 +375,62 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     PTIME(0, 13);
     __syncthreads();
-    for (int d = 1; d < 4; ++d) {   // T_bc = -T_bb sum_{m=c}^{b-1} A_bm T_mc, b - c = d
+    // off-diagonal blocks by diagonals d = b - c: X_bc = sum_{m=c}^{b-1} A_bm T_mc, T_bc = -T_bb X_bc.
+    // Each block is computed by 64 threads holding 2 x 2 tiles (rows rt, rt + 8; columns jt, jt + 8);
+    // A rows and T^T rows are read as float4 along k.
+    for (int d = 1; d < 4; ++d) {
       const int nb = 4 - d;
-      for (int e = tid; e < nb * 256; e += kPrepThreads) {
-        const int blk = e >> 8, bb = d + blk, cb = bb - d, r = (e >> 4) & 15, j = e & 15;
-        float sacc = 0.0f;
-        for (int m = cb; m < bb; ++m) {
+      const int blk = tid >> 6, t = tid & 63, rt = t >> 3, jt = t & 7;
+      const int bb = d + blk, cb = blk;
+      if (blk < nb) {   // X_bc^T[j][r] into XF
+        const float *a0 = AT + (16 * bb + rt) * LD, *a1 = a0 + 8 * LD;
+        const float *t0 = AT + (16 * cb + jt) * LD, *t1 = t0 + 8 * LD;   // T^T rows = columns of T
+        float x00 = 0.0f, x01 = 0.0f, x10 = 0.0f, x11 = 0.0f;         // x[r][j] for r in {rt, rt+8}, j in {jt, jt+8}
 #pragma unroll
-          for (int l = 0; l < 16; ++l) {
-            const float t = (m > cb || l >= j) ? AT[(16 * cb + j) * LD + 16 * m + l] : 0.0f;
-            sacc += AT[(16 * bb + r) * LD + 16 * m + l] * t;
+        for (int g = 0; g < 4; ++g) {   // block m = c: T[16c + l][16c + j] is zero for l < j
+          const int k = 16 * cb + 4 * g;
+          const float4 A0 = *reinterpret_cast<const float4 *>(a0 + k), A1 = *reinterpret_cast<const float4 *>(a1 + k);
+          const float4 T0 = *reinterpret_cast<const float4 *>(t0 + k), T1 = *reinterpret_cast<const float4 *>(t1 + k);
+          const float av0[4] = {A0.x, A0.y, A0.z, A0.w}, av1[4] = {A1.x, A1.y, A1.z, A1.w};
+          const float tv0[4] = {T0.x, T0.y, T0.z, T0.w}, tv1[4] = {T1.x, T1.y, T1.z, T1.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float u0 = (4 * g + e >= jt) ? tv0[e] : 0.0f, u1 = (4 * g + e >= jt + 8) ? tv1[e] : 0.0f;
+            x00 += av0[e] * u0; x01 += av0[e] * u1;
+            x10 += av1[e] * u0; x11 += av1[e] * u1;
           }
         }
-        XF[e] = sacc;
+        for (int k = 16 * (cb + 1); k < 16 * bb; k += 4) {
+          const float4 A0 = *reinterpret_cast<const float4 *>(a0 + k), A1 = *reinterpret_cast<const float4 *>(a1 + k);
+          const float4 T0 = *reinterpret_cast<const float4 *>(t0 + k), T1 = *reinterpret_cast<const float4 *>(t1 + k);
+          x00 += A0.x * T0.x + A0.y * T0.y + A0.z * T0.z + A0.w * T0.w;
+          x01 += A0.x * T1.x + A0.y * T1.y + A0.z * T1.z + A0.w * T1.w;
+          x10 += A1.x * T0.x + A1.y * T0.y + A1.z * T0.z + A1.w * T0.w;
+          x11 += A1.x * T1.x + A1.y * T1.y + A1.z * T1.z + A1.w * T1.w;
+        }
+        float *xt = XF + (blk * 16 + jt) * XLD;
+        xt[rt] = x00;
+        xt[rt + 8] = x10;
+        xt[8 * XLD + rt] = x01;
+        xt[8 * XLD + rt + 8] = x11;
       }
       __syncthreads();
-      for (int e = tid; e < nb * 256; e += kPrepThreads) {
-        const int blk = e >> 8, bb = d + blk, cb = bb - d, r = (e >> 4) & 15, j = e & 15;
-        float sacc = 0.0f;
+      if (blk < nb) {   // T_bc[r][j] = -sum_{l <= r} T_bb[r][l] X_bc[l][j], stored as T^T
+        const float *xa = XF + (blk * 16 + jt) * XLD, *xb = xa + 8 * XLD;
+        const float *tb = AT + (16 * bb) * LD + 16 * bb;               // tb[l * LD + r] = T_bb[r][l]
+        float y00 = 0.0f, y01 = 0.0f, y10 = 0.0f, y11 = 0.0f;         // y[r][j]
 #pragma unroll
-        for (int l = 0; l < 16; ++l)
-          if (l <= r) sacc -= AT[(16 * bb + l) * LD + 16 * bb + r] * XF[(blk << 8) + l * 16 + j];
-        AT[(16 * cb + j) * LD + 16 * bb + r] = sacc;
+        for (int l = 0; l < 16; ++l) {
+          const float t0v = l <= rt ? tb[l * LD + rt] : 0.0f, t1v = l <= rt + 8 ? tb[l * LD + rt + 8] : 0.0f;
+          const float x0 = xa[l], x1 = xb[l];
+          y00 -= t0v * x0; y01 -= t0v * x1;
+          y10 -= t1v * x0; y11 -= t1v * x1;
+        }
+        float *dst = AT + (16 * cb + jt) * LD + 16 * bb;
+        dst[rt] = y00;
+        dst[rt + 8] = y10;
+        dst[8 * LD + rt] = y01;
+        dst[8 * LD + rt + 8] = y11;
       }
       __syncthreads();
       PTIME(0, 13 + d);
@@ -399,19 +440,23 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // ---- T' = T diag(beta e^g / |k|), T'' = T diag(beta), hi/lo tiles --------
     if (tid == 0) bulk_wait_read();   // the Mq staging is about to be overwritten
     __syncthreads();
-    {
-      const int r = tid >> 2, qc = tid & 3;   // row r, columns 16 qc .. 16 qc + 15
+    {   // tiles with the row index r contiguous (MN-major operands): row j, 16-byte chunk r / 8
+      const int j = tid & 63;
+      const float f2 = s_beta[j], f1 = f2 * s_eg[j] * s_rk[j];
 #pragma unroll
-      for (int h8 = 0; h8 < 2; ++h8) {
+      for (int h = 0; h < 2; ++h) {
+        const int rg = (tid >> 6) + 4 * h, r0 = 8 * rg;
+        const float4 v0 = *reinterpret_cast<const float4 *>(AT + j * LD + r0);
+        const float4 v1 = *reinterpret_cast<const float4 *>(AT + j * LD + r0 + 4);
+        const float tv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         float t1[8], t2[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int j = 16 * qc + 8 * h8 + e;
-          const float tij = (j <= r) ? AT[j * LD + r] : 0.0f;
-          t2[e] = tij * s_beta[j];
-          t1[e] = t2[e] * s_eg[j] * s_rk[j];
+          const float tij = (r0 + e >= j) ? tv[e] : 0.0f;   // T[r][j], lower triangle
+          t1[e] = tij * f1;
+          t2[e] = tij * f2;
         }
-        const uint32_t off = sw128(r, 2 * qc + h8);
+        const uint32_t off = sw128(j, rg);
         st_split8_shared(sbase + P_OFF_T + off, sbase + P_OFF_T + BLK64 + off, t1);
         st_split8_shared(sbase + P_OFF_T + 2 * BLK64 + off, sbase + P_OFF_T + 3 * BLK64 + off, t2);
       }
@@ -420,15 +465,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
 
     PTIME(0, 6);
-    // ---- W = T' K  (A rows 64..127 are junk; only lanes 0..63 are read) -------
+    // ---- W = T' K  (A rows 64..127 are the next tile: junk lanes, never read) ---
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 128, false, true);
+      const uint32_t id = idesc_bf16(128, 128, true, true);
 #pragma unroll
       for (int part = 0; part < 2; ++part)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + P_COL_X, sdesc(sbase + P_OFF_T + part * BLK64 + kk * 32, 16, 1024),
+          mma_bf16(tmem + P_COL_X, sdesc(sbase + P_OFF_T + part * BLK64 + kk * 2048, BLK64, 1024),
                    sdesc(sbase + P_OFF_KQ + kk * 2048, P_KQ_KB, 1024), id, (part | kk) != 0);
       mma_commit(bar_mma);
     }
@@ -460,12 +505,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       bulk_store(rec + WS_W_HI, sbase + P_OFF_KQ, 4 * BLK64);
       bulk_commit();
       tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 128, false, true);
+      const uint32_t id = idesc_bf16(128, 128, true, true);
 #pragma unroll
       for (int part = 0; part < 2; ++part)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + P_COL_X, sdesc(sbase + P_OFF_T + (2 + part) * BLK64 + kk * 32, 16, 1024),
+          mma_bf16(tmem + P_COL_X, sdesc(sbase + P_OFF_T + (2 + part) * BLK64 + kk * 2048, BLK64, 1024),
                    sdesc(sbase + P_OFF_V + kk * 2048, BLK64, 1024), id, (part | kk) != 0);
       mma_commit(bar_mma);
     }
@@ -510,12 +555,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // H (128 dk rows x 64 dv columns) stays in registers of warps 0..7: warp w
 // holds rows 32 (w & 3) .. + 31 (its TMEM lane quarter), columns
 // 32 (w >> 2) .. + 31.  Per chunk:
-//   P  = [Q; W_hi] [H_hi | H_lo],  P2 = [W_hi; W_lo] H_hi          tensor cores
-//   U  = Ut - W H0,  U' = U e^(gamma_L - gamma) / |k|                warps 2, 3, 6, 7 (lanes 64..127)
+//   P  = [W_hi; Q] [H_hi | H_lo],  P2 = [W_lo; W_hi] H_hi          tensor cores
+//   U  = Ut - W H0,  U' = U e^(gamma_L - gamma) / |k|                warps 0, 1, 4, 5 (lanes 0..63)
 //   H' = K^T [U'_hi | U'_lo]                                         tensor cores
 //   H  = e^gamma_L H + H'                                            warps 0..7
-//   O  = [Mq_hi; Mq_lo] [U_hi | U_lo] + Mq_lo U_hi                   tensor cores
-//   o  = scale (e^gamma / |q| Q H0 + O)                              warps 0, 1, 4, 5 (lanes 0..63)
+//   O  = [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi              tensor cores
+//   o  = scale (e^gamma / |q| Q H0 + O)                              warps 2, 3, 6, 7 (lanes 64..127)
 // N = 128 products stack the hi and lo parts of one operand side by side, so
 // each fp32 product takes two MMA groups instead of three.  Warp 8 issues every
 // product and every copy and does nothing else; the roles meet only on
@@ -580,9 +625,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     mbar_arrive_expect_tx(fb, 6 * BLK64);
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb) {
-      tma_load_2d(st + kb * C_QW_KB, &tm_q, kh * D + kb * 64, t0_of(cw), fb);
+      bulk_load(st + kb * C_QW_KB, rec + WS_W_LO + kb * BLK64, BLK64, fb);
       bulk_load(st + kb * C_QW_KB + 64 * 128, rec + WS_W_HI + kb * BLK64, BLK64, fb);
-      bulk_load(st + kb * C_QW_KB + 128 * 128, rec + WS_W_LO + kb * BLK64, BLK64, fb);
+      tma_load_2d(st + kb * C_QW_KB + 128 * 128, &tm_q, kh * D + kb * 64, t0_of(cw), fb);
     }
     iss_qw = cw + 1;
   };
@@ -593,10 +638,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     for (int kb = 0; kb < 2; ++kb) tma_load_2d(st + C_OFF_K + kb * BLK64, &tm_k, kh * D + kb * 64, t0_of(cw), fb);
     iss_k = cw + 1;
   };
-  auto load_mq = [&](int cw) {   // Mq_hi | Mq_lo are contiguous in the record
+  auto load_mq = [&](int cw) {   // Mq_lo | Mq_hi are contiguous in the record
     const uint32_t st = sbase + (cw & 1) * C_STAGE, fb = full_mq + 8 * (cw & 1);
     mbar_arrive_expect_tx(fb, 2 * BLK64);
-    bulk_load(st + C_OFF_MQ, ws_record(p, n, h, cw) + WS_MQ_HI, 2 * BLK64, fb);
+    bulk_load(st + C_OFF_MQ, ws_record(p, n, h, cw) + WS_MQ, 2 * BLK64, fb);
     iss_mq = cw + 1;
   };
   if (ctrl && lane == 0) {
@@ -615,7 +660,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   }
   const int q4 = warp & 3, ch = (warp >> 2) & 1;     // lane quarter, column half
   const int row = 32 * q4 + lane;                    // TMEM lane / dk row of the state
-  const bool wrow = row >= 64;                       // W rows (state side) vs Q rows (output side)
+  const bool wrow = row < 64;                        // W rows (state side) vs Q rows (output side)
   const int r = row & 63;                            // chunk row
 
   // ---- the state: row `row`, columns 32 ch .. 32 ch + 31 of this dv slice --------------
@@ -665,17 +710,20 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const uint32_t id1 = idesc_bf16(128, 128, false, true), id2 = idesc_bf16(128, 64, false, true);
         const uint64_t bh = sdesc(sbase + C_OFF_H, BLK128, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * C_QW_KB + (kk & 3) * 32;
+        for (int kk = 0; kk < 8; ++kk) {   // A = rows [W_hi; Q]
+          const uint32_t aoff = (kk >> 2) * C_QW_KB + 64 * 128 + (kk & 3) * 32;
           mma_bf16(tmem + C_COL_P, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id1, kk > 0);
         }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * C_QW_KB + 64 * 128 + (kk & 3) * 32;
+        for (int kk = 0; kk < 8; ++kk) {   // A = rows [W_lo; W_hi]
+          const uint32_t aoff = (kk >> 2) * C_QW_KB + (kk & 3) * 32;
           mma_bf16(tmem + C_COL_P2, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id2, kk > 0);
         }
         mma_commit(bar_p);
       }
+      // chunk cw + 1's K goes to the stage of chunk cw - 1, whose K^T U' is complete (every
+      // warp passed it before h_ready); issued here, after P, to keep P off the copy issue
+      if (lane == 0 && cw >= 1 && cw + 1 < nw) load_k(cw + 1);
       __syncwarp();
       PTIME_T(1 + cw, 1, 32 * kCtrlWarp);
       chain_wait(bar_p, ph, abort_flag, p.err);
@@ -699,7 +747,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       }
       __syncwarp();
       PTIME_T(1 + cw, 4, 32 * kCtrlWarp);
-      // ---- O = [Mq_hi; Mq_lo] [U_hi | U_lo] + Mq_lo U_hi (rows in lanes 0..63) ----------------
+      // ---- O = [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi (rows in lanes 64..127) ----------
       if (cw > 0) {
         chain_wait(o_free, ph ^ 1, abort_flag, p.err);   // the previous O is read ...
         PTIME_T(1 + cw, 13, 32 * kCtrlWarp);
@@ -717,15 +765,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO1, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + BLK64 + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO2, 1);
+          mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ - BLK64 + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO2, 1);
         mma_commit(bar_o);
       }
       __syncwarp();
       PTIME_T(1 + cw, 9, 32 * kCtrlWarp);
-      chain_wait(bar_h, ph, abort_flag, p.err);
-      PTIME_T(1 + cw, 10, 32 * kCtrlWarp);
-      if (lane == 0 && cw + 2 < nw) load_k(cw + 2);    // K^T U' has read this stage's K
-      __syncwarp();
     }
     if (lane == 0) {
       // every product completes before tensor memory is released; after a
@@ -886,7 +930,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) *reinterpret_cast<uint4 *>(dst + 8 * c4) = pack8x2(oreg + 8 * c4);
         }
-        PTIME(1 + cw, 7);
+        PTIME_T(1 + cw, 7, 64);
       }
     }
   }

@@ -20,7 +20,7 @@ namespace gdr {
 namespace {
 
 constexpr int kThreads = 128;   // threads per block; 8 channels each
-constexpr int kTokens = 8;      // tokens per run
+constexpr int kTokens = 16;     // tokens per run
 
 struct ConvParams {
   const uint16_t *x;
@@ -44,10 +44,15 @@ __device__ int seq_of(const int32_t *cu, int n_seqs, int t) {
   return lo;
 }
 
-// Each thread: 8 channels x kTokens tokens.  All kTokens + 3 input rows are
-// loaded up front (independent 16-byte loads in flight), then each output
-// takes its taps from the rows of its own sequence, from the conv state or
-// zero before the sequence start.
+// unpack the 8 bf16 of a 16-byte row into floats (one integer op each)
+__device__ __forceinline__ void row8(const uint4 &u, float *f) { unpack8(u, f); }
+
+// Each thread: 8 channels x kTokens tokens.  A run that lies inside one
+// sequence (the common case) loads all kTokens + 3 input rows up front
+// (independent 16-byte loads in flight) and unpacks every row once into a
+// sliding window of four; a run that touches a sequence start or end takes
+// the general path, whose taps come from the rows of their own sequence, from
+// the conv state, or are zero.
 __global__ void __launch_bounds__(kThreads) causal_conv_kernel(ConvParams p) {
   const int C = p.channels;
   const int c0 = (blockIdx.x * kThreads + threadIdx.x) * 8;   // first channel of this thread
@@ -68,13 +73,6 @@ __global__ void __launch_bounds__(kThreads) causal_conv_kernel(ConvParams p) {
   if (t_begin >= p.total) return;
   const int t_end = min(t_begin + kTokens, p.total);
 
-  uint4 raw[kTokens + 3];   // rows t_begin - 3 .. t_begin + kTokens - 1
-#pragma unroll
-  for (int i = 0; i < kTokens + 3; ++i) {
-    const int pos = t_begin - 3 + i;
-    raw[i] = (pos >= 0 && pos < t_end) ? __ldg(reinterpret_cast<const uint4 *>(p.x + static_cast<size_t>(pos) * C + c0))
-                                       : make_uint4(0, 0, 0, 0);
-  }
   float w[4][8];
   {
     // w is [C][4]: channels c0..c0+7 occupy 32 contiguous bf16
@@ -90,7 +88,32 @@ __global__ void __launch_bounds__(kThreads) causal_conv_kernel(ConvParams p) {
   int n = seq_of(p.cu, p.n_seqs, t_begin);
   int seq_start = __ldg(p.cu + n), seq_end = __ldg(p.cu + n + 1);
 
+  if (t_begin - 3 >= seq_start && t_begin + kTokens < seq_end) {
+    // ---- inside one sequence, not its last token: no state, no boundary ----
+    uint4 raw[kTokens + 3];   // rows t_begin - 3 .. t_begin + kTokens - 1
 #pragma unroll
+    for (int i = 0; i < kTokens + 3; ++i)
+      raw[i] = __ldg(reinterpret_cast<const uint4 *>(p.x + static_cast<size_t>(t_begin - 3 + i) * C + c0));
+    float xw[4][8];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) row8(raw[j], xw[j]);
+#pragma unroll
+    for (int i = 0; i < kTokens; ++i) {
+      row8(raw[i + 3], xw[(i + 3) & 3]);
+      float out[8];
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const float acc = w[0][ch] * xw[i & 3][ch] + w[1][ch] * xw[(i + 1) & 3][ch] +
+                          w[2][ch] * xw[(i + 2) & 3][ch] + w[3][ch] * xw[(i + 3) & 3][ch];
+        out[ch] = silu_fast(acc);
+      }
+      *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(t_begin + i) * C + c0) = pack8x2(out);
+    }
+    return;
+  }
+
+  // ---- general path: sequence starts / ends inside the run ----
+#pragma unroll 1
   for (int i = 0; i < kTokens; ++i) {
     const int t = t_begin + i;
     if (t >= t_end) break;
@@ -105,31 +128,32 @@ __global__ void __launch_bounds__(kThreads) causal_conv_kernel(ConvParams p) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int pos = t - 3 + j;
-      float xv[8];
-      if (pos >= seq_start) {
-        unpack8(raw[i + j], xv);
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (pos >= seq_start) {   // (re-read: this path is rare and the row sits in L1 / L2)
+        v = __ldg(reinterpret_cast<const uint4 *>(p.x + static_cast<size_t>(pos) * C + c0));
       } else if (p.cs_in) {   // before the sequence start: the conv state, oldest first
         const int slot = 3 - (seq_start - pos);   // 1..3 positions before the start
-        unpack8(*reinterpret_cast<const uint4 *>(p.cs_in + (static_cast<size_t>(n) * 3 + slot) * C + c0), xv);
-      } else {
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) xv[ch] = 0.0f;
+        v = *reinterpret_cast<const uint4 *>(p.cs_in + (static_cast<size_t>(n) * 3 + slot) * C + c0);
       }
+      float xv[8];
+      unpack8(v, xv);
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) acc[ch] += w[j][ch] * xv[ch];
     }
     float out[8];
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) out[ch] = silu_f(acc[ch]);
-    *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(t) * C + c0) = pack8(out);
+    for (int ch = 0; ch < 8; ++ch) out[ch] = silu_fast(acc[ch]);
+    *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(t) * C + c0) = pack8x2(out);
     if (t == seq_end - 1 && p.cs_out) {   // last token: the last three inputs are the new conv state
 #pragma unroll
       for (int s = 0; s < 3; ++s) {
         const int pos = t - 2 + s;
-        uint4 v;
-        if (pos >= seq_start) v = raw[i + 1 + s];
-        else if (p.cs_in) v = *reinterpret_cast<const uint4 *>(p.cs_in + (static_cast<size_t>(n) * 3 + (3 - (seq_start - pos))) * C + c0);
-        else v = make_uint4(0, 0, 0, 0);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (pos >= seq_start) {
+          v = __ldg(reinterpret_cast<const uint4 *>(p.x + static_cast<size_t>(pos) * C + c0));
+        } else if (p.cs_in) {
+          v = *reinterpret_cast<const uint4 *>(p.cs_in + (static_cast<size_t>(n) * 3 + (3 - (seq_start - pos))) * C + c0);
+        }
         *reinterpret_cast<uint4 *>(p.cs_out + (static_cast<size_t>(n) * 3 + s) * C + c0) = v;
       }
     }

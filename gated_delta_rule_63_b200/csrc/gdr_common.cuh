@@ -35,6 +35,9 @@ __device__ __forceinline__ uint16_t f2bf_bits(float x) {
 __device__ __forceinline__ float round_bf16(float x) { return bf_bits2f(f2bf_bits(x)); }
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+// SiLU with the fast exponential and division (a few fp32 ulp; the callers round
+// the result to bf16)
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 // torch softplus default: beta 1, threshold 20
 __device__ __forceinline__ float softplus_f(float x) { return x > 20.0f ? x : log1pf(expf(x)); }

@@ -51,8 +51,8 @@ __global__ void __launch_bounds__(kThreads) gated_rmsnorm_kernel(const uint16_t 
   }
   float out[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) out[i] = ov[i] * inv * wv[i] * silu_f(zv[i]);
-  *reinterpret_cast<uint4 *>(y + row * 128 + part * 8) = pack8(out);
+  for (int i = 0; i < 8; ++i) out[i] = ov[i] * inv * wv[i] * silu_fast(zv[i]);
+  *reinterpret_cast<uint4 *>(y + row * 128 + part * 8) = pack8x2(out);
 }
 
 }  // namespace

@@ -12,13 +12,16 @@
 // written once: 128 KB of HBM traffic per (sequence, head), the whole cost.
 //
 // Layout of the work: one CTA of 256 threads per (value head, sequence).
-// Warp w holds rows 16w..16w+15 of H, lane l holds columns 4l..4l+3 (one
-// float4 per row), so each warp-wide access is one contiguous 512-byte row.
-// The 16 row loads are issued first and stay in flight while the conv, norms
-// and gates are computed.  The CTAs of the value heads that share a key head
-// form a thread-block cluster: the q/k conv state of that key head is read
-// by all of them, then (after a cluster barrier) rolled by the first one, so
-// the conv state can be updated in place.
+// The 64 KB tile of H arrives in shared memory by one bulk copy, issued first
+// and in flight while the conv, norms and gates are computed; with registers
+// freed from holding the tile, three CTAs share an SM, so about 192 KB of
+// state loads are in flight per SM.  Warp w then reads rows 16w..16w+15,
+// lane l columns 4l..4l+3 (one float4 per row, each warp-wide access one
+// contiguous 512-byte row), once for the reductions and once for the update,
+// which is stored straight from registers.  The CTAs of the value heads that
+// share a key head form a thread-block cluster: the q/k conv state of that
+// key head is read by all of them, then (after a cluster barrier) rolled by
+// the first one, so the conv state can be updated in place.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -30,6 +33,7 @@ namespace {
 
 constexpr int D = kHeadDim;
 constexpr int kThreads = 256;
+constexpr int kTileBytes = D * D * 4;   // one fp32 state tile
 
 struct DecodeParams {
   const uint16_t *x;
@@ -43,6 +47,7 @@ struct DecodeParams {
   int hk, hv, group, channels;
   float *state;
   uint16_t *o;
+  int *err;
 };
 
 __device__ __forceinline__ void cluster_arrive() {
@@ -52,14 +57,11 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
 
-__device__ __forceinline__ float4 ld_stream(const float *p) {
-  return __ldcs(reinterpret_cast<const float4 *>(p));
-}
 __device__ __forceinline__ void st_stream(float *p, float4 v) {
   __stcs(reinterpret_cast<float4 *>(p), v);
 }
 
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   const int h = blockIdx.x;          // value head
   const int n = blockIdx.y;          // sequence
   const int kh = h / p.group;        // key head shared by `group` value heads
@@ -70,13 +72,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
   __shared__ float s_red[8][2][D];   // per-warp partial H^T k and H^T q
   __shared__ float s_sum[3][4];      // per-warp partial |q|^2, |k|^2, q.k
   __shared__ float s_gate[2];        // exp(g), beta
+  __shared__ alignas(8) uint64_t s_bar;
+  __shared__ int s_ok;
+  extern __shared__ float4 s_tile[];   // H, [D][D / 4] float4
 
-  // 1. issue the 16 state row loads of this thread
+  // 1. one bulk copy of the 64 KB state tile into shared memory
   float *S = p.state + (static_cast<size_t>(n) * p.hv + h) * D * D;
   const int row0 = warp * 16;
-  float4 r[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) r[i] = ld_stream(S + (row0 + i) * D + lane * 4);
+  const uint32_t bar = smem_u32(&s_bar);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, D * D * 4);
+    bulk_load(smem_u32(s_tile), S, D * D * 4, bar);
+  }
 
   // 2. conv step of this head's q, k (key head kh) and v channels
   const size_t xoff = static_cast<size_t>(n) * C;
@@ -119,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
     if (lane == 0) { s_sum[0][warp] = a2; s_sum[1][warp] = b2; s_sum[2][warp] = ab; }
   }
   if (tid == 0) {
+    s_ok = mbar_wait(bar, 0, p.err) ? 1 : 0;   // the tile has landed (bounded wait)
     const float av = bf_bits2f(p.a[static_cast<size_t>(n) * p.hv + h]);
     const float bv = bf_bits2f(p.b[static_cast<size_t>(n) * p.hv + h]);
     const float g = -expf(p.A_log[h]) * softplus_f(av + p.dt_bias[h]);
@@ -135,13 +145,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
   if (tid < D) { s_q[tid] = vq * rq; s_k[tid] = vk * rk; }
   __syncthreads();
 
+  const bool ok = s_ok != 0;
+
   // 4. partial H^T k and H^T q over this warp's 16 rows
   float pk[4] = {0, 0, 0, 0}, pq[4] = {0, 0, 0, 0};
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
+    const float4 r = s_tile[(row0 + i) * (D / 4) + lane];
     const float ki = s_k[row0 + i], qi = s_q[row0 + i];
-    pk[0] += r[i].x * ki; pk[1] += r[i].y * ki; pk[2] += r[i].z * ki; pk[3] += r[i].w * ki;
-    pq[0] += r[i].x * qi; pq[1] += r[i].y * qi; pq[2] += r[i].z * qi; pq[3] += r[i].w * qi;
+    pk[0] += r.x * ki; pk[1] += r.y * ki; pk[2] += r.z * ki; pk[3] += r.w * ki;
+    pq[0] += r.x * qi; pq[1] += r.y * qi; pq[2] += r.z * qi; pq[3] += r.w * qi;
   }
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -158,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
     const float u = beta * (vv - eg * hk_);
     s_u[tid] = u;
     const float ov = p.scale * (eg * hq_ + u * kq);
-    p.o[(static_cast<size_t>(n) * p.hv + h) * D + tid] = f2bf_bits(ov);
+    if (ok) p.o[(static_cast<size_t>(n) * p.hv + h) * D + tid] = f2bf_bits(ov);
   }
   __syncthreads();
 
@@ -167,12 +180,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float ki = s_k[row0 + i];
-    float4 v = r[i];
+    float4 v = s_tile[(row0 + i) * (D / 4) + lane];
     v.x = eg * v.x + ki * u4.x;
     v.y = eg * v.y + ki * u4.y;
     v.z = eg * v.z + ki * u4.z;
     v.w = eg * v.w + ki * u4.w;
-    st_stream(S + (row0 + i) * D + lane * 4, v);
+    if (ok) st_stream(S + (row0 + i) * D + lane * 4, v);
   }
 
   // 7. roll the conv state: v channels by this CTA, q/k channels by the first
@@ -217,11 +230,21 @@ int launch_decode(const void *x, const void *conv_w, void *conv_state, const voi
   p.channels = 2 * hk * D + hv * D;
   p.state = state;
   p.o = static_cast<uint16_t *>(o);
+  p.err = device_error_ptr();
 
+  static bool smem_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return launch_status(e, "decode: cudaGetDevice");
+  if (dev >= 0 && dev < 64 && !smem_set[dev]) {
+    e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileBytes);
+    if (e != cudaSuccess) return launch_status(e, "decode: shared memory opt-in");
+    smem_set[dev] = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(hv, batch, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = kTileBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -187,13 +187,20 @@ int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_st
   if (!cu_dev) return GDR_ERR_NULL;
   const bool fused_conv = fuse && fuse->x;
   const bool fused_norm = fuse && fuse->z;
-  if (fused_conv || fused_norm) return GDR_ERR_UNSUPPORTED;   // fusion not built yet
+  if (fused_conv) return GDR_ERR_UNSUPPORTED;   // the conv runs as its own kernel (gdr_causal_conv)
+  if (fuse && !fuse->z && fuse->y) return GDR_ERR_NULL;   // y without the gate z
   if (total > 0) {
     if (!a || !b || !A_log || !dt_bias) return GDR_ERR_NULL;
-    if (!q || !k || !v || !o) return GDR_ERR_NULL;
+    if (!q || !k || !v) return GDR_ERR_NULL;
+    if (!o && !fused_norm) return GDR_ERR_NULL;
+    if (fused_norm && !fuse->y) return GDR_ERR_NULL;
   }
+  const void *z = fused_norm ? fuse->z : nullptr;
+  void *y = fused_norm ? fuse->y : nullptr;
+  const float *norm_w = fused_norm ? fuse->norm_w : nullptr;
+  const float eps = fused_norm ? fuse->eps : 0.0f;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(h0) ||
-      !aligned16(hT) || !aligned16(workspace))
+      !aligned16(hT) || !aligned16(workspace) || !aligned16(z) || !aligned16(y) || !aligned16(norm_w))
     return GDR_ERR_ALIGN;
   int max_chunks = 0;
   for (int i = 0; i < n_seqs; ++i) {
@@ -205,8 +212,12 @@ int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_st
   if (max_chunks > 0 &&
       (!workspace || workspace_bytes < chunk_prefill_workspace_bytes(n_seqs, hv, 1, hT == nullptr)))
     return GDR_ERR_WORKSPACE;
+  if (fused_norm && o) {   // o and y are separate outputs
+    const size_t out_bytes = static_cast<size_t>(total) * hv * kHeadDim * 2;
+    if (overlaps(o, out_bytes, y, out_bytes)) return GDR_ERR_ALIAS;
+  }
   return launch_chunk_prefill(q, k, v, qk_stride, v_stride, a, b, A_log, dt_bias, scale, hk, hv,
-                              cu_dev, n_seqs, total, max_chunks, h0, hT, o, workspace,
+                              cu_dev, n_seqs, total, max_chunks, h0, hT, o, z, norm_w, eps, y, workspace,
                               workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 

@@ -89,7 +89,12 @@ constexpr uint32_t BLK128 = 128 * 128;
 constexpr uint32_t C_OFF_H = 2 * C_STAGE;            // [H_hi | H_lo], each [128 dk][64 dv]
 constexpr uint32_t C_OFF_U = C_OFF_H + 2 * BLK128;   // [U_hi | U_lo | U'_hi | U'_lo], each [64 tok][64 dv]
 constexpr uint32_t C_OFF_BAR = C_OFF_U + 4 * BLK64;  // 13 mbarriers, tmem base, abort flag
-constexpr uint32_t C_SMEM = C_OFF_BAR + 128 + 1024;
+// fused gated norm: per-row partial sums of squares of this CTA's two column halves
+// [parity 2][half 2][64], the other dv slice's row sums [parity 2][64], two mbarriers
+constexpr uint32_t C_OFF_NORM = C_OFF_BAR + 128;
+constexpr uint32_t C_OFF_PEER = C_OFF_NORM + 2 * 2 * 64 * 4;
+constexpr uint32_t C_OFF_PBAR = C_OFF_PEER + 2 * 64 * 4;
+constexpr uint32_t C_SMEM = C_OFF_PBAR + 16 + 1024;
 static_assert(C_SMEM <= 232448, "chain shared memory exceeds 227 KB");
 static_assert((C_QW_KB | C_OFF_K | C_OFF_MQ | C_STAGE | C_OFF_H | C_OFF_U) % 1024 == 0,
               "swizzled tiles need 1 KB alignment");
@@ -135,7 +140,12 @@ struct PrefillParams {
   int win_chunks;       // chunks per window (record stride)
   const float *state_in;
   float *state_out;
-  uint16_t *o;
+  uint16_t *o;          // may be null when y is set
+  // gated RMSNorm fused into the output (y != null): y = o / sqrt(mean o^2 + eps) w SiLU(z)
+  const uint16_t *z;
+  const float *norm_w;  // null = ones
+  float eps;
+  uint16_t *y;
   int *err;
 };
 
@@ -587,6 +597,23 @@ __device__ __forceinline__ bool chain_wait(uint32_t bar, uint32_t parity, volati
   return false;
 }
 
+// the same for an mbarrier that another CTA of the cluster arrives on; it polls
+// (with a short back-off) instead of sleeping in try_wait
+__device__ __forceinline__ bool chain_wait_cluster(uint32_t bar, uint32_t parity, volatile uint32_t *abort, int *err) {
+  const long long start = clock64();
+  while (!*abort) {
+    if (mbar_test_wait_cluster(bar, parity)) return true;
+    __nanosleep(32);
+    if (clock64() - start > (1LL << 32)) {
+      *abort = 1u;
+      raise_device_error(err, GDR_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return false;
+}
+
+template <bool kNorm>   // gated RMSNorm fused into the output (p.y set, cluster of the two dv slices)
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              PrefillParams p) {
@@ -648,6 +675,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // full x 6, products x 3, o_free (4 output warps), h_ready (8 warps), u_ready (4 state warps), drain
     const uint32_t counts[13] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 8, 4, 1};
     for (int i = 0; i < 13; ++i) mbar_init(bars + 8 * i, counts[i]);
+    if (kNorm) {   // the other slice's 64 row sums: 256 transaction bytes per chunk
+      mbar_init(sbase + C_OFF_PBAR, 1);
+      mbar_init(sbase + C_OFF_PBAR + 8, 1);
+    }
     *abort_flag = 0u;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -692,6 +723,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   __syncthreads();   // barriers initialised, tensor memory allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const uint32_t peer = static_cast<uint32_t>(slice) ^ 1u;   // the other dv slice of this head
+  if (kNorm) cluster_sync_all();   // both CTAs' barriers exist before either arrives remotely
 
   if (ctrl) {
     // =========================== control warp ===========================
@@ -819,6 +852,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       const float g_r = nx_g, sb = nx_s, gL = nx_gL;
       if (cw + 1 < nw) load_sc(cw + 1);
       PTIME(1 + cw, 0);
+
       if (wrow) {
         // ---- U = Ut - W H0 and U' = U e^(gamma_L - gamma) / |k| (state rows) ----------------
         chain_wait(bar_p, ph, abort_flag, p.err);
@@ -910,6 +944,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
       // ---- output rows: o = scale (e^gamma / |q| Q H0 + O), overlapping the next chunk ---------
       if (!wrow) {
+        uint4 zr[kNorm ? 4 : 1];   // the norm's gate, this thread's 32 columns of row r
+        const size_t orow = (static_cast<size_t>(t0 + r) * p.hv + h) * D + slice * N + 32 * ch;
+        if (kNorm) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            zr[c4] = r < L ? __ldg(reinterpret_cast<const uint4 *>(p.z + orow) + c4) : make_uint4(0, 0, 0, 0);
+          if (tid == 64)   // this chunk's 64 row sums from the other slice: 256 bytes
+            mbar_arrive_expect_tx(sbase + C_OFF_PBAR + 8 * (cw & 1), 64 * 4);
+        }
         chain_wait(bar_o, ph, abort_flag, p.err);
         __syncwarp();
         tc_fence_after();
@@ -925,15 +968,52 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(o_free);
-        if (r < L) {
-          uint16_t *dst = p.o + (static_cast<size_t>(t0 + r) * p.hv + h) * D + slice * N + 32 * ch;
+        if (kNorm) {
+          // fused gated RMSNorm: the row's 128 values are split over this thread, the thread of
+          // the other column half and the two threads of the other dv slice (cluster peer)
+          const uint32_t pb = cw & 1;
+          float ss = 0.0f;
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) *reinterpret_cast<uint4 *>(dst + 8 * c4) = pack8x2(oreg + 8 * c4);
+          for (int j = 0; j < 32; ++j) {
+            oreg[j] = round_bf16(oreg[j]);   // the norm reads the bf16 o
+            ss += oreg[j] * oreg[j];
+          }
+          float *s_ss = reinterpret_cast<float *>(smem + C_OFF_NORM) + pb * 128;
+          s_ss[ch * 64 + r] = ss;
+          named_sync(1, 128);   // the four output warps
+          const float own = s_ss[r] + s_ss[64 + r];
+          const uint32_t peer_slot = smem_u32(smem + C_OFF_PEER) + (pb * 64 + r) * 4;
+          if (ch == 0) st_async_remote(map_peer(peer_slot, peer), own, map_peer(sbase + C_OFF_PBAR + 8 * pb, peer));
+          PTIME_T(1 + cw, 29, 64);
+          float total = own;
+          if (chain_wait_cluster(sbase + C_OFF_PBAR + 8 * pb, (cw >> 1) & 1, abort_flag, p.err))
+            total += reinterpret_cast<const float *>(smem + C_OFF_PEER)[pb * 64 + r];
+          PTIME_T(1 + cw, 30, 64);
+          const float inv = 1.0f / sqrtf(total * (1.0f / 128.0f) + p.eps);
+          if (r < L) {
+            const int col0 = slice * N + 32 * ch;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+              float zf[8], yv[8];
+              unpack8(zr[c4], zf);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float wv = p.norm_w ? __ldg(p.norm_w + col0 + 8 * c4 + e) : 1.0f;
+                yv[e] = oreg[8 * c4 + e] * inv * wv * silu_fast(zf[e]);
+              }
+              *reinterpret_cast<uint4 *>(p.y + orow + 8 * c4) = pack8x2(yv);
+              if (p.o) *reinterpret_cast<uint4 *>(p.o + orow + 8 * c4) = pack8x2(oreg + 8 * c4);
+            }
+          }
+        } else if (r < L) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) *reinterpret_cast<uint4 *>(p.o + orow + 8 * c4) = pack8x2(oreg + 8 * c4);
         }
         PTIME_T(1 + cw, 7, 64);
       }
     }
   }
+  if (kNorm) cluster_sync_all();   // no remote arrivals target a CTA that has left
   tc_fence_before();
   __syncthreads();
   if (!ctrl && p.state_out && *abort_flag == 0u) {
@@ -989,7 +1069,9 @@ int ensure_smem_attrs() {
   if (bit && (done.load(std::memory_order_acquire) & bit)) return GDR_OK;
   e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
+    e = cudaFuncSetAttribute(chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
   if (e != cudaSuccess) return launch_status(e, "prefill: shared memory opt-in");
   done.fetch_or(bit, std::memory_order_acq_rel);
   return GDR_OK;
@@ -1007,8 +1089,8 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
                          int64_t v_stride, const void *a, const void *b,
                          const float *A_log, const float *dt_bias, float scale, int hk, int hv,
                          const int32_t *cu_dev, int n_seqs, int total, int max_chunks,
-                         const float *h0, float *hT, void *o, void *workspace, size_t ws_bytes,
-                         cudaStream_t s) {
+                         const float *h0, float *hT, void *o, const void *z, const float *norm_w,
+                         float eps, void *y, void *workspace, size_t ws_bytes, cudaStream_t s) {
   if (n_seqs > 65535 || hv > 65535) return GDR_ERR_SHAPE;
   int st = ensure_smem_attrs();
   if (st) return st;
@@ -1049,6 +1131,10 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   p.ws = static_cast<uint8_t *>(workspace);
   p.win_chunks = win;
   p.o = static_cast<uint16_t *>(o);
+  p.z = static_cast<const uint16_t *>(z);
+  p.norm_w = norm_w;
+  p.eps = eps;
+  p.y = static_cast<uint16_t *>(y);
   p.err = device_error_ptr();
   const int n_windows = max_chunks > 0 ? (max_chunks + win - 1) / win : 1;
   for (int w = 0; w < n_windows; ++w) {
@@ -1062,8 +1148,24 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
       st = last_launch_status("prefill: prep kernel launch");
       if (st) return st;
     }
-    chain_kernel<<<dim3(NS, hv, n_seqs), kChainThreads, C_SMEM, s>>>(tq, tk, p);
-    st = last_launch_status("prefill: chain kernel launch");
+    if (y) {   // fused norm: the two dv slices of a head form a cluster and exchange row sums
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(NS, hv, n_seqs);
+      cfg.blockDim = dim3(kChainThreads, 1, 1);
+      cfg.dynamicSmemBytes = C_SMEM;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = NS;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      st = launch_status(cudaLaunchKernelEx(&cfg, chain_kernel<true>, tq, tk, p), "prefill: chain kernel launch");
+    } else {
+      chain_kernel<false><<<dim3(NS, hv, n_seqs), kChainThreads, C_SMEM, s>>>(tq, tk, p);
+      st = last_launch_status("prefill: chain kernel launch");
+    }
     if (st) return st;
   }
   return GDR_OK;

@@ -108,12 +108,16 @@ GDR_API int gdr_causal_conv(const void *x, const void *w, const void *conv_state
                     int channels, void *y, void *stream);
 
 /*
- * Optional fusion of the conv in front of and the gated RMSNorm behind the
- * prefill (pass NULL to gdr_chunk_prefill to run the recurrence alone).
- * When `x` is set, q, k and v are read as the conv output of x (channels laid
- * out [q | k | v] = hk*128 + hk*128 + hv*128) and the q/k/v arguments of
- * gdr_chunk_prefill must be NULL.  When `z` is set, y receives the gated
- * RMSNorm of o.
+ * Optional fusion around the prefill (pass NULL to gdr_chunk_prefill to run
+ * the recurrence alone).
+ *  - Gated RMSNorm (`z` set): y receives o / sqrt(mean(o^2) + eps) * w * SiLU(z)
+ *    row by row, computed from the bf16-rounded o inside the prefill (the two
+ *    64-column halves of a head run as a thread-block cluster and exchange their
+ *    row sums of squares); o is written as well only when gdr_chunk_prefill's o
+ *    is not NULL.  y must not overlap o (GDR_ERR_ALIAS).
+ *  - Conv (`x` set): not fused in this version; the call returns
+ *    GDR_ERR_UNSUPPORTED.  Run gdr_causal_conv and pass its output's q, k, v
+ *    column ranges as strided views.
  */
 typedef struct gdr_prefill_fuse {
   const void *x;             /* bf16 [T][hk*128*2 + hv*128] conv input, or NULL */
@@ -146,7 +150,7 @@ typedef struct gdr_prefill_fuse {
  *   h0:       fp32 [n_seqs][hv][128][128] initial state (H = S^T), or NULL = zeros
  *   hT:       fp32 [n_seqs][hv][128][128] final state, or NULL; may equal h0
  *             (in place), must not overlap it otherwise.
- *   o:        bf16 [T][hv][128]; may be NULL only when fuse->y is set.
+ *   o:        bf16 [T][hv][128]; may be NULL when fuse->y is set (fused norm).
  *   fuse:     NULL, or conv / gated-norm fusion (see gdr_prefill_fuse_t).
  *   workspace, workspace_bytes: device scratch, 16-byte aligned, at least
  *             gdr_chunk_prefill_workspace_size(n_seqs, hv, 1, hT != NULL)

@@ -206,6 +206,58 @@ def test_full_path_T4096_unfused():
     assert rel_l2(hT.cpu().numpy(), ref["hT"]) <= TOL_STATE
 
 
+def run_full_gpu(inp, fused_norm, keep_o=False):
+    """conv -> prefill (-> gated norm, fused into the prefill or as its own call)."""
+    cu_d = dev_i32(inp.cu_seqlens)
+    y = G.causal_conv(dev_bf16(inp.x), dev_bf16(inp.conv_w), cu_d, inp.cu_seqlens)
+    T, hk, hv = inp.T, inp.hk, inp.hv
+    q = y[:, : hk * 128].view(T, hk, 128)
+    k = y[:, hk * 128: 2 * hk * 128].view(T, hk, 128)
+    v = y[:, 2 * hk * 128:].view(T, hv, 128)
+    hT = torch.empty((inp.n_seqs, hv, 128, 128), device="cuda")
+    z = dev_bf16(inp.z).reshape(T, hv, 128)
+    w = dev_f32(inp.norm_w) if inp.norm_w is not None else None
+    h0 = dev_f32(inp.h0) if inp.h0 is not None else None
+    args = (q, k, v, dev_bf16(inp.a), dev_bf16(inp.b), dev_f32(inp.A_log), dev_f32(inp.dt_bias), cu_d,
+            inp.cu_seqlens)
+    if fused_norm:
+        out = torch.full((T, hv, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+        o = torch.empty((T, hv, 128), dtype=torch.bfloat16, device="cuda") if keep_o else None
+        G.chunk_prefill(*args, h0=h0, hT=hT, o=o, scale=inp.scale,
+                        fuse={"z": z, "norm_w": w, "eps": inp.eps, "y": out})
+    else:
+        o = G.chunk_prefill(*args, h0=h0, hT=hT, scale=inp.scale)
+        out = G.gated_rmsnorm(o, z, w, eps=inp.eps)
+    torch.cuda.synchronize()
+    return (host_bits(o) if o is not None else None), host_bits(out), hT.cpu().numpy()
+
+
+def test_fused_gated_norm_varlen_matches_unfused_and_oracle():
+    """The gated RMSNorm fused into the prefill's output equals the separate norm call."""
+    inp = GI.make_full_inputs(80, [200, 65, 1, 0, 130], h0_std=0.02, norm_w_std=0.1)
+    o_u, y_u, h_u = run_full_gpu(inp, fused_norm=False)
+    o_f, y_f, h_f = run_full_gpu(inp, fused_norm=True, keep_o=True)
+    assert np.array_equal(o_f, o_u)                 # the recurrence is the same
+    assert np.array_equal(h_f, h_u)
+    assert ulp_diff_bf16(y_f, y_u).max() <= 1       # only the sum-of-squares order differs
+    ref = O.full_path(inp)
+    assert rel_l2(bits_f64(y_f), bits_f64(ref["y"])) <= TOL_BF16
+    cu = inp.cu_seqlens
+    for n in range(inp.n_seqs):                     # every sequence on its own
+        s, e = int(cu[n]), int(cu[n + 1])
+        if e > s:
+            assert rel_l2(bits_f64(y_f[s:e]), bits_f64(ref["y"][s:e])) <= TOL_BF16
+
+
+def test_full_path_T4096_fused_norm():
+    """The bench workload with the gated norm fused, against the oracle."""
+    inp = GI.workload_full_T4096()
+    _, y_f, h_f = run_full_gpu(inp, fused_norm=True)
+    ref = O.full_path(inp)
+    assert rel_l2(bits_f64(y_f), bits_f64(ref["y"])) <= TOL_BF16
+    assert rel_l2(h_f, ref["hT"]) <= TOL_STATE
+
+
 def test_prefill_long_context_sampled_heads():
     """B=1, T=262144: every head on the GPU, three heads through the oracle."""
     inp = GI.workload_core_T262144()

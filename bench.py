@@ -2,7 +2,7 @@
 """Benchmark of the gated delta-rule layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload full_T4096|decode_B64|core_T262144|varlen8|core_T128]
+                    [--part all|prefill|decode] [--decode-steps S] [--no-cpu-baseline]
 
 A step of the default workload is one pass of the prefill path of one layer
 over B=1, T=4096 tokens: causal conv4+SiLU over the 10240 q|k|v channels ->
@@ -10,6 +10,9 @@ chunk-64 gated delta rule (16 key / 48 value heads, dim 128) -> gated RMSNorm.
 The decode path (B=64 sequences, one token each, 1000 consecutive steps) is
 measured in the same run and reported under "decode".  Inputs are seeded
 synthetic tensors (gdr_inputs) with the layer's shapes; there are no weights.
+
+`--part prefill` / `--part decode` run one of the two paths alone (for
+profiling); the default `all` is the benchmark.
 
 Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs its own
 replica of the workload (the path has no cross-GPU exchange) and the value is
@@ -44,6 +47,12 @@ B_CORE = (2 * GI.HK * GI.DK + GI.HV * GI.DV) * 2 + 2 * GI.HV * 2 + GI.HV * GI.DV
 B_NORM = 3 * GI.HV * GI.DV * 2                           # o, z read + y write
 B_FUSED = CX * 2 + 2 * GI.HV * 2 + 2 * GI.HV * GI.DV * 2 # x, a, b, z read + y write
 STATE_BYTES = GI.HV * GI.DK * GI.DV * 4                  # one sequence's fp32 state
+
+# DRAM bytes (read + written) per launch from one ncu capture of the current kernels:
+# prefill = prep + state chain on full_T4096, decode = one B=64 step (a replayed launch,
+# partly served from L2)
+TRAFFIC_PREFILL = (84.805888 + 196.792576 + 287.766016 + 41.982720) * 1e6
+TRAFFIC_DECODE = (206.692096 + 149.694720) * 1e6
 
 
 def measured_peaks():
@@ -191,7 +200,7 @@ def bench_ours(args, rank, world, device):
             ev[i][1].record()
         torch.cuda.synchronize()
         # decode: B=64, 1000 consecutive steps, state updated in place
-        dec_res = bench_decode(torch, G, device, args)
+        dec_res = bench_decode(torch, G, device, args, steps=args.decode_steps) if args.part == "all" else None
     if world > 1:
         torch.distributed.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -205,7 +214,7 @@ def bench_ours(args, rank, world, device):
     value = world * T / (ms * 1e-3)
 
     # end to end through the C ABI with host buffers (pinned), copies inside
-    e2e = bench_e2e(torch, G, inp, device, args)
+    e2e = bench_e2e(torch, G, inp, device, args) if args.part == "all" else None
 
     prefill_bytes = T * B_CORE + inp.n_seqs * STATE_BYTES
     achieved = prefill_bytes / (pms * 1e-3) / 1e9
@@ -220,14 +229,14 @@ def bench_ours(args, rank, world, device):
                    "fused": False},
         "roofline": {"kernel": "gdr_chunk_prefill", "bound": "hbm", "achieved": achieved,
                      "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                     "peak_kind": peak_kind, "traffic": None,
+                     "peak_kind": peak_kind, "traffic": TRAFFIC_PREFILL,
                      "algorithmic_bytes_per_launch": prefill_bytes, "ms_per_launch": pms},
         "step_roofline": {"bytes_per_token_unfused": B_CONV + B_CORE + B_NORM,
                           "bytes_per_token_fused": B_FUSED,
                           "frac_of_fused_hbm_roofline": (T * B_FUSED + STATE_BYTES) / (ms * 1e-3) / 1e9 / hbm_peak},
         "decode": dec_res,
         "e2e": e2e,
-        "gpu_launches": 4 * args.steps + dec_res["launches"],
+        "gpu_launches": 4 * args.steps + (dec_res["launches"] if dec_res else 0),
         "clocks": clk.summary(),
     }
     return res
@@ -261,7 +270,7 @@ def bench_decode(torch, G, device, args, steps=1000):
             "steps": steps, "launches": steps,
             "roofline": {"kernel": "gdr_decode_step", "bound": "hbm", "achieved": achieved,
                          "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                         "algorithmic_bytes_per_launch": bytes_step, "traffic": None}}
+                         "algorithmic_bytes_per_launch": bytes_step, "traffic": TRAFFIC_DECODE}}
 
 
 def bench_e2e(torch, G, inp, device, args):
@@ -349,6 +358,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--part", choices=["all", "prefill", "decode"], default="all")
+    ap.add_argument("--decode-steps", type=int, default=1000)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -367,6 +378,14 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local)
+    if args.part == "decode":
+        torch.cuda.set_device(device)
+        import gated_delta_rule_63_b200 as G
+        G.lib()
+        res = bench_decode(torch, G, device, args, steps=args.decode_steps)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
     res = bench_ours(args, rank, world, device)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:

@@ -50,8 +50,11 @@ struct DecodeParams {
   int *err;
 };
 
+// Relaxed arrive: what it guards are this thread's reads of the shared q/k conv
+// state, and their values have been consumed (the conv outputs are computed) before
+// the arrive, so no release fence is needed.
 __device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");

@@ -65,16 +65,19 @@ constexpr uint32_t P_OFF_KQ = 0;                     // 2 k-blocks
 constexpr uint32_t P_OFF_V = P_OFF_KQ + 2 * P_KQ_KB; // V [dv block 2][64 rows][128 B]
 constexpr uint32_t P_OFF_T = P_OFF_V + 2 * BLK64;    // T'_hi, T'_lo, T''_hi, T''_lo
 constexpr int LD = 68;                               // fp32 row stride of AT (rows 16-byte aligned)
-constexpr int XLD = 20;                              // fp32 row stride of the X^T blocks
+constexpr int XLD = 20;                              // fp32 row stride of the 16 x 16 X^T blocks
+constexpr int XLD2 = 36;                             // fp32 row stride of the 32 x 32 X^T block
 constexpr uint32_t P_OFF_AT = P_OFF_T + 4 * BLK64;   // A below / T^T on and above the diagonal
 constexpr uint32_t P_OFF_XF = P_OFF_AT + 64 * LD * 4;
-constexpr uint32_t P_OFF_SC = P_OFF_XF + 3 * 16 * XLD * 4;  // gamma, rq, rk, beta, e^gamma, block decay, e^g
+constexpr uint32_t P_OFF_SC = P_OFF_XF + 32 * XLD2 * 4;  // gamma, rq, rk, beta, e^gamma, block decay, e^g
+static_assert(32 * XLD2 >= 3 * 16 * XLD, "X^T scratch holds both block sizes");
 constexpr uint32_t P_OFF_BAR = P_OFF_SC + 7 * 64 * 4;
 constexpr uint32_t P_SMEM = P_OFF_BAR + 32 + 1024;
 static_assert((P_OFF_V | P_OFF_T) % 1024 == 0, "swizzled tiles need 1 KB alignment");
 constexpr uint32_t P_TM_COLS = 256;                  // two prep CTAs per SM
-constexpr uint32_t P_COL_S = 0;                      // [K K^T ; Q K^T]
-constexpr uint32_t P_COL_X = 128;                    // W, then Ut (128 cols)
+constexpr uint32_t P_COL_S = 0;                      // [K K^T ; Q K^T] (64 cols, dead once A and Mq are built)
+constexpr uint32_t P_COL_W = 0;                      // W = T' K, lanes 0..63 (128 cols)
+constexpr uint32_t P_COL_U = 128;                    // Ut = T'' V, lanes 64..127 (128 cols)
 
 // ---- chain kernel ------------------------------------------------------------
 constexpr int kChainThreads = 288;                    // warps 0..7 state and output, warp 8 control
@@ -241,9 +244,22 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                                       : P_OFF_KQ + (cc >> 3) * P_KQ_KB + tile * 64 * 128;
       st_shared16(sbase + base + sw128(r, cc & 7), make_uint4(0, 0, 0, 0));
     }
+    fence_proxy_async();
     __syncthreads();
   }
   if (ok) {
+    // ---- [K; Q] K^T on the raw tiles, while the norms and gates are computed ----------
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t koff = (kk >> 2) * P_KQ_KB + (kk & 3) * 32;
+        mma_bf16(tmem + P_COL_S, sdesc(sbase + P_OFF_KQ + koff, 16, 1024),
+                 sdesc(sbase + P_OFF_KQ + koff, 16, 1024), id, kk > 0);
+      }
+      mma_commit(bar_mma);
+    }
     // 1/|k| (rows 0..63 of the KQ tile) and 1/|q| (rows 64..127), two threads per row
     const int row = tid >> 1, part = tid & 1;
     float ss = 0.0f;
@@ -284,18 +300,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
 
     PTIME(0, 2);
-    // ---- [K; Q] K^T ------------------------------------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t koff = (kk >> 2) * P_KQ_KB + (kk & 3) * 32;
-        mma_bf16(tmem + P_COL_S, sdesc(sbase + P_OFF_KQ + koff, 16, 1024),
-                 sdesc(sbase + P_OFF_KQ + koff, 16, 1024), id, kk > 0);
-      }
-      mma_commit(bar_mma);
-    }
     ok = cta_wait(bar_mma, 0, p.err);
   }
   if (ok) {
@@ -385,19 +389,21 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     PTIME(0, 13);
     __syncthreads();
-    // off-diagonal blocks by diagonals d = b - c: X_bc = sum_{m=c}^{b-1} A_bm T_mc, T_bc = -T_bb X_bc.
-    // Each block is computed by 64 threads holding 2 x 2 tiles (rows rt, rt + 8; columns jt, jt + 8);
-    // A rows and T^T rows are read as float4 along k.
-    for (int d = 1; d < 4; ++d) {
-      const int nb = 4 - d;
+    // off-diagonal blocks.  Level 1: the two 16 x 16 blocks (1, 0) and (3, 2) that complete
+    // the 32 x 32 diagonal halves, X_bc = A_bc T_cc, T_bc = -T_bb X_bc, on 64 threads per block with 2 x 2
+    // tiles (rows rt, rt + 8; columns jt, jt + 8).  Level 2: the 32 x 32 block below the
+    // diagonal of the two 32 x 32 halves T1, T2 (complete after level 1),
+    // X = A21 T1, T21 = -T2 X, on all 256 threads with 2 x 2 tiles (rows rt, rt + 16;
+    // columns jt, jt + 16).  A rows and T^T rows are read as float4 along k.
+    {
       const int blk = tid >> 6, t = tid & 63, rt = t >> 3, jt = t & 7;
-      const int bb = d + blk, cb = blk;
-      if (blk < nb) {   // X_bc^T[j][r] into XF
+      const int bb = 1 + 2 * blk, cb = 2 * blk;
+      if (blk < 2) {   // X_bc^T[j][r] into XF
         const float *a0 = AT + (16 * bb + rt) * LD, *a1 = a0 + 8 * LD;
         const float *t0 = AT + (16 * cb + jt) * LD, *t1 = t0 + 8 * LD;   // T^T rows = columns of T
         float x00 = 0.0f, x01 = 0.0f, x10 = 0.0f, x11 = 0.0f;         // x[r][j] for r in {rt, rt+8}, j in {jt, jt+8}
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {   // block m = c: T[16c + l][16c + j] is zero for l < j
+        for (int g = 0; g < 4; ++g) {   // T[16c + l][16c + j] is zero for l < j
           const int k = 16 * cb + 4 * g;
           const float4 A0 = *reinterpret_cast<const float4 *>(a0 + k), A1 = *reinterpret_cast<const float4 *>(a1 + k);
           const float4 T0 = *reinterpret_cast<const float4 *>(t0 + k), T1 = *reinterpret_cast<const float4 *>(t1 + k);
@@ -410,14 +416,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             x10 += av1[e] * u0; x11 += av1[e] * u1;
           }
         }
-        for (int k = 16 * (cb + 1); k < 16 * bb; k += 4) {
-          const float4 A0 = *reinterpret_cast<const float4 *>(a0 + k), A1 = *reinterpret_cast<const float4 *>(a1 + k);
-          const float4 T0 = *reinterpret_cast<const float4 *>(t0 + k), T1 = *reinterpret_cast<const float4 *>(t1 + k);
-          x00 += A0.x * T0.x + A0.y * T0.y + A0.z * T0.z + A0.w * T0.w;
-          x01 += A0.x * T1.x + A0.y * T1.y + A0.z * T1.z + A0.w * T1.w;
-          x10 += A1.x * T0.x + A1.y * T0.y + A1.z * T0.z + A1.w * T0.w;
-          x11 += A1.x * T1.x + A1.y * T1.y + A1.z * T1.z + A1.w * T1.w;
-        }
         float *xt = XF + (blk * 16 + jt) * XLD;
         xt[rt] = x00;
         xt[rt + 8] = x10;
@@ -425,7 +423,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         xt[8 * XLD + rt + 8] = x11;
       }
       __syncthreads();
-      if (blk < nb) {   // T_bc[r][j] = -sum_{l <= r} T_bb[r][l] X_bc[l][j], stored as T^T
+      if (blk < 2) {   // T_bc[r][j] = -sum_{l <= r} T_bb[r][l] X_bc[l][j], stored as T^T
         const float *xa = XF + (blk * 16 + jt) * XLD, *xb = xa + 8 * XLD;
         const float *tb = AT + (16 * bb) * LD + 16 * bb;               // tb[l * LD + r] = T_bb[r][l]
         float y00 = 0.0f, y01 = 0.0f, y10 = 0.0f, y11 = 0.0f;         // y[r][j]
@@ -443,7 +441,59 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         dst[8 * LD + rt + 8] = y11;
       }
       __syncthreads();
-      PTIME(0, 13 + d);
+      PTIME(0, 14);
+    }
+    {
+      const int rt = tid >> 4, jt = tid & 15;
+      {   // X^T[j][r] = sum_{k >= j} A[32 + r][k] T[k][j], r, j < 32, into XF (stride XLD2)
+        const float *a0 = AT + (32 + rt) * LD, *a1 = a0 + 16 * LD;
+        const float *t0 = AT + jt * LD, *t1 = t0 + 16 * LD;
+        float x00 = 0.0f, x01 = 0.0f, x10 = 0.0f, x11 = 0.0f;   // x[r][j], r in {rt, rt+16}, j in {jt, jt+16}
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const int k0 = 4 * g;
+          const float4 A0 = *reinterpret_cast<const float4 *>(a0 + k0), A1 = *reinterpret_cast<const float4 *>(a1 + k0);
+          const float4 T0 = *reinterpret_cast<const float4 *>(t0 + k0), T1 = *reinterpret_cast<const float4 *>(t1 + k0);
+          const float av0[4] = {A0.x, A0.y, A0.z, A0.w}, av1[4] = {A1.x, A1.y, A1.z, A1.w};
+          const float tv0[4] = {T0.x, T0.y, T0.z, T0.w}, tv1[4] = {T1.x, T1.y, T1.z, T1.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {   // T is lower triangular: T[k][j] = 0 for k < j
+            const float u0 = (k0 + e >= jt) ? tv0[e] : 0.0f, u1 = (k0 + e >= jt + 16) ? tv1[e] : 0.0f;
+            x00 += av0[e] * u0; x01 += av0[e] * u1;
+            x10 += av1[e] * u0; x11 += av1[e] * u1;
+          }
+        }
+        float *xt = XF + jt * XLD2;
+        xt[rt] = x00;
+        xt[rt + 16] = x10;
+        xt[16 * XLD2 + rt] = x01;
+        xt[16 * XLD2 + rt + 16] = x11;
+      }
+      __syncthreads();
+      {   // T21[r][j] = -sum_{l <= r} T2[r][l] X[l][j], T2[r][l] = AT[(32 + l) LD + 32 + r]; stored as T^T
+        const float *xa = XF + jt * XLD2, *xb = xa + 16 * XLD2;
+        const float *tb = AT + 32 * LD + 32;
+        float y00 = 0.0f, y01 = 0.0f, y10 = 0.0f, y11 = 0.0f;   // y[r][j]
+#pragma unroll
+        for (int l4 = 0; l4 < 8; ++l4) {
+          const float4 X0 = *reinterpret_cast<const float4 *>(xa + 4 * l4), X1 = *reinterpret_cast<const float4 *>(xb + 4 * l4);
+          const float x0v[4] = {X0.x, X0.y, X0.z, X0.w}, x1v[4] = {X1.x, X1.y, X1.z, X1.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int l = 4 * l4 + e;
+            const float t0v = l <= rt ? tb[l * LD + rt] : 0.0f, t1v = l <= rt + 16 ? tb[l * LD + rt + 16] : 0.0f;
+            y00 -= t0v * x0v[e]; y01 -= t0v * x1v[e];
+            y10 -= t1v * x0v[e]; y11 -= t1v * x1v[e];
+          }
+        }
+        float *dst = AT + jt * LD + 32;
+        dst[rt] = y00;
+        dst[rt + 16] = y10;
+        dst[16 * LD + rt] = y01;
+        dst[16 * LD + rt + 16] = y11;
+      }
+      __syncthreads();
+      PTIME(0, 15);
     }
 
     PTIME(0, 5);
@@ -475,7 +525,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
 
     PTIME(0, 6);
-    // ---- W = T' K  (A rows 64..127 are the next tile: junk lanes, never read) ---
+    // ---- W = T' K (rows in lanes 0..63) and Ut = T'' V (rows in lanes 64..127), one wait ----
+    // MN-major A operands of 128 rows: W's second row block and Ut's first are other tiles,
+    // whose products land in lanes that are never read
     if (tid == 0) {
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 128, true, true);
@@ -483,72 +535,62 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       for (int part = 0; part < 2; ++part)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + P_COL_X, sdesc(sbase + P_OFF_T + part * BLK64 + kk * 2048, BLK64, 1024),
+          mma_bf16(tmem + P_COL_W, sdesc(sbase + P_OFF_T + part * BLK64 + kk * 2048, BLK64, 1024),
                    sdesc(sbase + P_OFF_KQ + kk * 2048, P_KQ_KB, 1024), id, (part | kk) != 0);
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + P_COL_U, sdesc(sbase + P_OFF_T + (1 + part) * BLK64 + kk * 2048, BLK64, 1024),
+                   sdesc(sbase + P_OFF_V + kk * 2048, BLK64, 1024), id, (part | kk) != 0);
       mma_commit(bar_mma);
     }
     ok = cta_wait(bar_mma, 1, p.err);
   }
+  PTIME(0, 7);
   if (ok) {
-    PTIME(0, 7);
-    if ((warp & 2) == 0) {   // warps 0, 1, 4, 5 own lanes 0..63; k-block = warp >> 2
+    if ((warp & 2) == 0) {
+      // warps 0, 1, 4, 5 (lanes 0..63): W rows -> [W_hi kb0 | W_hi kb1 | W_lo kb0 | W_lo kb1]
+      // over the dead K/Q tiles; k-block = warp >> 2
       const int kb = warp >> 2, r = 32 * (warp & 1) + lane;
-      const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + P_COL_X + 64 * kb;
+      const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + P_COL_W + 64 * kb;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         float w[32];
         tmem_ld32(tl + 32 * hh, w);
         tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {   // [W_hi kb0 | W_hi kb1 | W_lo kb0 | W_lo kb1] over the dead K/Q tiles
+        for (int c4 = 0; c4 < 4; ++c4) {
           const uint32_t off = kb * BLK64 + sw128(r, 4 * hh + c4);
           st_split8_shared(sbase + P_OFF_KQ + off, sbase + P_OFF_KQ + 2 * BLK64 + off, w + 8 * c4);
         }
       }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    PTIME(0, 8);
-    // ---- Ut = T'' V (N = 128) ---------------------------------------------------
-    if (tid == 0) {
-      bulk_store(rec + WS_W_HI, sbase + P_OFF_KQ, 4 * BLK64);
-      bulk_commit();
-      tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 128, true, true);
+    } else {
+      // warps 2, 3, 6, 7 (lanes 64..127): Ut rows -> fp32 [slice][row][64] over the T tiles
+      const int sl = warp >> 2, r = 32 * (warp & 1) + lane;
+      const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + P_COL_U + 64 * sl;
+      const uint32_t dst = sbase + P_OFF_T + (static_cast<uint32_t>(sl) * 64 + r) * 256;
 #pragma unroll
-      for (int part = 0; part < 2; ++part)
+      for (int hh = 0; hh < 2; ++hh) {
+        float u[32];
+        tmem_ld32(tl + 32 * hh, u);
+        tmem_wait_ld();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + P_COL_X, sdesc(sbase + P_OFF_T + (2 + part) * BLK64 + kk * 2048, BLK64, 1024),
-                   sdesc(sbase + P_OFF_V + kk * 2048, BLK64, 1024), id, (part | kk) != 0);
-      mma_commit(bar_mma);
-    }
-    ok = cta_wait(bar_mma, 0, p.err);
-  }
-  PTIME(0, 9);
-  if (ok && (warp & 2) == 0) {   // Ut rows -> fp32 [slice][row][64] staged over the T'' tiles
-    const int sl = warp >> 2, r = 32 * (warp & 1) + lane;
-    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + P_COL_X + 64 * sl;
-    const uint32_t dst = sbase + P_OFF_T + (static_cast<uint32_t>(sl) * 64 + r) * 256;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      float u[32];
-      tmem_ld32(tl + 32 * hh, u);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        const uint32_t j = (8 * hh + c4) ^ (r & 7);
-        st_shared16(dst + 16 * j, make_uint4(__float_as_uint(u[4 * c4]), __float_as_uint(u[4 * c4 + 1]),
-                                             __float_as_uint(u[4 * c4 + 2]), __float_as_uint(u[4 * c4 + 3])));
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const uint32_t j = (8 * hh + c4) ^ (r & 7);
+          st_shared16(dst + 16 * j, make_uint4(__float_as_uint(u[4 * c4]), __float_as_uint(u[4 * c4 + 1]),
+                                               __float_as_uint(u[4 * c4 + 2]), __float_as_uint(u[4 * c4 + 3])));
+        }
       }
     }
   }
+  PTIME(0, 9);
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   if (tid == 0) {
     if (ok) {
+      bulk_store(rec + WS_W_HI, sbase + P_OFF_KQ, 4 * BLK64);
       bulk_store(rec + WS_UT, sbase + P_OFF_T, 4 * BLK64);
       bulk_commit();
     }

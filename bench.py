@@ -51,8 +51,9 @@ STATE_BYTES = GI.HV * GI.DK * GI.DV * 4                  # one sequence's fp32 s
 # DRAM bytes (read + written) per launch from one ncu capture of the current kernels:
 # prefill = prep + state chain on full_T4096, decode = one B=64 step (a replayed launch,
 # partly served from L2)
-TRAFFIC_PREFILL = (84.805888 + 196.792576 + 287.766016 + 41.982720) * 1e6
-TRAFFIC_DECODE = (206.692096 + 149.694720) * 1e6
+# (None until the changed kernels are captured again)
+TRAFFIC_PREFILL = None
+TRAFFIC_DECODE = None
 
 
 def measured_peaks():
@@ -229,7 +230,7 @@ def bench_ours(args, rank, world, device):
                    "fused": False},
         "roofline": {"kernel": "gdr_chunk_prefill", "bound": "hbm", "achieved": achieved,
                      "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                     "peak_kind": peak_kind, "traffic": TRAFFIC_PREFILL,
+                     "peak_kind": peak_kind, "traffic": TRAFFIC_PREFILL if TRAFFIC_PREFILL else None,
                      "algorithmic_bytes_per_launch": prefill_bytes, "ms_per_launch": pms},
         "step_roofline": {"bytes_per_token_unfused": B_CONV + B_CORE + B_NORM,
                           "bytes_per_token_fused": B_FUSED,
@@ -270,7 +271,7 @@ def bench_decode(torch, G, device, args, steps=1000):
             "steps": steps, "launches": steps,
             "roofline": {"kernel": "gdr_decode_step", "bound": "hbm", "achieved": achieved,
                          "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                         "algorithmic_bytes_per_launch": bytes_step, "traffic": TRAFFIC_DECODE}}
+                         "algorithmic_bytes_per_launch": bytes_step, "traffic": TRAFFIC_DECODE if TRAFFIC_DECODE else None}}
 
 
 def bench_e2e(torch, G, inp, device, args):

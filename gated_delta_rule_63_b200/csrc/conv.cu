@@ -20,7 +20,7 @@ namespace gdr {
 namespace {
 
 constexpr int kThreads = 128;   // threads per block; 8 channels each
-constexpr int kTokens = 16;     // tokens per run
+constexpr int kTokens = 8;      // tokens per run
 
 struct ConvParams {
   const uint16_t *x;

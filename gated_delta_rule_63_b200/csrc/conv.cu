@@ -54,6 +54,8 @@ __device__ __forceinline__ void row8(const uint4 &u, float *f) { unpack8(u, f); 
 // the general path, whose taps come from the rows of their own sequence, from
 // the conv state, or are zero.
 __global__ void __launch_bounds__(kThreads) causal_conv_kernel(ConvParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int C = p.channels;
   const int c0 = (blockIdx.x * kThreads + threadIdx.x) * 8;   // first channel of this thread
   if (c0 >= C) return;
@@ -177,8 +179,7 @@ int launch_causal_conv(const void *x, const void *w, const void *cs_in, void *cs
   p.channels = channels;
   const int groups = channels / 8;
   dim3 grid((groups + kThreads - 1) / kThreads, total > 0 ? (total + kTokens - 1) / kTokens : 1);
-  causal_conv_kernel<<<grid, kThreads, 0, s>>>(p);
-  return last_launch_status();
+  return launch_status(launch_pdl(causal_conv_kernel, grid, dim3(kThreads), 0, s, 1, p), "conv: kernel launch");
 }
 
 }  // namespace gdr

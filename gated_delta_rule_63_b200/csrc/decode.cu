@@ -83,6 +83,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   float *S = p.state + (static_cast<size_t>(n) * p.hv + h) * D * D;
   const int row0 = warp * 16;
   const uint32_t bar = smem_u32(&s_bar);
+  grid_dep_wait();     // the previous step's state and conv state are complete
+  grid_dep_launch();   // the next step's CTAs may take the SMs this grid frees
   if (tid == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
@@ -244,19 +246,9 @@ int launch_decode(const void *x, const void *conv_w, void *conv_state, const voi
     if (e != cudaSuccess) return launch_status(e, "decode: shared memory opt-in");
     smem_set[dev] = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(hv, batch, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kTileBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.group;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return launch_status(cudaLaunchKernelEx(&cfg, decode_kernel, p));
+  return launch_status(launch_pdl(decode_kernel, dim3(hv, batch, 1), dim3(kThreads), kTileBytes, s,
+                                  static_cast<unsigned>(p.group), p),
+                       "decode: kernel launch");
 }
 
 }  // namespace gdr

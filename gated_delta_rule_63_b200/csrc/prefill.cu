@@ -180,6 +180,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
   PTIME_INIT();
+  grid_dep_wait();
+  grid_dep_launch();
   const int cw = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
   const int seq_start = p.cu[n], seq_end = p.cu[n + 1];
   const int t0 = seq_start + (p.win0 + cw) * C;
@@ -660,6 +662,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              PrefillParams p) {
   PTIME_INIT();
+  grid_dep_wait();
+  grid_dep_launch();
   const int slice = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
   const int seq_start = p.cu[n], seq_end = p.cu[n + 1];
   const int n_all = (seq_end - seq_start + C - 1) / C;
@@ -1186,28 +1190,17 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
     p.state_out = last ? hT : (carry_in_ws ? carry_buf : hT);
     const int nc = std::min(win, max_chunks - p.win0);
     if (nc > 0) {
-      prep_kernel<<<dim3(nc, hv, n_seqs), kPrepThreads, P_SMEM, s>>>(tq, tk, tv, p);
-      st = last_launch_status("prefill: prep kernel launch");
+      st = launch_status(launch_pdl(prep_kernel, dim3(nc, hv, n_seqs), dim3(kPrepThreads), P_SMEM, s, 1, tq, tk, tv, p),
+                         "prefill: prep kernel launch");
       if (st) return st;
     }
-    if (y) {   // fused norm: the two dv slices of a head form a cluster and exchange row sums
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(NS, hv, n_seqs);
-      cfg.blockDim = dim3(kChainThreads, 1, 1);
-      cfg.dynamicSmemBytes = C_SMEM;
-      cfg.stream = s;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = NS;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      st = launch_status(cudaLaunchKernelEx(&cfg, chain_kernel<true>, tq, tk, p), "prefill: chain kernel launch");
-    } else {
-      chain_kernel<false><<<dim3(NS, hv, n_seqs), kChainThreads, C_SMEM, s>>>(tq, tk, p);
-      st = last_launch_status("prefill: chain kernel launch");
-    }
+    // with the fused norm the two dv slices of a head form a cluster and exchange row sums
+    st = y ? launch_status(launch_pdl(chain_kernel<true>, dim3(NS, hv, n_seqs), dim3(kChainThreads), C_SMEM, s,
+                                      static_cast<unsigned>(NS), tq, tk, p),
+                           "prefill: chain kernel launch")
+           : launch_status(launch_pdl(chain_kernel<false>, dim3(NS, hv, n_seqs), dim3(kChainThreads), C_SMEM, s, 1,
+                                      tq, tk, p),
+                           "prefill: chain kernel launch");
     if (st) return st;
   }
   return GDR_OK;

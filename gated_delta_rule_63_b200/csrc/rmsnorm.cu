@@ -22,6 +22,8 @@ constexpr int kRowsPerBlock = kThreads / 16;
 __global__ void __launch_bounds__(kThreads) gated_rmsnorm_kernel(const uint16_t *o, const uint16_t *z,
                                                                  const float *w, float eps,
                                                                  int64_t rows, uint16_t *y) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + (threadIdx.x >> 4);
   const int part = threadIdx.x & 15;   // 8 columns each
   float ov[8], zv[8];
@@ -61,10 +63,10 @@ int launch_gated_rmsnorm(const void *o, const void *z, const float *w, float eps
                          void *y, cudaStream_t s) {
   const int64_t blocks = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
   if (blocks > 0x7FFFFFFF) return GDR_ERR_SHAPE;
-  gated_rmsnorm_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
-      static_cast<const uint16_t *>(o), static_cast<const uint16_t *>(z), w, eps, rows,
-      static_cast<uint16_t *>(y));
-  return last_launch_status();
+  return launch_status(launch_pdl(gated_rmsnorm_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, s, 1,
+                                  static_cast<const uint16_t *>(o), static_cast<const uint16_t *>(z), w, eps,
+                                  rows, static_cast<uint16_t *>(y)),
+                       "gated norm: kernel launch");
 }
 
 }  // namespace gdr

@@ -217,7 +217,7 @@ int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_st
     if (overlaps(o, out_bytes, y, out_bytes)) return GDR_ERR_ALIAS;
   }
   return launch_chunk_prefill(q, k, v, qk_stride, v_stride, a, b, A_log, dt_bias, scale, hk, hv,
-                              cu_dev, n_seqs, total, max_chunks, h0, hT, o, z, norm_w, eps, y, workspace,
+                              cu_dev, cu_host, n_seqs, total, max_chunks, h0, hT, o, z, norm_w, eps, y, workspace,
                               workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 

@@ -68,7 +68,7 @@ int launch_decode(const void *x, const void *conv_w, void *conv_state, const voi
 int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_stride,
                          int64_t v_stride, const void *a, const void *b,
                          const float *A_log, const float *dt_bias, float scale, int hk, int hv,
-                         const int32_t *cu_dev, int n_seqs, int total, int max_chunks,
+                         const int32_t *cu_dev, const int32_t *cu_host, int n_seqs, int total, int max_chunks,
                          const float *h0, float *hT, void *o, const void *z, const float *norm_w,
                          float eps, void *y, void *workspace, size_t ws_bytes, cudaStream_t s);
 size_t chunk_prefill_workspace_bytes(int n_seqs, int hv, int window_chunks, bool need_carry);

@@ -60,24 +60,31 @@ constexpr uint32_t WS_REC = 82944;       // record size (81 KiB)
 
 // ---- prep kernel -------------------------------------------------------------
 constexpr int kPrepThreads = 256;
+// Three prep CTAs share an SM (67 KB of shared memory, 128 TMEM columns and 80
+// registers a thread each), so regions are reused as the chunk moves on:
+//   k-block kb (16 KB): K rows (8 KB) | Q rows (8 KB); once K K^T and Q K^T are
+//     done the Q half stages Mq (lo in kb 0, hi in kb 1), then receives V
+//     (dv block kb); after the W product the K half takes W_hi, and after the
+//     Ut product the Q half takes W_lo.
+//   T region (32 KB): A / T^T and the X^T scratch during the inverse, then
+//     T'_hi, T'_lo, T''_hi, T''_lo, then Ut (fp32).
 constexpr uint32_t P_KQ_KB = 128 * 128;              // [K rows 0..63 | Q rows 64..127] per k-block
 constexpr uint32_t P_OFF_KQ = 0;                     // 2 k-blocks
-constexpr uint32_t P_OFF_V = P_OFF_KQ + 2 * P_KQ_KB; // V [dv block 2][64 rows][128 B]
-constexpr uint32_t P_OFF_T = P_OFF_V + 2 * BLK64;    // T'_hi, T'_lo, T''_hi, T''_lo
+constexpr uint32_t P_Q_HALF = 64 * 128;              // offset of the Q half in a k-block
+constexpr uint32_t P_OFF_T = P_OFF_KQ + 2 * P_KQ_KB; // T'_hi, T'_lo, T''_hi, T''_lo
 constexpr int LD = 68;                               // fp32 row stride of AT (rows 16-byte aligned)
 constexpr int XLD = 20;                              // fp32 row stride of the 16 x 16 X^T blocks
 constexpr int XLD2 = 36;                             // fp32 row stride of the 32 x 32 X^T block
-constexpr uint32_t P_OFF_AT = P_OFF_T + 4 * BLK64;   // A below / T^T on and above the diagonal
+constexpr uint32_t P_OFF_AT = P_OFF_T;               // A below / T^T on and above the diagonal
 constexpr uint32_t P_OFF_XF = P_OFF_AT + 64 * LD * 4;
-constexpr uint32_t P_OFF_SC = P_OFF_XF + 32 * XLD2 * 4;  // gamma, rq, rk, beta, e^gamma, block decay, e^g
+constexpr uint32_t P_OFF_SC = P_OFF_T + 4 * BLK64;   // gamma, rq, rk, beta, e^gamma, block decay, e^g
 static_assert(32 * XLD2 >= 3 * 16 * XLD, "X^T scratch holds both block sizes");
-constexpr uint32_t P_OFF_BAR = P_OFF_SC + 7 * 64 * 4;
-constexpr uint32_t P_SMEM = P_OFF_BAR + 32 + 1024;
-static_assert((P_OFF_V | P_OFF_T) % 1024 == 0, "swizzled tiles need 1 KB alignment");
-constexpr uint32_t P_TM_COLS = 256;                  // two prep CTAs per SM
-constexpr uint32_t P_COL_S = 0;                      // [K K^T ; Q K^T] (64 cols, dead once A and Mq are built)
-constexpr uint32_t P_COL_W = 0;                      // W = T' K, lanes 0..63 (128 cols)
-constexpr uint32_t P_COL_U = 128;                    // Ut = T'' V, lanes 64..127 (128 cols)
+static_assert(P_OFF_XF + 32 * XLD2 * 4 <= P_OFF_SC, "the inverse's scratch fits the T region");
+constexpr uint32_t P_OFF_BAR = P_OFF_SC + 7 * 64 * 4;   // 4 mbarriers, TMEM base
+constexpr uint32_t P_SMEM = P_OFF_BAR + 48 + 1024;
+static_assert(P_OFF_T % 1024 == 0, "swizzled tiles need 1 KB alignment");
+static_assert(3 * (P_SMEM + 1024) <= 228 * 1024, "three prep CTAs per SM");
+constexpr uint32_t P_TM_COLS = 128;                  // [K K^T ; Q K^T] (64 cols), then W, then Ut
 
 // ---- chain kernel ------------------------------------------------------------
 constexpr int kChainThreads = 288;                    // warps 0..7 state and output, warp 8 control
@@ -132,7 +139,13 @@ __device__ long long *g_prefill_times;
   } while (0)
 #endif
 
+// cu_seqlens travels in the launch parameters when there are at most kCuParam
+// sequences (a constant-bank read instead of a dependent global load at CTA start)
+constexpr int kCuParam = 64;
+
 struct PrefillParams {
+  int n_seqs;
+  int cu_param[kCuParam + 1];
   const uint16_t *a, *b;
   const float *A_log, *dt_bias;
   float scale;
@@ -169,6 +182,10 @@ __device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity, int *err
   return ok;
 }
 
+__device__ __forceinline__ int cu_at(const PrefillParams &p, int i) {
+  return p.n_seqs <= kCuParam ? p.cu_param[i] : __ldg(p.cu + i);
+}
+
 __device__ __forceinline__ uint8_t *ws_record(const PrefillParams &p, int n, int h, int cw) {
   return p.ws + ((static_cast<size_t>(n) * p.hv + h) * p.win_chunks + cw) * WS_REC;
 }
@@ -176,14 +193,14 @@ __device__ __forceinline__ uint8_t *ws_record(const PrefillParams &p, int n, int
 // =============================================================================
 // prep: one chunk of one value head
 // =============================================================================
-__global__ void __launch_bounds__(kPrepThreads, 2)
+__global__ void __launch_bounds__(kPrepThreads, 3)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-            const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
+            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ PrefillParams p) {
   PTIME_INIT();
   grid_dep_wait();
   grid_dep_launch();
   const int cw = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
-  const int seq_start = p.cu[n], seq_end = p.cu[n + 1];
+  const int seq_start = cu_at(p, n), seq_end = cu_at(p, n + 1);
   const int t0 = seq_start + (p.win0 + cw) * C;
   if (t0 >= seq_end) return;   // the window runs past this sequence (uniform exit)
   const int L = min(C, seq_end - t0);
@@ -200,7 +217,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   float *s_rq = s_g + 64, *s_rk = s_g + 128, *s_beta = s_g + 192, *s_eg = s_g + 256, *s_eb = s_g + 320;
   float *s_e1 = s_g + 384;   // e^(g_t): one step of decay
   const uint32_t bar_tma = sbase + P_OFF_BAR, bar_mma = sbase + P_OFF_BAR + 8;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + P_OFF_BAR + 16);
+  const uint32_t bar_v = sbase + P_OFF_BAR + 16, bar_u = sbase + P_OFF_BAR + 24;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + P_OFF_BAR + 32);
+  const uint32_t q_half0 = sbase + P_OFF_KQ + P_Q_HALF, q_half1 = q_half0 + P_KQ_KB;
   uint8_t *rec = ws_record(p, n, h, cw);
 
   if (warp == 0) {
@@ -210,13 +229,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   if (tid == 0) {
     mbar_init(bar_tma, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_u, 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar_tma, 6 * BLK64);
+    mbar_arrive_expect_tx(bar_tma, 4 * BLK64);
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb) {
       tma_load_2d(sbase + P_OFF_KQ + kb * P_KQ_KB, &tm_k, kh * D + kb * 64, t0, bar_tma);
-      tma_load_2d(sbase + P_OFF_KQ + kb * P_KQ_KB + 64 * 128, &tm_q, kh * D + kb * 64, t0, bar_tma);
-      tma_load_2d(sbase + P_OFF_V + kb * BLK64, &tm_v, h * D + kb * 64, t0, bar_tma);
+      tma_load_2d(sbase + P_OFF_KQ + kb * P_KQ_KB + P_Q_HALF, &tm_q, kh * D + kb * 64, t0, bar_tma);
     }
   }
   // gates of the chunk's rows; padding rows get no decay and no write
@@ -240,10 +260,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
   if (ok && L < C) {   // rows past the sequence end hold other tokens: zero them
     const uint32_t nz = static_cast<uint32_t>(C - L) * 16;   // rows x 16-B chunks per tile
-    for (uint32_t e = tid; e < 3 * nz; e += kPrepThreads) {
+    for (uint32_t e = tid; e < 2 * nz; e += kPrepThreads) {   // K and Q (V when it arrives)
       const uint32_t tile = e / nz, rem = e % nz, r = L + rem / 16, cc = rem % 16;
-      const uint32_t base = tile == 2 ? P_OFF_V + (cc >> 3) * BLK64
-                                      : P_OFF_KQ + (cc >> 3) * P_KQ_KB + tile * 64 * 128;
+      const uint32_t base = P_OFF_KQ + (cc >> 3) * P_KQ_KB + tile * P_Q_HALF;
       st_shared16(sbase + base + sw128(r, cc & 7), make_uint4(0, 0, 0, 0));
     }
     fence_proxy_async();
@@ -257,7 +276,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t koff = (kk >> 2) * P_KQ_KB + (kk & 3) * 32;
-        mma_bf16(tmem + P_COL_S, sdesc(sbase + P_OFF_KQ + koff, 16, 1024),
+        mma_bf16(tmem, sdesc(sbase + P_OFF_KQ + koff, 16, 1024),
                  sdesc(sbase + P_OFF_KQ + koff, 16, 1024), id, kk > 0);
       }
       mma_commit(bar_mma);
@@ -344,7 +363,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
     }
     PTIME(0, 11);
-    tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + P_COL_S + 32 * hf, sv);
+    tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + 32 * hf, sv);
     tmem_wait_ld();
     if (row < 64) {   // A_ij = beta_i / |k_i| * (k_i.k_j) / |k_j| * e^(g_i - g_j), j < i
       // (columns j >= i hold junk until T^T overwrites them)
@@ -361,16 +380,22 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         float m[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) m[e] = sv[8 * c4 + e] * qi * colf[8 * c4 + e];
-        const uint32_t off = sw128(i, 4 * hf + c4);   // staged in the T region, stored in bulk
-        st_split8_shared(sbase + P_OFF_T + BLK64 + off, sbase + P_OFF_T + off, m);   // [Mq_lo | Mq_hi]
+        const uint32_t off = sw128(i, 4 * hf + c4);   // staged in the dead Q halves, stored in bulk
+        st_split8_shared(q_half1 + off, q_half0 + off, m);   // Mq_hi, Mq_lo
       }
     }
     PTIME(0, 12);
     fence_proxy_async();
     __syncthreads();
-    if (tid == 0) {   // Mq_lo | Mq_hi, contiguous in shared memory and in the record
-      bulk_store(rec + WS_MQ, sbase + P_OFF_T, 2 * BLK64);
+    if (tid == 128) {   // (a thread the inverse below leaves idle)
+      bulk_store(rec + WS_MQ, q_half0, BLK64);           // Mq_lo
+      bulk_store(rec + WS_MQ + BLK64, q_half1, BLK64);   // Mq_hi
       bulk_commit();
+      bulk_wait_read();
+      // V (dv block kb into the Q half of k-block kb), in flight during the inverse
+      mbar_arrive_expect_tx(bar_v, 2 * BLK64);
+      tma_load_2d(q_half0, &tm_v, h * D, t0, bar_v);
+      tma_load_2d(q_half1, &tm_v, h * D + 64, t0, bar_v);
     }
 
     PTIME(0, 4);
@@ -500,21 +525,26 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     PTIME(0, 5);
     // ---- T' = T diag(beta e^g / |k|), T'' = T diag(beta), hi/lo tiles --------
-    if (tid == 0) bulk_wait_read();   // the Mq staging is about to be overwritten
-    __syncthreads();
     {   // tiles with the row index r contiguous (MN-major operands): row j, 16-byte chunk r / 8
       const int j = tid & 63;
       const float f2 = s_beta[j], f1 = f2 * s_eg[j] * s_rk[j];
+      float tv[2][8];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int rg = (tid >> 6) + 4 * h, r0 = 8 * rg;
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r0 = 8 * ((tid >> 6) + 4 * hh);
         const float4 v0 = *reinterpret_cast<const float4 *>(AT + j * LD + r0);
         const float4 v1 = *reinterpret_cast<const float4 *>(AT + j * LD + r0 + 4);
-        const float tv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        tv[hh][0] = v0.x; tv[hh][1] = v0.y; tv[hh][2] = v0.z; tv[hh][3] = v0.w;
+        tv[hh][4] = v1.x; tv[hh][5] = v1.y; tv[hh][6] = v1.z; tv[hh][7] = v1.w;
+      }
+      __syncthreads();   // T^T is read out: the tiles take its place
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int rg = (tid >> 6) + 4 * hh, r0 = 8 * rg;
         float t1[8], t2[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float tij = (r0 + e >= j) ? tv[e] : 0.0f;   // T[r][j], lower triangle
+          const float tij = (r0 + e >= j) ? tv[hh][e] : 0.0f;   // T[r][j], lower triangle
           t1[e] = tij * f1;
           t2[e] = tij * f2;
         }
@@ -524,79 +554,123 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
     }
     fence_proxy_async();
-    __syncthreads();
+    ok = cta_wait(bar_v, 0, p.err);   // V has landed in the Q halves
+    if (ok && L < C) {   // rows past the sequence end hold other tokens: zero them
+      const uint32_t nz = static_cast<uint32_t>(C - L) * 16;
+      for (uint32_t e = tid; e < nz; e += kPrepThreads) {
+        const uint32_t r = L + e / 16, cc = e % 16;
+        st_shared16(q_half0 + (cc >> 3) * P_KQ_KB + sw128(r, cc & 7), make_uint4(0, 0, 0, 0));
+      }
+      fence_proxy_async();
+      __syncthreads();
+    }
 
     PTIME(0, 6);
-    // ---- W = T' K (rows in lanes 0..63) and Ut = T'' V (rows in lanes 64..127), one wait ----
-    // MN-major A operands of 128 rows: W's second row block and Ut's first are other tiles,
-    // whose products land in lanes that are never read
-    if (tid == 0) {
+    // ---- W = T' K (rows in lanes 0..63), then Ut = T'' V (rows in lanes 64..127) in the
+    // same TMEM columns once W has been read out.  MN-major A operands of 128 rows: W's
+    // second row block and Ut's first are other tiles, whose products land in lanes that
+    // are never read
+    if (ok && tid == 0) {
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 128, true, true);
 #pragma unroll
       for (int part = 0; part < 2; ++part)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + P_COL_W, sdesc(sbase + P_OFF_T + part * BLK64 + kk * 2048, BLK64, 1024),
+          mma_bf16(tmem, sdesc(sbase + P_OFF_T + part * BLK64 + kk * 2048, BLK64, 1024),
                    sdesc(sbase + P_OFF_KQ + kk * 2048, P_KQ_KB, 1024), id, (part | kk) != 0);
-#pragma unroll
-      for (int part = 0; part < 2; ++part)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + P_COL_U, sdesc(sbase + P_OFF_T + (1 + part) * BLK64 + kk * 2048, BLK64, 1024),
-                   sdesc(sbase + P_OFF_V + kk * 2048, BLK64, 1024), id, (part | kk) != 0);
       mma_commit(bar_mma);
     }
-    ok = cta_wait(bar_mma, 1, p.err);
   }
   PTIME(0, 7);
+  // ok is uniform across the CTA here; below, the warps of TMEM lanes 0..63 (W) and
+  // 64..127 (Ut) wait on their own products
+  bool good = ok;
   if (ok) {
     if ((warp & 2) == 0) {
-      // warps 0, 1, 4, 5 (lanes 0..63): W rows -> [W_hi kb0 | W_hi kb1 | W_lo kb0 | W_lo kb1]
-      // over the dead K/Q tiles; k-block = warp >> 2
+      // warps 0, 1, 4, 5: W rows of k-block kb = warp >> 2; W_hi goes into the K half at
+      // once (K is dead once W is done), W_lo into the Q half once Ut has read V there
       const int kb = warp >> 2, r = 32 * (warp & 1) + lane;
-      const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + P_COL_W + 64 * kb;
+      const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + 64 * kb;
+      const uint32_t hi_base = sbase + P_OFF_KQ + kb * P_KQ_KB, lo_base = hi_base + P_Q_HALF;
+      bool wok = lane == 0 ? mbar_wait(bar_mma, 1, p.err) : true;
+      wok = __shfl_sync(0xffffffffu, wok ? 1 : 0, 0) != 0;
+      tc_fence_after();
+      uint4 lo[8];
+      if (wok) {
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float w[32];
-        tmem_ld32(tl + 32 * hh, w);
-        tmem_wait_ld();
+        for (int hh = 0; hh < 2; ++hh) {
+          float w[32];
+          tmem_ld32(tl + 32 * hh, w);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const uint32_t off = kb * BLK64 + sw128(r, 4 * hh + c4);
-          st_split8_shared(sbase + P_OFF_KQ + off, sbase + P_OFF_KQ + 2 * BLK64 + off, w + 8 * c4);
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint4 hi;
+            split8x2(w + 8 * c4, hi, lo[4 * hh + c4]);
+            st_shared16(hi_base + sw128(r, 4 * hh + c4), hi);
+          }
         }
       }
+      tc_fence_before();
+      const bool all_w = named_sync_or(1, 128, !wok) == false;   // W is out of TMEM
+      if (tid == 0 && all_w) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, 128, true, true);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem, sdesc(sbase + P_OFF_T + (1 + part) * BLK64 + kk * 2048, BLK64, 1024),
+                     sdesc(q_half0 + kk * 2048, P_KQ_KB, 1024), id, (part | kk) != 0);
+        mma_commit(bar_u);
+      }
+      bool uok = all_w;
+      if (lane == 0 && uok) uok = mbar_wait(bar_u, 0, p.err);
+      uok = __shfl_sync(0xffffffffu, uok ? 1 : 0, 0) != 0;
+      if (uok) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) st_shared16(lo_base + sw128(r, i), lo[i]);
+      }
+      good = uok;
     } else {
       // warps 2, 3, 6, 7 (lanes 64..127): Ut rows -> fp32 [slice][row][64] over the T tiles
       const int sl = warp >> 2, r = 32 * (warp & 1) + lane;
-      const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + P_COL_U + 64 * sl;
+      const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + 64 * sl;
       const uint32_t dst = sbase + P_OFF_T + (static_cast<uint32_t>(sl) * 64 + r) * 256;
+      bool uok = lane == 0 ? mbar_wait(bar_u, 0, p.err) : true;
+      uok = __shfl_sync(0xffffffffu, uok ? 1 : 0, 0) != 0;
+      tc_fence_after();
+      if (uok) {
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float u[32];
-        tmem_ld32(tl + 32 * hh, u);
-        tmem_wait_ld();
+        for (int hh = 0; hh < 2; ++hh) {
+          float u[32];
+          tmem_ld32(tl + 32 * hh, u);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const uint32_t j = (8 * hh + c4) ^ (r & 7);
-          st_shared16(dst + 16 * j, make_uint4(__float_as_uint(u[4 * c4]), __float_as_uint(u[4 * c4 + 1]),
-                                               __float_as_uint(u[4 * c4 + 2]), __float_as_uint(u[4 * c4 + 3])));
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const uint32_t j = (8 * hh + c4) ^ (r & 7);
+            st_shared16(dst + 16 * j, make_uint4(__float_as_uint(u[4 * c4]), __float_as_uint(u[4 * c4 + 1]),
+                                                 __float_as_uint(u[4 * c4 + 2]), __float_as_uint(u[4 * c4 + 3])));
+          }
         }
       }
+      good = uok;
     }
   }
   PTIME(0, 9);
   fence_proxy_async();
   tc_fence_before();
-  __syncthreads();
+  ok = __syncthreads_and(good) != 0;
   if (tid == 0) {
     if (ok) {
-      bulk_store(rec + WS_W_HI, sbase + P_OFF_KQ, 4 * BLK64);
+      bulk_store(rec + WS_W_HI, sbase + P_OFF_KQ, BLK64);                     // W_hi, k-block 0
+      bulk_store(rec + WS_W_HI + BLK64, sbase + P_OFF_KQ + P_KQ_KB, BLK64);   // W_hi, k-block 1
+      bulk_store(rec + WS_W_LO, q_half0, BLK64);                              // W_lo, k-block 0
+      bulk_store(rec + WS_W_LO + BLK64, q_half1, BLK64);                      // W_lo, k-block 1
       bulk_store(rec + WS_UT, sbase + P_OFF_T, 4 * BLK64);
       bulk_commit();
     }
-    bulk_wait_all();   // the stores must finish before the shared memory goes away
+    bulk_wait_read();   // the stores have read the shared memory before it goes away
   }
   PTIME(0, 10);
   if (warp == 0) tmem_dealloc(tmem, P_TM_COLS);
@@ -660,12 +734,12 @@ __device__ __forceinline__ bool chain_wait_cluster(uint32_t bar, uint32_t parity
 template <bool kNorm>   // gated RMSNorm fused into the output (p.y set, cluster of the two dv slices)
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-             PrefillParams p) {
+             const __grid_constant__ PrefillParams p) {
   PTIME_INIT();
   grid_dep_wait();
   grid_dep_launch();
   const int slice = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
-  const int seq_start = p.cu[n], seq_end = p.cu[n + 1];
+  const int seq_start = cu_at(p, n), seq_end = cu_at(p, n + 1);
   const int n_all = (seq_end - seq_start + C - 1) / C;
   const int c_end = min(n_all, p.win0 + p.win_chunks);
   const int nw = max(0, c_end - p.win0);              // chunks of this window
@@ -1114,6 +1188,9 @@ int ensure_smem_attrs() {
   const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
   if (bit && (done.load(std::memory_order_acquire) & bit)) return GDR_OK;
   e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+  if (e == cudaSuccess)   // room for three prep CTAs per SM
+    e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
   if (e == cudaSuccess)
@@ -1134,7 +1211,7 @@ size_t chunk_prefill_workspace_bytes(int n_seqs, int hv, int window_chunks, bool
 int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_stride,
                          int64_t v_stride, const void *a, const void *b,
                          const float *A_log, const float *dt_bias, float scale, int hk, int hv,
-                         const int32_t *cu_dev, int n_seqs, int total, int max_chunks,
+                         const int32_t *cu_dev, const int32_t *cu_host, int n_seqs, int total, int max_chunks,
                          const float *h0, float *hT, void *o, const void *z, const float *norm_w,
                          float eps, void *y, void *workspace, size_t ws_bytes, cudaStream_t s) {
   if (n_seqs > 65535 || hv > 65535) return GDR_ERR_SHAPE;
@@ -1174,6 +1251,8 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   p.hv = hv;
   p.group = hv / hk;
   p.cu = cu_dev;
+  p.n_seqs = n_seqs;
+  for (int i = 0; i <= kCuParam; ++i) p.cu_param[i] = i <= n_seqs ? cu_host[i] : 0;
   p.ws = static_cast<uint8_t *>(workspace);
   p.win_chunks = win;
   p.o = static_cast<uint16_t *>(o);

@@ -5,13 +5,20 @@
 // SiLU(sum_j w[c][j] x[t-3+j][c]), fp32 math, bf16 output; inputs before a
 // sequence start come from the conv state (oldest first) or are zero.
 //
-// Memory-bound: each thread owns 8 adjacent channels (one 16-byte vector) of
-// a run of kTokens tokens; the run's rows and its 3-row halo are loaded up
-// front so that all its loads are in flight together.  x is read once (plus
-// the halo, mostly from L2) and y written once, with coalesced 16-byte
-// accesses.
+// Memory-bound stencil.  The input is cut into tiles of 64 tokens x 128
+// channels; a tile and its 3-row halo (67 rows x 256 bytes) arrive in shared
+// memory by one TMA copy.  CTAs are persistent (five per SM) and keep two
+// tiles in flight: while one tile is computed the next is loading, so the
+// SM's copies stream continuously and x is read from HBM once (the halo rows
+// are L2 hits).  Each thread computes 8 channels (one 16-byte vector) of 8
+// tokens from a sliding window of unpacked rows and writes y with coalesced
+// 16-byte stores.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <algorithm>
+#include <atomic>
 
 #include "gdr_common.cuh"
 #include "gdr_host.h"
@@ -19,11 +26,17 @@
 namespace gdr {
 namespace {
 
-constexpr int kThreads = 128;   // threads per block; 8 channels each
-constexpr int kTokens = 8;      // tokens per run
+constexpr int kThreads = 128;                 // 16 channel groups x 8 token groups
+constexpr int kTileT = 64;                    // tokens per tile
+constexpr int kTileC = 128;                   // channels per tile
+constexpr int kRows = kTileT + 3;             // with the 3-row halo
+constexpr uint32_t kRowBytes = kTileC * 2;    // 256
+constexpr uint32_t kBufBytes = kRows * kRowBytes;
+constexpr int kBufs = 2;                      // tiles in flight per CTA
+constexpr int kCtasPerSm = 5;
+constexpr uint32_t kSmem = kBufs * kBufBytes + 1024;   // tile buffers, 1 KB alignment slack
 
 struct ConvParams {
-  const uint16_t *x;
   const uint16_t *w;
   const uint16_t *cs_in;
   uint16_t *cs_out;
@@ -32,6 +45,9 @@ struct ConvParams {
   int n_seqs;
   int total;
   int channels;
+  int n_ctiles;   // channel tiles
+  int n_tiles;    // channel tiles x token tiles
+  int *err;
 };
 
 // sequence containing token t: largest n with cu[n] <= t (skipping empty ones)
@@ -44,122 +60,150 @@ __device__ int seq_of(const int32_t *cu, int n_seqs, int t) {
   return lo;
 }
 
-// unpack the 8 bf16 of a 16-byte row into floats (one integer op each)
-__device__ __forceinline__ void row8(const uint4 &u, float *f) { unpack8(u, f); }
+__device__ __forceinline__ void load_tile(const CUtensorMap *tm, uint32_t dst, uint32_t bar, int tile,
+                                          const ConvParams &p) {
+  const int ct = tile % p.n_ctiles, tt = tile / p.n_ctiles;
+  mbar_arrive_expect_tx(bar, kBufBytes);
+  // rows before token 0 and past the last token read as zero
+  tma_load_2d(dst, tm, ct * kTileC, tt * kTileT - 3, bar);
+}
 
-// Each thread: 8 channels x kTokens tokens.  A run that lies inside one
-// sequence (the common case) loads all kTokens + 3 input rows up front
-// (independent 16-byte loads in flight) and unpacks every row once into a
-// sliding window of four; a run that touches a sequence start or end takes
-// the general path, whose taps come from the rows of their own sequence, from
-// the conv state, or are zero.
-__global__ void __launch_bounds__(kThreads) causal_conv_kernel(ConvParams p) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+causal_conv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ ConvParams p) {
   grid_dep_wait();
   grid_dep_launch();
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ alignas(8) uint64_t s_bar[kBufs];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int tid = threadIdx.x;
   const int C = p.channels;
-  const int c0 = (blockIdx.x * kThreads + threadIdx.x) * 8;   // first channel of this thread
-  if (c0 >= C) return;
-  const int t_begin = blockIdx.y * kTokens;
+  const uint32_t bar0 = smem_u32(&s_bar[0]);
 
-  // empty sequences: their conv state passes through unchanged (run once)
-  if (blockIdx.y == 0 && p.cs_out) {
+  if (tid == 0) {
+    for (int i = 0; i < kBufs; ++i) mbar_init(bar0 + 8 * i, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_x);
+    for (int i = 0; i < kBufs; ++i) {
+      const int tile = blockIdx.x + i * gridDim.x;
+      if (tile < p.n_tiles) load_tile(&tm_x, sbase + i * kBufBytes, bar0 + 8 * i, tile, p);
+    }
+  }
+  // empty sequences: their conv state passes through unchanged (first CTA)
+  if (blockIdx.x == 0 && p.cs_out) {
     for (int n = 0; n < p.n_seqs; ++n) {
       if (__ldg(p.cu + n + 1) != __ldg(p.cu + n)) continue;
-      for (int s = 0; s < 3; ++s) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (p.cs_in) v = *reinterpret_cast<const uint4 *>(p.cs_in + (static_cast<size_t>(n) * 3 + s) * C + c0);
-        *reinterpret_cast<uint4 *>(p.cs_out + (static_cast<size_t>(n) * 3 + s) * C + c0) = v;
-      }
-    }
-  }
-  if (t_begin >= p.total) return;
-  const int t_end = min(t_begin + kTokens, p.total);
-
-  float w[4][8];
-  {
-    // w is [C][4]: channels c0..c0+7 occupy 32 contiguous bf16
-    const uint4 *wp = reinterpret_cast<const uint4 *>(p.w + static_cast<size_t>(c0) * 4);
-    float tmp[32];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) unpack8(__ldg(wp + i), tmp + 8 * i);
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) w[j][ch] = tmp[ch * 4 + j];
-  }
-  int n = seq_of(p.cu, p.n_seqs, t_begin);
-  int seq_start = __ldg(p.cu + n), seq_end = __ldg(p.cu + n + 1);
-
-  if (t_begin - 3 >= seq_start && t_begin + kTokens < seq_end) {
-    // ---- inside one sequence, not its last token: no state, no boundary ----
-    uint4 raw[kTokens + 3];   // rows t_begin - 3 .. t_begin + kTokens - 1
-#pragma unroll
-    for (int i = 0; i < kTokens + 3; ++i)
-      raw[i] = __ldg(reinterpret_cast<const uint4 *>(p.x + static_cast<size_t>(t_begin - 3 + i) * C + c0));
-    float xw[4][8];
-#pragma unroll
-    for (int j = 0; j < 3; ++j) row8(raw[j], xw[j]);
-#pragma unroll
-    for (int i = 0; i < kTokens; ++i) {
-      row8(raw[i + 3], xw[(i + 3) & 3]);
-      float out[8];
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const float acc = w[0][ch] * xw[i & 3][ch] + w[1][ch] * xw[(i + 1) & 3][ch] +
-                          w[2][ch] * xw[(i + 2) & 3][ch] + w[3][ch] * xw[(i + 3) & 3][ch];
-        out[ch] = silu_fast(acc);
-      }
-      *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(t_begin + i) * C + c0) = pack8x2(out);
-    }
-    return;
-  }
-
-  // ---- general path: sequence starts / ends inside the run ----
-#pragma unroll 1
-  for (int i = 0; i < kTokens; ++i) {
-    const int t = t_begin + i;
-    if (t >= t_end) break;
-    while (t >= seq_end) {   // next non-empty sequence
-      ++n;
-      seq_start = __ldg(p.cu + n);
-      seq_end = __ldg(p.cu + n + 1);
-    }
-    float acc[8];
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) acc[ch] = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int pos = t - 3 + j;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (pos >= seq_start) {   // (re-read: this path is rare and the row sits in L1 / L2)
-        v = __ldg(reinterpret_cast<const uint4 *>(p.x + static_cast<size_t>(pos) * C + c0));
-      } else if (p.cs_in) {   // before the sequence start: the conv state, oldest first
-        const int slot = 3 - (seq_start - pos);   // 1..3 positions before the start
-        v = *reinterpret_cast<const uint4 *>(p.cs_in + (static_cast<size_t>(n) * 3 + slot) * C + c0);
-      }
-      float xv[8];
-      unpack8(v, xv);
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) acc[ch] += w[j][ch] * xv[ch];
-    }
-    float out[8];
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) out[ch] = silu_fast(acc[ch]);
-    *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(t) * C + c0) = pack8x2(out);
-    if (t == seq_end - 1 && p.cs_out) {   // last token: the last three inputs are the new conv state
-#pragma unroll
-      for (int s = 0; s < 3; ++s) {
-        const int pos = t - 2 + s;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (pos >= seq_start) {
-          v = __ldg(reinterpret_cast<const uint4 *>(p.x + static_cast<size_t>(pos) * C + c0));
-        } else if (p.cs_in) {
-          v = *reinterpret_cast<const uint4 *>(p.cs_in + (static_cast<size_t>(n) * 3 + (3 - (seq_start - pos))) * C + c0);
+      for (int c = tid * 8; c < C; c += kThreads * 8)
+        for (int s = 0; s < 3; ++s) {
+          const size_t at = (static_cast<size_t>(n) * 3 + s) * C + c;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (p.cs_in) v = *reinterpret_cast<const uint4 *>(p.cs_in + at);
+          *reinterpret_cast<uint4 *>(p.cs_out + at) = v;
         }
-        *reinterpret_cast<uint4 *>(p.cs_out + (static_cast<size_t>(n) * 3 + s) * C + c0) = v;
-      }
     }
   }
+  __syncthreads();   // barriers initialised
+
+  const int cg = tid & 15, tg = tid >> 4;   // channel group, token group
+  int k = 0;
+  for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++k) {
+    const int buf = k % kBufs;
+    const uint32_t parity = (k / kBufs) & 1;
+    const int ct = tile % p.n_ctiles, tt = tile / p.n_ctiles;
+    const int c0 = ct * kTileC + cg * 8;          // first channel of this thread
+    const int row0 = tt * kTileT - 3;             // token of tile row 0
+    const int tb = tt * kTileT + tg * 8;          // first token of this thread
+    const uint32_t tbuf = sbase + buf * kBufBytes + cg * 16;
+    const bool ok = mbar_wait(bar0 + 8 * buf, parity, p.err);
+    if (ok && c0 < C && tb < p.total) {
+      float w[4][8];
+      {   // w is [C][4]: channels c0..c0+7 occupy 32 contiguous bf16
+        const uint4 *wp = reinterpret_cast<const uint4 *>(p.w + static_cast<size_t>(c0) * 4);
+        float tmp[32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) unpack8(__ldg(wp + i), tmp + 8 * i);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) w[j][ch] = tmp[ch * 4 + j];
+      }
+      auto row = [&](int t) { return ld_shared16(tbuf + (t - row0) * kRowBytes); };   // token t's 8 inputs
+      int n = seq_of(p.cu, p.n_seqs, tb);
+      int seq_start = __ldg(p.cu + n), seq_end = __ldg(p.cu + n + 1);
+      if (tb - 3 >= seq_start && tb + 8 < seq_end) {
+        // ---- inside one sequence, not its last token: no state, no boundary ----
+        float xw[4][8];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) unpack8(row(tb - 3 + j), xw[j]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          unpack8(row(tb + i), xw[(i + 3) & 3]);
+          float out[8];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const float acc = w[0][ch] * xw[i & 3][ch] + w[1][ch] * xw[(i + 1) & 3][ch] +
+                              w[2][ch] * xw[(i + 2) & 3][ch] + w[3][ch] * xw[(i + 3) & 3][ch];
+            out[ch] = silu_fast(acc);
+          }
+          *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(tb + i) * C + c0) = pack8x2(out);
+        }
+      } else {
+        // ---- sequence starts / ends among these tokens ----
+        const int te = min(tb + 8, p.total);
+#pragma unroll 1
+        for (int t = tb; t < te; ++t) {
+          while (t >= seq_end) {   // next non-empty sequence
+            ++n;
+            seq_start = __ldg(p.cu + n);
+            seq_end = __ldg(p.cu + n + 1);
+          }
+          // input at position pos of sequence n: the tile row, or the conv state before the start
+          auto tap = [&](int pos) {
+            if (pos >= seq_start) return row(pos);
+            if (p.cs_in)   // 1..3 positions before the start: the conv state, oldest first
+              return *reinterpret_cast<const uint4 *>(
+                  p.cs_in + (static_cast<size_t>(n) * 3 + (3 - (seq_start - pos))) * C + c0);
+            return make_uint4(0, 0, 0, 0);
+          };
+          float acc[8];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) acc[ch] = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float xv[8];
+            unpack8(tap(t - 3 + j), xv);
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) acc[ch] += w[j][ch] * xv[ch];
+          }
+          float out[8];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) out[ch] = silu_fast(acc[ch]);
+          *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(t) * C + c0) = pack8x2(out);
+          if (t == seq_end - 1 && p.cs_out) {   // last token: the last three inputs are the new conv state
+#pragma unroll
+            for (int s = 0; s < 3; ++s)
+              *reinterpret_cast<uint4 *>(p.cs_out + (static_cast<size_t>(n) * 3 + s) * C + c0) = tap(t - 2 + s);
+          }
+        }
+      }
+    }
+    __syncthreads();   // every thread is done with this buffer
+    if (tid == 0) {
+      const int next = tile + kBufs * gridDim.x;
+      if (next < p.n_tiles) load_tile(&tm_x, sbase + buf * kBufBytes, bar0 + 8 * buf, next, p);
+    }
+  }
+}
+
+int conv_grid(int n_tiles) {
+  static std::atomic<int> sms[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  int n = dev >= 0 && dev < 64 ? sms[dev].load(std::memory_order_relaxed) : 0;
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return -1;
+    if (dev >= 0 && dev < 64) sms[dev].store(n, std::memory_order_relaxed);
+  }
+  return std::max(1, std::min(n_tiles, n * kCtasPerSm));
 }
 
 }  // namespace
@@ -167,8 +211,20 @@ __global__ void __launch_bounds__(kThreads) causal_conv_kernel(ConvParams p) {
 int launch_causal_conv(const void *x, const void *w, const void *cs_in, void *cs_out,
                        const int32_t *cu_dev, int n_seqs, int total, int channels, void *y,
                        cudaStream_t s) {
+  static std::atomic<uint64_t> attr_done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return launch_status(e, "conv: cudaGetDevice");
+  const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (!bit || !(attr_done.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(causal_conv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(causal_conv_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return launch_status(e, "conv: shared memory opt-in");
+    attr_done.fetch_or(bit, std::memory_order_acq_rel);
+  }
   ConvParams p;
-  p.x = static_cast<const uint16_t *>(x);
   p.w = static_cast<const uint16_t *>(w);
   p.cs_in = static_cast<const uint16_t *>(cs_in);
   p.cs_out = static_cast<uint16_t *>(cs_out);
@@ -177,9 +233,28 @@ int launch_causal_conv(const void *x, const void *w, const void *cs_in, void *cs
   p.n_seqs = n_seqs;
   p.total = total;
   p.channels = channels;
-  const int groups = channels / 8;
-  dim3 grid((groups + kThreads - 1) / kThreads, total > 0 ? (total + kTokens - 1) / kTokens : 1);
-  return launch_status(launch_pdl(causal_conv_kernel, grid, dim3(kThreads), 0, s, 1, p), "conv: kernel launch");
+  p.n_ctiles = (channels + kTileC - 1) / kTileC;
+  const int64_t n_tiles = static_cast<int64_t>(p.n_ctiles) * ((total + kTileT - 1) / kTileT);
+  if (n_tiles > 0x7FFFFFFF) return GDR_ERR_SHAPE;
+  p.n_tiles = static_cast<int>(n_tiles);
+  p.err = device_error_ptr();
+  // x as [total rows][channels] bf16; boxes of 67 rows x 128 channels, no swizzle;
+  // with no tokens no tile is loaded and the weights serve as a base address
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return launch_status(cudaErrorSymbolNotFound, "conv: cuTensorMapEncodeTiled lookup");
+  CUtensorMap tm;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(channels), static_cast<cuuint64_t>(total > 0 ? total : 1)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(channels) * 2};
+  const cuuint32_t box[2] = {kTileC, kRows};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(total > 0 ? x : w), dims, strides, box,
+          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return launch_status(cudaErrorInvalidValue, "conv: tensor map encoding");
+  const int grid = conv_grid(p.n_tiles);
+  if (grid < 0) return launch_status(cudaErrorInvalidDevice, "conv: SM count");
+  return launch_status(launch_pdl(causal_conv_kernel, dim3(grid), dim3(kThreads), kSmem, s, 1, tm, p),
+                       "conv: kernel launch");
 }
 
 }  // namespace gdr

@@ -38,6 +38,22 @@ void set_last_error(const char *step, cudaError_t e) {
 }
 void clear_last_error() { t_last_error[0] = 0; }
 const char *t_last_error_ptr() { return t_last_error; }
+
+EncodeTiledFn tensor_map_encoder() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (!f) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !ptr)
+      return nullptr;
+    f = reinterpret_cast<EncodeTiledFn>(ptr);
+    fn.store(f, std::memory_order_release);
+  }
+  return f;
+}
+
 }  // namespace gdr
 
 using namespace gdr;

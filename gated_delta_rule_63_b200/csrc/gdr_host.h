@@ -1,6 +1,7 @@
 // gdr_host.h -- host-side argument checks shared by the entry points.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -37,6 +38,14 @@ inline int check_cu_seqlens(const int32_t *cu, int n_seqs) {
     if (cu[i + 1] < cu[i]) return GDR_ERR_CU_SEQLENS;
   return GDR_OK;
 }
+
+// cuTensorMapEncodeTiled, looked up once through the runtime's driver entry
+// points (no link against libcuda); null when the driver does not provide it
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
 
 // Device address of the library's error word on the current device (cached).
 int *device_error_ptr();

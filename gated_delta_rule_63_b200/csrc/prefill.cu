@@ -1145,30 +1145,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 }
 
 // ---- host side ---------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static std::atomic<EncodeTiledFn> fn{nullptr};
-  EncodeTiledFn f = fn.load(std::memory_order_acquire);
-  if (!f) {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !ptr)
-      return nullptr;
-    f = reinterpret_cast<EncodeTiledFn>(ptr);
-    fn.store(f, std::memory_order_release);
-  }
-  return f;
-}
-
 // [rows][cols] bf16 with a row stride in elements; 64 x 64 boxes, 128B swizzle;
 // rows past `rows` read as zero
 bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t row_stride) {
-  EncodeTiledFn f = encode_fn();
+  EncodeTiledFn f = tensor_map_encoder();
   if (!f) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {row_stride * 2};
@@ -1235,7 +1215,7 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   // with no tokens no tile is ever loaded; any aligned device address serves as a base
   const void *any = v ? v : (hT ? static_cast<const void *>(hT) : static_cast<const void *>(h0));
   if (!any) return GDR_OK;
-  if (!encode_fn()) return launch_status(cudaErrorSymbolNotFound, "prefill: cuTensorMapEncodeTiled lookup");
+  if (!tensor_map_encoder()) return launch_status(cudaErrorSymbolNotFound, "prefill: cuTensorMapEncodeTiled lookup");
   if (!make_map(&tq, q ? q : any, static_cast<uint64_t>(hk) * D, rows, static_cast<uint64_t>(qk_stride)) ||
       !make_map(&tk, k ? k : any, static_cast<uint64_t>(hk) * D, rows, static_cast<uint64_t>(qk_stride)) ||
       !make_map(&tv, v ? v : any, static_cast<uint64_t>(hv) * D, rows, static_cast<uint64_t>(v_stride)))

@@ -274,34 +274,55 @@ def bench_decode(torch, G, device, args, steps=1000):
 
 
 def bench_e2e(torch, G, inp, device, args):
-    """Same prefill step through the C ABI from pinned host buffers, copies included."""
+    """Same prefill step through the C ABI from pinned host buffers, copies included.
+
+    Consecutive steps are pipelined the way a server would run them: the host-to-device
+    copies of step i+1 run while step i computes and while its result is copied back (two
+    device buffer sets, one stream for each copy direction and one for the kernels)."""
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()
     hx, ha, hb, hz = pin(inp.x), pin(inp.a), pin(inp.b), pin(inp.z)
-    run = PrefillRunner(torch, G, inp, device)
-    hy = torch.empty(run.y.shape, dtype=torch.bfloat16).pin_memory()
-    hT = torch.empty(run.hT.shape, dtype=torch.float32).pin_memory()
+    runs = [PrefillRunner(torch, G, inp, device) for _ in range(2)]
+    hys = [torch.empty(runs[0].y.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    hTs = [torch.empty(runs[0].hT.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    out_done = [None, None]
 
-    def one():
-        run.x.view(torch.int16).copy_(hx, non_blocking=True)
-        run.a.view(torch.int16).copy_(ha, non_blocking=True)
-        run.b.view(torch.int16).copy_(hb, non_blocking=True)
-        run.z.view(torch.int16).view(-1).copy_(hz.view(-1), non_blocking=True)
-        run.step()
-        hy.copy_(run.y, non_blocking=True)
-        hT.copy_(run.hT, non_blocking=True)
+    def one(i):
+        k = i % 2
+        run = runs[k]
+        with torch.cuda.stream(s_in):
+            if out_done[k] is not None:   # this buffer set's previous step is complete
+                s_in.wait_event(out_done[k])
+            run.x.view(torch.int16).copy_(hx, non_blocking=True)
+            run.a.view(torch.int16).copy_(ha, non_blocking=True)
+            run.b.view(torch.int16).copy_(hb, non_blocking=True)
+            run.z.view(torch.int16).view(-1).copy_(hz.view(-1), non_blocking=True)
+            in_done = torch.cuda.Event()
+            in_done.record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(in_done)
+            run.step()
+            run_done = torch.cuda.Event()
+            run_done.record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(run_done)
+            hys[k].copy_(run.y, non_blocking=True)
+            hTs[k].copy_(run.hT, non_blocking=True)
+            out_done[k] = torch.cuda.Event()
+            out_done[k].record(s_out)
 
-    for _ in range(max(1, args.warmup)):
-        one()
+    for i in range(max(1, args.warmup)):
+        one(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        one()
-    e1.record()
+    e0.record(s_in)
+    for i in range(args.steps):
+        one(i)
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
     h2d = (inp.x.nbytes + inp.a.nbytes + inp.b.nbytes + inp.z.nbytes)
-    d2h = hy.numel() * 2 + hT.numel() * 4
+    d2h = hys[0].numel() * 2 + hTs[0].numel() * 4
     return {"value": inp.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 

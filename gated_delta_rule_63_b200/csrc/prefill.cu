@@ -611,6 +611,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           }
         }
       }
+      fence_proxy_async();   // W_hi is visible to the bulk copy below
       tc_fence_before();
       const bool all_w = named_sync_or(1, 128, !wok) == false;   // W is out of TMEM
       if (tid == 0 && all_w) {
@@ -623,6 +624,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             mma_bf16(tmem, sdesc(sbase + P_OFF_T + (1 + part) * BLK64 + kk * 2048, BLK64, 1024),
                      sdesc(q_half0 + kk * 2048, P_KQ_KB, 1024), id, (part | kk) != 0);
         mma_commit(bar_u);
+        // W_hi goes out while Ut is computed
+        bulk_store(rec + WS_W_HI, sbase + P_OFF_KQ, BLK64);                     // k-block 0
+        bulk_store(rec + WS_W_HI + BLK64, sbase + P_OFF_KQ + P_KQ_KB, BLK64);   // k-block 1
+        bulk_commit();
       }
       bool uok = all_w;
       if (lane == 0 && uok) uok = mbar_wait(bar_u, 0, p.err);
@@ -631,7 +636,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
         for (int i = 0; i < 8; ++i) st_shared16(lo_base + sw128(r, i), lo[i]);
       }
-      good = uok;
+      fence_proxy_async();
+      good = named_sync_or(1, 128, !uok) == false;
+      if (tid == 0 && good) {
+        bulk_store(rec + WS_W_LO, q_half0, BLK64);            // k-block 0
+        bulk_store(rec + WS_W_LO + BLK64, q_half1, BLK64);    // k-block 1
+        bulk_commit();
+      }
     } else {
       // warps 2, 3, 6, 7 (lanes 64..127): Ut rows -> fp32 [slice][row][64] over the T tiles
       const int sl = warp >> 2, r = 32 * (warp & 1) + lane;
@@ -654,24 +665,19 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           }
         }
       }
-      good = uok;
+      fence_proxy_async();
+      good = named_sync_or(2, 128, !uok) == false;
+      if (tid == 64 && good) {
+        bulk_store(rec + WS_UT, sbase + P_OFF_T, 4 * BLK64);
+        bulk_commit();
+      }
     }
   }
   PTIME(0, 9);
-  fence_proxy_async();
+  // the threads that issued stores (0: W, 64: Ut) wait until the shared memory is read
+  if (tid == 0 || tid == 64) bulk_wait_read();
   tc_fence_before();
-  ok = __syncthreads_and(good) != 0;
-  if (tid == 0) {
-    if (ok) {
-      bulk_store(rec + WS_W_HI, sbase + P_OFF_KQ, BLK64);                     // W_hi, k-block 0
-      bulk_store(rec + WS_W_HI + BLK64, sbase + P_OFF_KQ + P_KQ_KB, BLK64);   // W_hi, k-block 1
-      bulk_store(rec + WS_W_LO, q_half0, BLK64);                              // W_lo, k-block 0
-      bulk_store(rec + WS_W_LO + BLK64, q_half1, BLK64);                      // W_lo, k-block 1
-      bulk_store(rec + WS_UT, sbase + P_OFF_T, 4 * BLK64);
-      bulk_commit();
-    }
-    bulk_wait_read();   // the stores have read the shared memory before it goes away
-  }
+  __syncthreads();
   PTIME(0, 10);
   if (warp == 0) tmem_dealloc(tmem, P_TM_COLS);
 }

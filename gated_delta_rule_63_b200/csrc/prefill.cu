@@ -222,11 +222,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   const uint32_t q_half0 = sbase + P_OFF_KQ + P_Q_HALF, q_half1 = q_half0 + P_KQ_KB;
   uint8_t *rec = ws_record(p, n, h, cw);
 
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_holder), P_TM_COLS);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
+  if (tid == 0) {   // the copies go out first
     mbar_init(bar_tma, 1);
     mbar_init(bar_mma, 1);
     mbar_init(bar_v, 1);
@@ -239,16 +235,21 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       tma_load_2d(sbase + P_OFF_KQ + kb * P_KQ_KB + P_Q_HALF, &tm_q, kh * D + kb * 64, t0, bar_tma);
     }
   }
-  // gates of the chunk's rows; padding rows get no decay and no write
-  float g = 0.0f;
-  if (tid < 64) {
-    float beta = 0.0f;
-    if (tid < L) {
-      const size_t ab = static_cast<size_t>(t0 + tid) * p.hv + h;
-      g = -expf(p.A_log[h]) * softplus_f(bf_bits2f(p.a[ab]) + p.dt_bias[h]);
-      beta = sigmoid_f(bf_bits2f(p.b[ab]));
-    }
-    s_beta[tid] = beta;
+  // gate inputs of the chunk's rows (threads 0..63), in flight until the gates are
+  // needed after the norms; padding rows get no decay and no write
+  uint16_t a_raw = 0, b_raw = 0;
+  float a_log = 0.0f, dtb = 0.0f;
+  const bool gate_row = tid < L;
+  if (gate_row) {
+    const size_t ab = static_cast<size_t>(t0 + tid) * p.hv + h;
+    a_raw = __ldg(p.a + ab);
+    b_raw = __ldg(p.b + ab);
+    a_log = __ldg(p.A_log + h);
+    dtb = __ldg(p.dt_bias + h);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_holder), P_TM_COLS);
+    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -294,6 +295,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
     if (part == 0) (row < 64 ? s_rk : s_rq)[row & 63] = 1.0f / sqrtf(ss + 1e-6f);
+    // gates: g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b) (threads 0..63)
+    float g = 0.0f;
+    if (tid < 64) {
+      float beta = 0.0f;
+      if (gate_row) {
+        g = -expf(a_log) * softplus_f(bf_bits2f(a_raw) + dtb);
+        beta = sigmoid_f(bf_bits2f(b_raw));
+      }
+      s_beta[tid] = beta;
+    }
     // inclusive scan of g over the chunk (threads 0..63)
     float run = g;
     if (tid < 64) {

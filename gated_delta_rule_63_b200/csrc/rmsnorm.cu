@@ -19,6 +19,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kRowsPerBlock = kThreads / 16;
 
+template <bool kWeight>   // a norm weight is given (otherwise ones)
 __global__ void __launch_bounds__(kThreads) gated_rmsnorm_kernel(const uint16_t *o, const uint16_t *z,
                                                                  const float *w, float eps,
                                                                  int64_t rows, uint16_t *y) {
@@ -41,19 +42,18 @@ __global__ void __launch_bounds__(kThreads) gated_rmsnorm_kernel(const uint16_t 
   for (int off = 8; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
   const float inv = 1.0f / sqrtf(ss * (1.0f / 128.0f) + eps);
   if (row >= rows) return;
-  float wv[8];
-  if (w) {
+  float sv[8];   // o / rms, times the weight when there is one
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sv[i] = ov[i] * inv;
+  if (kWeight) {
     const float4 w0 = *reinterpret_cast<const float4 *>(w + part * 8);
     const float4 w1 = *reinterpret_cast<const float4 *>(w + part * 8 + 4);
-    wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
-    wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) wv[i] = 1.0f;
+    sv[0] *= w0.x; sv[1] *= w0.y; sv[2] *= w0.z; sv[3] *= w0.w;
+    sv[4] *= w1.x; sv[5] *= w1.y; sv[6] *= w1.z; sv[7] *= w1.w;
   }
   float out[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) out[i] = ov[i] * inv * wv[i] * silu_fast(zv[i]);
+  for (int i = 0; i < 8; ++i) out[i] = sv[i] * silu_fast(zv[i]);
   *reinterpret_cast<uint4 *>(y + row * 128 + part * 8) = pack8x2(out);
 }
 
@@ -63,7 +63,7 @@ int launch_gated_rmsnorm(const void *o, const void *z, const float *w, float eps
                          void *y, cudaStream_t s) {
   const int64_t blocks = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
   if (blocks > 0x7FFFFFFF) return GDR_ERR_SHAPE;
-  return launch_status(launch_pdl(gated_rmsnorm_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, s, 1,
+  return launch_status(launch_pdl(w ? gated_rmsnorm_kernel<true> : gated_rmsnorm_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, s, 1,
                                   static_cast<const uint16_t *>(o), static_cast<const uint16_t *>(z), w, eps,
                                   rows, static_cast<uint16_t *>(y)),
                        "gated norm: kernel launch");

@@ -158,6 +158,31 @@ def test_prefill_lengths_and_varlen(lengths):
     check_core(inp)
 
 
+@pytest.mark.parametrize("window", [1, 3])
+@pytest.mark.parametrize("final_state", [True, False])
+def test_prefill_windows_carry_state(window, final_state):
+    """Sequences longer than the workspace window: the state crosses windows in hT, or in the
+    workspace tail when the caller asks for no final state."""
+    inp = GI.make_core_inputs(80 + window, [300, 64, 1, 190], prenorm_qk=False, h0_std=0.02)
+    hv = inp.v.shape[1]
+    hT = torch.full((inp.n_seqs, hv, 128, 128), float("nan"), device="cuda") if final_state else None
+    ws = G.prefill_workspace(inp.cu_seqlens, hv, "cuda", window=window, has_final_state=final_state)
+    o = G.chunk_prefill(dev_bf16(inp.q), dev_bf16(inp.k), dev_bf16(inp.v), dev_bf16(inp.a),
+                        dev_bf16(inp.b), dev_f32(inp.A_log), dev_f32(inp.dt_bias),
+                        dev_i32(inp.cu_seqlens), inp.cu_seqlens, h0=dev_f32(inp.h0), hT=hT,
+                        scale=inp.scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert G.get_device_error() == 0
+    ref_bits, _, ref_hT = O.core_path(inp)
+    o_bits = host_bits(o)
+    cu = inp.cu_seqlens
+    for n in range(inp.n_seqs):
+        s, e = int(cu[n]), int(cu[n + 1])
+        assert rel_l2(bits_f64(o_bits[s:e]), bits_f64(ref_bits[s:e])) <= TOL_BF16
+    if final_state:
+        assert rel_l2(hT.cpu().numpy(), ref_hT) <= TOL_STATE
+
+
 def test_prefill_scale_and_zero_initial_state():
     inp = GI.make_core_inputs(70, [150, 7], prenorm_qk=True, scale=128 ** -0.5)
     check_core(inp)

@@ -169,6 +169,18 @@ class PrefillRunner:
         G.gated_rmsnorm(self.o, self.z, None, inp.eps, self.y)
 
 
+def max_over_ranks(torch, values, device):
+    """Per-rank timings -> their maximum over the ranks (every rank receives it)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_rate(world, units_per_rank, ms):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def bench_ours(args, rank, world, device):
     import torch
     import gated_delta_rule_63_b200 as G
@@ -215,10 +227,8 @@ def bench_ours(args, rank, world, device):
     ms = sum(step_ms) / len(step_ms)
     pms = sum(pre_ms) / len(pre_ms)
     if world > 1:
-        t = torch.tensor([ms, pms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, pms = float(t[0]), float(t[1])
-    value = world * T / (ms * 1e-3)
+        ms, pms = max_over_ranks(torch, [ms, pms], device)
+    value = job_rate(world, T, ms)
 
     # end to end through the C ABI with host buffers (pinned), copies inside
     e2e = bench_e2e(torch, G, inp, device, args) if args.part == "all" else None

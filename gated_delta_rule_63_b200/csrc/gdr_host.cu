@@ -68,7 +68,7 @@ const char *gdr_status_string(int status) {
     case GDR_ERR_ALIGN: return "GDR_ERR_ALIGN: tensor pointer not 16-byte aligned";
     case GDR_ERR_CU_SEQLENS: return "GDR_ERR_CU_SEQLENS: offsets must start at 0 and not decrease";
     case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED: head dims or grouping not implemented";
-    case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE";
+    case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE: workspace missing or too small for one chunk window";
     case GDR_ERR_CUDA: return "GDR_ERR_CUDA: CUDA launch failed";
     case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a bounded wait in a kernel ran out";
     case GDR_ERR_ALIAS: return "GDR_ERR_ALIAS: buffers overlap";

@@ -28,6 +28,13 @@
  *    16-byte aligned.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
  *    enqueued asynchronously; no call synchronises the device.
+ *  - Kernels are launched with programmatic dependent launch: each may be
+ *    scheduled while the work before it on the stream drains, but waits for
+ *    that work to complete (griddepcontrol.wait) before it reads or writes any
+ *    memory, so stream order is kept.  A caller's kernel that follows on the
+ *    stream and is itself launched with programmatic stream serialization
+ *    must wait the same way (cudaGridDependencySynchronize) before it reads
+ *    this library's outputs; one launched without it is simply ordered.
  *  - The recurrent state is stored transposed, H = S^T, as
  *    [n][hv][dk][dv] fp32 (the dv index is contiguous).
  *  - Supported dims: dk = dv = 128, hk >= 1, hv % hk == 0, hv / hk <= 8.
@@ -57,7 +64,7 @@ typedef enum gdr_status {
   GDR_ERR_ALIGN = 3,       /* a tensor pointer is not 16-byte aligned */
   GDR_ERR_CU_SEQLENS = 4,  /* cu_seqlens does not start at 0 or decreases */
   GDR_ERR_UNSUPPORTED = 5, /* head dims / grouping outside what the kernels implement */
-  GDR_ERR_WORKSPACE = 6,   /* reserved */
+  GDR_ERR_WORKSPACE = 6,   /* the prefill workspace is NULL or too small for one chunk window */
   GDR_ERR_CUDA = 7,        /* the CUDA launch failed (see cudaGetLastError) */
   GDR_ERR_TIMEOUT = 8,     /* (device error word) a bounded wait inside a kernel ran out */
   GDR_ERR_ALIAS = 9        /* two buffers overlap where the call forbids it */

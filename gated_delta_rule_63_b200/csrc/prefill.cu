@@ -482,23 +482,37 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       PTIME(0, 14);
     }
     {
-      const int rt = tid >> 4, jt = tid & 15;
+      // The triangular factors make half of these products zero; each warp takes two
+      // adjacent columns (resp. rows) so that its loops skip the zero k-groups (l-groups)
+      // with warp-uniform bounds.
       {   // X^T[j][r] = sum_{k >= j} A[32 + r][k] T[k][j], r, j < 32, into XF (stride XLD2)
+        const int rt = lane & 15, jt = 2 * warp + (lane >> 4);   // outputs (rt | rt+16, jt | jt+16)
         const float *a0 = AT + (32 + rt) * LD, *a1 = a0 + 16 * LD;
         const float *t0 = AT + jt * LD, *t1 = t0 + 16 * LD;
         float x00 = 0.0f, x01 = 0.0f, x10 = 0.0f, x11 = 0.0f;   // x[r][j], r in {rt, rt+16}, j in {jt, jt+16}
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
+        const int g0 = warp >> 1, g1 = 4 + (warp >> 1);         // first k-groups holding k >= jt, k >= jt + 16
+#pragma unroll 1
+        for (int g = g0; g < 8; ++g) {
           const int k0 = 4 * g;
           const float4 A0 = *reinterpret_cast<const float4 *>(a0 + k0), A1 = *reinterpret_cast<const float4 *>(a1 + k0);
-          const float4 T0 = *reinterpret_cast<const float4 *>(t0 + k0), T1 = *reinterpret_cast<const float4 *>(t1 + k0);
+          const float4 T0 = *reinterpret_cast<const float4 *>(t0 + k0);
           const float av0[4] = {A0.x, A0.y, A0.z, A0.w}, av1[4] = {A1.x, A1.y, A1.z, A1.w};
-          const float tv0[4] = {T0.x, T0.y, T0.z, T0.w}, tv1[4] = {T1.x, T1.y, T1.z, T1.w};
+          const float tv0[4] = {T0.x, T0.y, T0.z, T0.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {   // T is lower triangular: T[k][j] = 0 for k < j
-            const float u0 = (k0 + e >= jt) ? tv0[e] : 0.0f, u1 = (k0 + e >= jt + 16) ? tv1[e] : 0.0f;
-            x00 += av0[e] * u0; x01 += av0[e] * u1;
-            x10 += av1[e] * u0; x11 += av1[e] * u1;
+            const float u0 = (k0 + e >= jt) ? tv0[e] : 0.0f;
+            x00 += av0[e] * u0;
+            x10 += av1[e] * u0;
+          }
+          if (g >= g1) {
+            const float4 T1 = *reinterpret_cast<const float4 *>(t1 + k0);
+            const float tv1[4] = {T1.x, T1.y, T1.z, T1.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float u1 = (k0 + e >= jt + 16) ? tv1[e] : 0.0f;
+              x01 += av0[e] * u1;
+              x11 += av1[e] * u1;
+            }
           }
         }
         float *xt = XF + jt * XLD2;
@@ -509,19 +523,28 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
       __syncthreads();
       {   // T21[r][j] = -sum_{l <= r} T2[r][l] X[l][j], T2[r][l] = AT[(32 + l) LD + 32 + r]; stored as T^T
+        const int rt = 2 * warp + (lane >> 4), jt = lane & 15;   // outputs (rt | rt+16, jt | jt+16)
         const float *xa = XF + jt * XLD2, *xb = xa + 16 * XLD2;
         const float *tb = AT + 32 * LD + 32;
         float y00 = 0.0f, y01 = 0.0f, y10 = 0.0f, y11 = 0.0f;   // y[r][j]
-#pragma unroll
-        for (int l4 = 0; l4 < 8; ++l4) {
+        const int la = warp >> 1, lb = 4 + (warp >> 1);         // last l-groups holding l <= rt, l <= rt + 16
+#pragma unroll 1
+        for (int l4 = 0; l4 <= lb; ++l4) {
           const float4 X0 = *reinterpret_cast<const float4 *>(xa + 4 * l4), X1 = *reinterpret_cast<const float4 *>(xb + 4 * l4);
           const float x0v[4] = {X0.x, X0.y, X0.z, X0.w}, x1v[4] = {X1.x, X1.y, X1.z, X1.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int l = 4 * l4 + e;
-            const float t0v = l <= rt ? tb[l * LD + rt] : 0.0f, t1v = l <= rt + 16 ? tb[l * LD + rt + 16] : 0.0f;
-            y00 -= t0v * x0v[e]; y01 -= t0v * x1v[e];
+            const float t1v = l <= rt + 16 ? tb[l * LD + rt + 16] : 0.0f;
             y10 -= t1v * x0v[e]; y11 -= t1v * x1v[e];
+          }
+          if (l4 <= la) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int l = 4 * l4 + e;
+              const float t0v = l <= rt ? tb[l * LD + rt] : 0.0f;
+              y00 -= t0v * x0v[e]; y01 -= t0v * x1v[e];
+            }
           }
         }
         float *dst = AT + jt * LD + 32;

@@ -1,7 +1,8 @@
 // gdr_common.cuh -- device helpers shared by the gated delta-rule kernels.
 //
 // Plain inline PTX for the sm_100a features the kernels use: mbarriers,
-// tcgen05 (TMEM allocation, MMA, loads, fences), cp.async, and the
+// tcgen05 (TMEM allocation, MMA, loads, fences), TMA and bulk copies, stores
+// into a cluster peer's shared memory, programmatic dependent launch, and the
 // 128-byte swizzle of shared-memory operand tiles.
 #pragma once
 
@@ -24,7 +25,6 @@ __device__ __forceinline__ void raise_device_error(int *err, int code) {
 // ---------------------------------------------------------------------------
 // small numerics
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ float bf_bits2f(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
@@ -54,32 +54,6 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
   }
 }
 
-__device__ __forceinline__ uint32_t pack2bf(float lo, float hi) {
-  return static_cast<uint32_t>(f2bf_bits(lo)) | (static_cast<uint32_t>(f2bf_bits(hi)) << 16);
-}
-
-__device__ __forceinline__ uint4 pack8(const float *f) {
-  uint4 u;
-  u.x = pack2bf(f[0], f[1]);
-  u.y = pack2bf(f[2], f[3]);
-  u.z = pack2bf(f[4], f[5]);
-  u.w = pack2bf(f[6], f[7]);
-  return u;
-}
-
-// Split fp32 values into a bf16 pair hi + lo with hi = bf16(x), lo = bf16(x - hi).
-// hi + lo carries about 16 significant bits of x.
-__device__ __forceinline__ void split8(const float *f, uint4 &hi, uint4 &lo) {
-  float h[8], l[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    h[i] = round_bf16(f[i]);
-    l[i] = f[i] - h[i];
-  }
-  hi = pack8(h);
-  lo = pack8(l);
-}
-
 // ---------------------------------------------------------------------------
 // shared memory addressing
 // ---------------------------------------------------------------------------
@@ -93,17 +67,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) {
   return r * 128u + ((c ^ (r & 7u)) << 4);
 }
-
-// ---------------------------------------------------------------------------
-// cp.async (16 bytes, zero-filled when src_bytes == 0)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
 // make generic-proxy shared memory writes visible to the async proxy (tensor core)
 __device__ __forceinline__ void fence_proxy_async() {
@@ -379,7 +342,6 @@ __device__ __forceinline__ void bulk_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
 }
 // this thread's bulk stores are complete
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
 }  // namespace gdr
 

@@ -183,6 +183,25 @@ def test_prefill_windows_carry_state(window, final_state):
         assert rel_l2(hT.cpu().numpy(), ref_hT) <= TOL_STATE
 
 
+@pytest.mark.parametrize("case", ["no_decay", "instant_decay", "no_write", "full_write"])
+def test_prefill_degenerate_gates(case):
+    """Limits of the gates on the GPU path: g = 0 (exp(A_log) = 0), g far below zero (the
+    state is forgotten at every token), beta = 0 (nothing is written, the state only decays)
+    and beta = 1 (every token overwrites)."""
+    inp = GI.make_core_inputs(90, [130, 64], prenorm_qk=False, h0_std=0.02)
+    hv = inp.v.shape[1]
+    if case == "no_decay":
+        inp.A_log = np.full(hv, -1e30, np.float32)
+    elif case == "instant_decay":   # g = -16 softplus(20 + dt_bias), about -320 per token
+        inp.A_log = np.full(hv, np.log(16.0), np.float32)
+        inp.a = GI.f32_to_bf16_bits(np.full(inp.a.shape, 20.0, np.float32))
+    elif case == "no_write":
+        inp.b = GI.f32_to_bf16_bits(np.full(inp.b.shape, -200.0, np.float32))
+    else:
+        inp.b = GI.f32_to_bf16_bits(np.full(inp.b.shape, 200.0, np.float32))
+    check_core(inp)
+
+
 def test_prefill_scale_and_zero_initial_state():
     inp = GI.make_core_inputs(70, [150, 7], prenorm_qk=True, scale=128 ** -0.5)
     check_core(inp)

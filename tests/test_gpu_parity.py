@@ -138,6 +138,27 @@ def test_decode_small_batch_several_steps():
     assert np.array_equal(cs, O.round_bf16(ref_cs))
 
 
+@pytest.mark.parametrize("case", ["no_decay", "instant_decay", "no_write", "full_write"])
+def test_decode_degenerate_gates(case):
+    """The decode step at the gates' limits (as the prefill test of the same name)."""
+    dec = GI.make_decode_inputs(54, 2, 3)
+    if case == "no_decay":
+        dec.A_log = np.full(dec.hv, -1e30, np.float32)
+    elif case == "instant_decay":
+        dec.A_log = np.full(dec.hv, np.log(16.0), np.float32)
+        dec.a = GI.f32_to_bf16_bits(np.full(dec.a.shape, 20.0, np.float32))
+    elif case == "no_write":
+        dec.b = GI.f32_to_bf16_bits(np.full(dec.b.shape, -200.0, np.float32))
+    else:
+        dec.b = GI.f32_to_bf16_bits(np.full(dec.b.shape, 200.0, np.float32))
+    outs, st, cs = run_gpu_decode(dec, 3, keep=range(3))
+    kept, H, ref_cs = O.decode_steps(dec, keep_o=tuple(range(3)))
+    for s in range(3):
+        assert rel_l2(bits_f64(outs[s]), bits_f64(kept[s])) <= TOL_BF16, s
+    assert rel_l2(st, H) <= TOL_STATE
+    assert np.array_equal(cs, O.round_bf16(ref_cs))
+
+
 def test_decode_full_batch_sampled_heads():
     dec = GI.make_decode_inputs(53, 64, 3)
     heads = [0, 1, 2, 25, 47]

@@ -49,9 +49,9 @@ B_FUSED = CX * 2 + 2 * GI.HV * 2 + 2 * GI.HV * GI.DV * 2 # x, a, b, z read + y w
 STATE_BYTES = GI.HV * GI.DK * GI.DV * 4                  # one sequence's fp32 state
 
 # DRAM bytes (read + written) per launch from one ncu capture of the current kernels:
-# prefill = prep + state chain on full_T4096 (281.0 + 327.3 MB), decode = one B=64 step
+# prefill = prep + state chain on full_T4096 (283.5 + 327.3 MB), decode = one B=64 step
 # (a replayed launch, partly served from L2)
-TRAFFIC_PREFILL = 608_322_816
+TRAFFIC_PREFILL = 610_779_392
 TRAFFIC_DECODE = 355_618_304
 
 

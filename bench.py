@@ -346,6 +346,117 @@ def bench_e2e(torch, G, inp, device, args):
 
 
 # ---------------------------------------------------------------------------
+# --sweep: the same kernels over other sizes (one JSON line each); inputs drawn
+# on the device with torch's generator from the workload distributions
+# ---------------------------------------------------------------------------
+def _dev_inputs(torch, device, seed, T, n_seqs, full):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    hk, hv, d = GI.HK, GI.HV, GI.DK
+    rn = lambda *shape: torch.randn(shape, device=device, generator=g)
+    out = {}
+    if full:
+        out["x"] = rn(T, CX).to(torch.bfloat16)
+        out["w"] = (rn(CX, 4) * 0.5).to(torch.bfloat16)
+        out["z"] = rn(T, hv, d).to(torch.bfloat16)
+    else:
+        unit = lambda x: (x / x.norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+        out["q"], out["k"] = unit(rn(T, hk, d)), unit(rn(T, hk, d))
+        out["v"] = rn(T, hv, d).to(torch.bfloat16)
+    out["a"], out["b"] = rn(T, hv).to(torch.bfloat16), rn(T, hv).to(torch.bfloat16)
+    A = torch.empty(hv, device=device, dtype=torch.float64).uniform_(1.0, 16.0, generator=g)
+    dt = torch.empty(hv, device=device, dtype=torch.float64).uniform_(1e-3, 0.1, generator=g)
+    out["A_log"], out["dt_bias"] = torch.log(A).float(), torch.log(torch.expm1(dt)).float()
+    out["h0"] = (rn(n_seqs, hv, d, d) * 0.02) if full else None
+    return out
+
+
+def _time_ms(torch, fn, flush, reps=5):
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for i in range(reps):
+        flush.fill_(float(i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts)
+
+
+def bench_sweep(torch, G, device):
+    hbm_peak, _, _ = measured_peaks()
+    hk, hv, d = GI.HK, GI.HV, GI.DK
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    lines = []
+    # recurrence alone, one sequence (config 3 is T = 262144)
+    for T in (1024, 4096, 16384, 65536, 262144):
+        x = _dev_inputs(torch, device, 3, T, 1, full=False)
+        cu_host = np.array([0, T], dtype=np.int32)
+        cu = torch.from_numpy(cu_host).to(device)
+        o = torch.empty((T, hv, d), dtype=torch.bfloat16, device=device)
+        hT = torch.empty((1, hv, d, d), dtype=torch.float32, device=device)
+        ws = G.prefill_workspace(cu_host, hv, device)
+        run = lambda: G.chunk_prefill(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"], cu,
+                                      cu_host, hT=hT, o=o, workspace=ws)
+        ms = _time_ms(torch, run, flush)
+        byts = T * B_CORE + STATE_BYTES
+        lines.append({"sweep": "prefill recurrence, B=1", "T": T, "tokens_per_s": T / (ms * 1e-3), "ms": ms,
+                      "hbm_frac": byts / (ms * 1e-3) / 1e9 / hbm_peak})
+        del x, o, hT, ws
+    # full path over 8 packed sequences with an initial state (config 4)
+    lengths = GI.varlen8_lengths(4)
+    cu_host = GI.cu_seqlens_from_lengths(lengths)
+    T, N = int(cu_host[-1]), len(lengths)
+    x = _dev_inputs(torch, device, 4, T, N, full=True)
+    cu = torch.from_numpy(cu_host).to(device)
+    conv_y = torch.empty((T, CX), dtype=torch.bfloat16, device=device)
+    o = torch.empty((T, hv, d), dtype=torch.bfloat16, device=device)
+    y = torch.empty((T, hv, d), dtype=torch.bfloat16, device=device)
+    hT = torch.empty((N, hv, d, d), dtype=torch.float32, device=device)
+    ws = G.prefill_workspace(cu_host, hv, device)
+
+    def full_step():
+        G.causal_conv(x["x"], x["w"], cu, cu_host, None, None, conv_y)
+        q = conv_y[:, : hk * d].view(T, hk, d)
+        k = conv_y[:, hk * d: 2 * hk * d].view(T, hk, d)
+        v = conv_y[:, 2 * hk * d:].view(T, hv, d)
+        G.chunk_prefill(q, k, v, x["a"], x["b"], x["A_log"], x["dt_bias"], cu, cu_host, h0=x["h0"], hT=hT, o=o,
+                        workspace=ws)
+        G.gated_rmsnorm(o, x["z"], None, 1e-6, y)
+    ms = _time_ms(torch, full_step, flush)
+    byts = T * B_FUSED + 2 * N * STATE_BYTES
+    lines.append({"sweep": "full path, 8 packed sequences U{1024..32768}, h0", "T": T,
+                  "lengths": [int(v) for v in lengths], "tokens_per_s": T / (ms * 1e-3), "ms": ms,
+                  "frac_of_fused_hbm_roofline": byts / (ms * 1e-3) / 1e9 / hbm_peak})
+    del x, conv_y, o, y, hT, ws
+    # decode over batch sizes
+    for B in (1, 8, 64, 256):
+        dec = GI.make_decode_inputs(2, B, 1)
+        xs, as_, bs = to_dev(torch, dec.x, device)[0], to_dev(torch, dec.a, device)[0], to_dev(torch, dec.b, device)[0]
+        cw, cs = to_dev(torch, dec.conv_w, device), to_dev(torch, dec.conv_state, device)
+        st = torch.from_numpy(dec.state).to(device)
+        Al, db = torch.from_numpy(dec.A_log).to(device), torch.from_numpy(dec.dt_bias).to(device)
+        od = torch.empty((B, hv, d), dtype=torch.bfloat16, device=device)
+        step = lambda: G.decode_step(xs, cw, cs, as_, bs, Al, db, st, od)
+        for _ in range(5):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(200):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 200
+        lines.append({"sweep": "decode", "B": B, "steps_per_s": 1e3 / ms, "ms": ms,
+                      "hbm_frac": B * STATE_BYTES * 2 / (ms * 1e-3) / 1e9 / hbm_peak})
+    return lines
+
+
+# ---------------------------------------------------------------------------
 # CPU baseline: the fp64 oracle as it stands, on the host cores
 # ---------------------------------------------------------------------------
 def oracle_step(O, inp):
@@ -399,6 +510,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--part", choices=["all", "prefill", "decode"], default="all")
     ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the bench line: the kernels over other sizes, one JSON line each")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -417,6 +530,14 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local)
+    if args.sweep:
+        torch.cuda.set_device(device)
+        import gated_delta_rule_63_b200 as G
+        G.lib()
+        for line in bench_sweep(torch, G, device):
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+        return
     if args.part == "decode":
         torch.cuda.set_device(device)
         import gated_delta_rule_63_b200 as G

@@ -16,7 +16,7 @@ import numpy as np
 
 __all__ = [
     "GdrError", "lib", "status_string", "prepare_chunks", "causal_conv", "chunk_prefill",
-    "chunk_prefill_noalloc", "prefill_workspace", "prefill_window",
+    "chunk_prefill_noalloc", "prefill_workspace", "prefill_fused_workspace", "prefill_window",
     "decode_step", "gated_rmsnorm", "get_device_error", "HEAD_DIM", "CHUNK",
 ]
 
@@ -72,6 +72,8 @@ def lib(path: Optional[str] = None):
     L.gdr_chunk_prefill_noalloc.restype = ctypes.c_int
     L.gdr_chunk_prefill_noalloc_scratch_bytes.restype = ctypes.c_size_t
     L.gdr_chunk_prefill_noalloc_scratch_bytes.argtypes = []
+    L.gdr_chunk_prefill_fused_workspace_size.restype = ctypes.c_size_t
+    L.gdr_chunk_prefill_fused_workspace_size.argtypes = [ctypes.c_int] * 6
     L.gdr_chunk_prefill_workspace_size.restype = ctypes.c_size_t
     L.gdr_chunk_prefill_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int]
@@ -204,12 +206,27 @@ def prefill_workspace(cu_seqlens_host, hv: int, device, window: Optional[int] = 
     return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
 
 
+def prefill_fused_workspace(cu_seqlens_host, hk: int, hv: int, device, window: Optional[int] = None,
+                            has_final_state: bool = True):
+    """Workspace for gdr_chunk_prefill with the conv fused: the conv output, then the records."""
+    torch = _torch()
+    cu = np.asarray(cu_seqlens_host)
+    n = len(cu) - 1
+    T = int(cu[-1]) if n > 0 else 0
+    if window is None:
+        window = prefill_window(cu_seqlens_host, hv, has_final_state=has_final_state)
+    nbytes = lib().gdr_chunk_prefill_fused_workspace_size(max(n, 1), int(hk), int(hv), T, max(int(window), 1),
+                                                          int(has_final_state))
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
 def chunk_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_host, h0=None, hT=None,
                   o=None, scale: float = 1.0, fuse: Optional[dict] = None, workspace=None,
                   window: Optional[int] = None, stream=None):
     """Chunk-64 prefill.  q, k [T, hk, 128], v [T, hv, 128], a, b [T, hv] bf16.
 
-    q, k, v may be token-strided views (e.g. slices of the [T, q|k|v] conv output).
+    q, k, v may be token-strided views (e.g. slices of the [T, q|k|v] conv output); with the
+    conv fused (``fuse`` holding "x", "conv_w" and "hk") they are None.
 
     Returns o [T, hv, 128] bf16 (and writes hT [N, hv, 128, 128] fp32 when given).
     ``fuse`` (optional) maps gdr_prefill_fuse_t field names to tensors.
@@ -232,7 +249,10 @@ def chunk_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_host, h0
         T = a.shape[0]
         o = torch.empty((T, hv, HEAD_DIM), dtype=bf, device=a.device)
     if workspace is None:
-        workspace = prefill_workspace(cu_seqlens_host, hv, a.device, window, hT is not None)
+        if fuse is not None and fuse.get("x") is not None:
+            workspace = prefill_fused_workspace(cu_seqlens_host, hk, hv, a.device, window, hT is not None)
+        else:
+            workspace = prefill_workspace(cu_seqlens_host, hv, a.device, window, hT is not None)
     _check("gdr_chunk_prefill", lib().gdr_chunk_prefill(
         _ptr(q, bf, "q", rows=True), _ptr(k, bf, "k", rows=True), _ptr(v, bf, "v", rows=True),
         _tok_stride(q), _tok_stride(v), _ptr(a, bf, "a"), _ptr(b, bf, "b"),

@@ -76,7 +76,7 @@ const char *gdr_status_string(int status) {
   }
 }
 
-int gdr_abi_version(void) { return 1; }
+int gdr_abi_version(void) { return 2; }
 
 const char *gdr_last_error_string(void) { return gdr::t_last_error_ptr(); }
 
@@ -180,6 +180,13 @@ size_t gdr_chunk_prefill_workspace_size(int n_seqs, int hv, int window_chunks, i
   return chunk_prefill_workspace_bytes(n_seqs, hv, window_chunks, has_final_state == 0);
 }
 
+size_t gdr_chunk_prefill_fused_workspace_size(int n_seqs, int hk, int hv, int total_tokens, int window_chunks,
+                                              int has_final_state) {
+  if (n_seqs <= 0 || hk <= 0 || hv <= 0 || total_tokens < 0 || window_chunks <= 0) return 0;
+  return fused_conv_bytes(total_tokens, (2 * hk + hv) * kHeadDim) +
+         chunk_prefill_workspace_bytes(n_seqs, hv, window_chunks, has_final_state == 0);
+}
+
 int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_stride,
                       int64_t v_stride, const void *a, const void *b, const float *A_log,
                       const float *dt_bias, float scale, int hk, int hv, const int32_t *cu_dev,
@@ -189,6 +196,13 @@ int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_st
   clear_last_error();
   int st = check_heads(hk, hv);
   if (st) return st;
+  const bool fused_conv = fuse && fuse->x;
+  const bool fused_norm = fuse && fuse->z;
+  const int channels = (2 * hk + hv) * kHeadDim;
+  if (fused_conv) {   // q, k, v are the conv output the call makes: rows of [q | k | v]
+    if (q || k || v) return GDR_ERR_SHAPE;
+    qk_stride = v_stride = channels;
+  }
   if (qk_stride == 0) qk_stride = static_cast<int64_t>(hk) * kHeadDim;
   if (v_stride == 0) v_stride = static_cast<int64_t>(hv) * kHeadDim;
   if (qk_stride < static_cast<int64_t>(hk) * kHeadDim || v_stride < static_cast<int64_t>(hv) * kHeadDim)
@@ -199,15 +213,14 @@ int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_st
   if (st) return st;
   if (n_seqs == 0) return GDR_OK;
   const int total = cu_host[n_seqs];
-  if (total == 0 && !hT) return GDR_OK;   // nothing to compute, nothing to write
+  const bool conv_state_out = fused_conv && fuse->conv_state_out;   // passes through empty sequences too
+  if (total == 0 && !hT && !conv_state_out) return GDR_OK;   // nothing to compute, nothing to write
   if (!cu_dev) return GDR_ERR_NULL;
-  const bool fused_conv = fuse && fuse->x;
-  const bool fused_norm = fuse && fuse->z;
-  if (fused_conv) return GDR_ERR_UNSUPPORTED;   // the conv runs as its own kernel (gdr_causal_conv)
   if (fuse && !fuse->z && fuse->y) return GDR_ERR_NULL;   // y without the gate z
+  if (fused_conv && !fuse->conv_w) return GDR_ERR_NULL;
   if (total > 0) {
     if (!a || !b || !A_log || !dt_bias) return GDR_ERR_NULL;
-    if (!q || !k || !v) return GDR_ERR_NULL;
+    if (!fused_conv && (!q || !k || !v)) return GDR_ERR_NULL;
     if (!o && !fused_norm) return GDR_ERR_NULL;
     if (fused_norm && !fuse->y) return GDR_ERR_NULL;
   }
@@ -218,6 +231,9 @@ int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_st
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(h0) ||
       !aligned16(hT) || !aligned16(workspace) || !aligned16(z) || !aligned16(y) || !aligned16(norm_w))
     return GDR_ERR_ALIGN;
+  if (fused_conv && (!aligned16(fuse->x) || !aligned16(fuse->conv_w) || !aligned16(fuse->conv_state_in) ||
+                     !aligned16(fuse->conv_state_out)))
+    return GDR_ERR_ALIGN;
   int max_chunks = 0;
   for (int i = 0; i < n_seqs; ++i) {
     const int nc = (cu_host[i + 1] - cu_host[i] + kChunk - 1) / kChunk;
@@ -225,12 +241,33 @@ int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_st
   }
   const size_t state_bytes = static_cast<size_t>(n_seqs) * hv * kHeadDim * kHeadDim * 4;
   if (h0 != hT && overlaps(h0, state_bytes, hT, state_bytes)) return GDR_ERR_ALIAS;
-  if (max_chunks > 0 &&
-      (!workspace || workspace_bytes < chunk_prefill_workspace_bytes(n_seqs, hv, 1, hT == nullptr)))
+  // with the conv fused its output comes first in the workspace, then the chunk records
+  const size_t conv_bytes = fused_conv ? fused_conv_bytes(total, channels) : 0;
+  const size_t rec_bytes = max_chunks > 0 ? chunk_prefill_workspace_bytes(n_seqs, hv, 1, hT == nullptr) : 0;
+  if ((conv_bytes | rec_bytes) != 0 && (!workspace || workspace_bytes < conv_bytes + rec_bytes))
     return GDR_ERR_WORKSPACE;
+  if (fused_conv) {
+    const size_t cs_bytes = static_cast<size_t>(n_seqs) * 3 * channels * 2;
+    const size_t x_bytes = static_cast<size_t>(total) * channels * 2;
+    if (overlaps(fuse->conv_state_in, cs_bytes, fuse->conv_state_out, cs_bytes) ||
+        overlaps(fuse->x, x_bytes, workspace, conv_bytes))
+      return GDR_ERR_ALIAS;
+  }
   if (fused_norm && o) {   // o and y are separate outputs
     const size_t out_bytes = static_cast<size_t>(total) * hv * kHeadDim * 2;
     if (overlaps(o, out_bytes, y, out_bytes)) return GDR_ERR_ALIAS;
+  }
+  if (fused_conv) {
+    uint8_t *conv_out = static_cast<uint8_t *>(workspace);
+    st = launch_causal_conv(fuse->x, fuse->conv_w, fuse->conv_state_in, fuse->conv_state_out, cu_dev, n_seqs,
+                            total, channels, conv_out, static_cast<cudaStream_t>(stream));
+    if (st) return st;
+    if (total == 0 && !hT) return GDR_OK;
+    q = conv_out;
+    k = conv_out + static_cast<size_t>(hk) * kHeadDim * 2;
+    v = conv_out + static_cast<size_t>(2 * hk) * kHeadDim * 2;
+    workspace = conv_out + conv_bytes;
+    workspace_bytes -= conv_bytes;
   }
   return launch_chunk_prefill(q, k, v, qk_stride, v_stride, a, b, A_log, dt_bias, scale, hk, hv,
                               cu_dev, cu_host, n_seqs, total, max_chunks, h0, hT, o, z, norm_w, eps, y, workspace,

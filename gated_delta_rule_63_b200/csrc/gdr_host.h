@@ -82,4 +82,11 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
                          float eps, void *y, void *workspace, size_t ws_bytes, cudaStream_t s);
 size_t chunk_prefill_workspace_bytes(int n_seqs, int hv, int window_chunks, bool need_carry);
 
+// Conv output of `total` tokens of `channels` bf16 kept in the workspace when the conv is
+// fused into the prefill (a whole number of KiB, so the records after it stay aligned).
+inline size_t fused_conv_bytes(int total, int channels) {
+  const size_t b = static_cast<size_t>(total) * channels * 2;
+  return (b + 1023) & ~static_cast<size_t>(1023);
+}
+
 }  // namespace gdr

@@ -73,7 +73,9 @@ typedef enum gdr_status {
 /* Human-readable name of a status code.  Never NULL. */
 GDR_API const char *gdr_status_string(int status);
 
-/* ABI version of this header; bumped on any signature change. */
+/* ABI version of this header, bumped whenever a signature or what a call does
+ * changes (2: the conv fused into gdr_chunk_prefill,
+ * gdr_chunk_prefill_fused_workspace_size). */
 GDR_API int gdr_abi_version(void);
 
 /*
@@ -122,9 +124,14 @@ GDR_API int gdr_causal_conv(const void *x, const void *w, const void *conv_state
  *    64-column halves of a head run as a thread-block cluster and exchange their
  *    row sums of squares); o is written as well only when gdr_chunk_prefill's o
  *    is not NULL.  y must not overlap o (GDR_ERR_ALIAS).
- *  - Conv (`x` set): not fused in this version; the call returns
- *    GDR_ERR_UNSUPPORTED.  Run gdr_causal_conv and pass its output's q, k, v
- *    column ranges as strided views.
+ *  - Conv (`x` set): the call runs the causal conv of gdr_causal_conv on x
+ *    (with conv_w and the optional conv states) into the head of the
+ *    workspace and reads q, k, v from that output; q, k and v must then be
+ *    NULL (GDR_ERR_SHAPE otherwise) and the workspace must hold
+ *    gdr_chunk_prefill_fused_workspace_size(...) bytes.  conv_state_out
+ *    receives the last three inputs of every sequence (empty ones included),
+ *    as from gdr_causal_conv.  The results equal the separate calls bit for
+ *    bit: the same kernels run, one after the other on the stream.
  */
 typedef struct gdr_prefill_fuse {
   const void *x;             /* bf16 [T][hk*128*2 + hv*128] conv input, or NULL */
@@ -145,7 +152,8 @@ typedef struct gdr_prefill_fuse {
  * dense products run on the tcgen05 tensor cores and the state carried from
  * chunk to chunk stays fp32.
  *   q, k:     bf16 [T][hk][128] rows, consecutive tokens qk_token_stride
- *             elements apart (0 = dense, hk*128)
+ *             elements apart (0 = dense, hk*128); NULL (with v) when the conv
+ *             is fused (fuse->x), the strides are then ignored
  *   v:        bf16 [T][hv][128] rows, consecutive tokens v_token_stride
  *             elements apart (0 = dense, hv*128).  The strides let q, k, v be
  *             read in place from the [T][q | k | v] conv output (stride
@@ -186,6 +194,16 @@ GDR_API int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64
  */
 GDR_API size_t gdr_chunk_prefill_workspace_size(int n_seqs, int hv, int window_chunks,
                                                 int has_final_state);
+
+/*
+ * Bytes of device workspace gdr_chunk_prefill needs with the conv fused
+ * (gdr_prefill_fuse_t.x set): the conv output of the total_tokens tokens,
+ * [total_tokens][hk*128*2 + hv*128] bf16 rounded up to a whole KiB, followed by
+ * gdr_chunk_prefill_workspace_size(n_seqs, hv, window_chunks, has_final_state).
+ * Returns 0 for invalid sizes.
+ */
+GDR_API size_t gdr_chunk_prefill_fused_workspace_size(int n_seqs, int hk, int hv, int total_tokens,
+                                                      int window_chunks, int has_final_state);
 
 /*
  * gdr_chunk_prefill_noalloc -- gdr_chunk_prefill without a caller workspace.

@@ -43,7 +43,7 @@ def test_status_strings(L):
     for code in range(1, 10):
         assert G.status_string(code).startswith("GDR_ERR_")
     assert "UNKNOWN" in G.status_string(12345)
-    assert L.gdr_abi_version() == 1
+    assert L.gdr_abi_version() == 2
 
 
 @pytest.mark.parametrize("lengths", [[0], [1], [64], [65, 0, 128, 1, 63], [5000, 3, 64 * 7 + 1],
@@ -118,6 +118,38 @@ def test_prefill_workspace_size(L):
     assert L.gdr_chunk_prefill_workspace_size(2, 48, 5, 1) == 5 * one
     assert L.gdr_chunk_prefill_workspace_size(2, 48, 5, 0) == 5 * one + 2 * 48 * 128 * 128 * 4
     assert L.gdr_chunk_prefill_workspace_size(0, 48, 5, 1) == 0
+
+
+def test_prefill_with_fused_conv_checks_on_host(L):
+    """Conv fused into the prefill (fuse.x): q, k, v must be NULL, conv_w is required, and the
+    workspace holds the conv output in front of the chunk records."""
+    cu, cup = _cu([10, 5])
+    fz = G.FuseArgs()
+    fz.x, fz.conv_w = FAKE, FAKE
+
+    def call(q=None, wsb=1 << 30, fuse=fz):
+        return L.gdr_chunk_prefill(q, None, None, 0, 0, FAKE, FAKE, FAKE, FAKE, 1.0, 16, 48, FAKE, cup, 2,
+                                   None, FAKE, FAKE, ctypes.byref(fuse), FAKE, wsb, None)
+    assert call(q=FAKE) == 2                   # q, k, v come from the conv
+    no_w = G.FuseArgs()
+    no_w.x = FAKE
+    assert call(fuse=no_w) == 1                # conv weights required
+    need = L.gdr_chunk_prefill_fused_workspace_size(2, 16, 48, 15, 1, 1)
+    assert call(wsb=need - 16) == 6            # the conv output does not fit in front of the records
+    odd = G.FuseArgs()
+    odd.x, odd.conv_w, odd.conv_state_in = FAKE, FAKE, ODD
+    assert call(fuse=odd) == 3
+
+
+def test_fused_workspace_size(L):
+    conv = 100 * 10240 * 2                      # already a whole number of KiB
+    assert L.gdr_chunk_prefill_fused_workspace_size(2, 16, 48, 100, 1, 1) == conv + 2 * 48 * 82944
+    # one key and one value head: 3 tokens x 384 channels x 2 B = 2304 B, rounded up to 3 KiB
+    assert L.gdr_chunk_prefill_fused_workspace_size(2, 1, 1, 3, 1, 1) == 3072 + 2 * 82944
+    assert L.gdr_chunk_prefill_fused_workspace_size(2, 16, 48, 100, 2, 0) == (
+        conv + L.gdr_chunk_prefill_workspace_size(2, 48, 2, 0))
+    assert L.gdr_chunk_prefill_fused_workspace_size(0, 16, 48, 100, 1, 1) == 0
+    assert L.gdr_chunk_prefill_fused_workspace_size(2, 16, 48, -1, 1, 1) == 0
 
 
 def test_other_entry_points_reject_bad_arguments(L):

@@ -314,6 +314,59 @@ def test_fused_gated_norm_varlen_matches_unfused_and_oracle():
             assert rel_l2(bits_f64(y_f[s:e]), bits_f64(ref["y"][s:e])) <= TOL_BF16
 
 
+def run_fused_conv_gpu(inp, fused_norm):
+    """One gdr_chunk_prefill call that runs the conv too (fuse.x), optionally the norm."""
+    cu_d = dev_i32(inp.cu_seqlens)
+    T, hv = inp.T, inp.hv
+    hT = torch.full((inp.n_seqs, hv, 128, 128), float("nan"), device="cuda")
+    cs_out = torch.full(inp.conv_state.shape if inp.conv_state is not None else (inp.n_seqs, 3, inp.x.shape[1]),
+                        float("nan"), dtype=torch.bfloat16, device="cuda")
+    fuse = {"x": dev_bf16(inp.x), "conv_w": dev_bf16(inp.conv_w), "hk": inp.hk, "conv_state_out": cs_out}
+    if inp.conv_state is not None:
+        fuse["conv_state_in"] = dev_bf16(inp.conv_state)
+    y = None
+    if fused_norm:
+        y = torch.empty((T, hv, 128), dtype=torch.bfloat16, device="cuda")
+        fuse.update({"z": dev_bf16(inp.z).reshape(T, hv, 128), "eps": inp.eps, "y": y, "keep_o": True,
+                     "norm_w": dev_f32(inp.norm_w) if inp.norm_w is not None else None})
+    h0 = dev_f32(inp.h0) if inp.h0 is not None else None
+    o = G.chunk_prefill(None, None, None, dev_bf16(inp.a), dev_bf16(inp.b), dev_f32(inp.A_log),
+                        dev_f32(inp.dt_bias), cu_d, inp.cu_seqlens, h0=h0, hT=hT, scale=inp.scale, fuse=fuse)
+    torch.cuda.synchronize()
+    assert G.get_device_error() == 0
+    return host_bits(o), (host_bits(y) if y is not None else None), hT.cpu().numpy(), host_bits(cs_out)
+
+
+@pytest.mark.parametrize("fused_norm", [False, True])
+def test_fused_conv_equals_separate_calls(fused_norm):
+    """The conv fused into the prefill call gives the separate calls' results bit for bit,
+    conv state included, on packed sequences with empty ones, conv and recurrent states."""
+    inp = GI.make_full_inputs(81, [200, 65, 1, 0, 130], h0_std=0.02, conv_state_std=1.0, norm_w_std=0.1)
+    o_f, y_f, h_f, cs_f = run_fused_conv_gpu(inp, fused_norm)
+    # the same three kernels called one by one
+    cu_d = dev_i32(inp.cu_seqlens)
+    T, hk, hv = inp.T, inp.hk, inp.hv
+    cs_sep = torch.empty(inp.conv_state.shape, dtype=torch.bfloat16, device="cuda")
+    yc = G.causal_conv(dev_bf16(inp.x), dev_bf16(inp.conv_w), cu_d, inp.cu_seqlens,
+                       dev_bf16(inp.conv_state), cs_sep)
+    q = yc[:, : hk * 128].view(T, hk, 128)
+    k = yc[:, hk * 128: 2 * hk * 128].view(T, hk, 128)
+    v = yc[:, 2 * hk * 128:].view(T, hv, 128)
+    hT = torch.empty((inp.n_seqs, hv, 128, 128), device="cuda")
+    o = G.chunk_prefill(q, k, v, dev_bf16(inp.a), dev_bf16(inp.b), dev_f32(inp.A_log), dev_f32(inp.dt_bias),
+                        cu_d, inp.cu_seqlens, h0=dev_f32(inp.h0), hT=hT, scale=inp.scale)
+    torch.cuda.synchronize()
+    assert np.array_equal(o_f, host_bits(o))
+    assert np.array_equal(h_f, hT.cpu().numpy())
+    assert np.array_equal(cs_f, host_bits(cs_sep))
+    ref = O.full_path(inp)
+    assert np.array_equal(cs_f, ref["conv_state_out"])
+    assert rel_l2(bits_f64(o_f), bits_f64(ref["o"])) <= TOL_BF16
+    assert rel_l2(h_f, ref["hT"]) <= TOL_STATE
+    if fused_norm:
+        assert rel_l2(bits_f64(y_f), bits_f64(ref["y"])) <= TOL_BF16
+
+
 def test_full_path_T4096_fused_norm():
     """The bench workload with the gated norm fused, against the oracle."""
     inp = GI.workload_full_T4096()

@@ -37,6 +37,10 @@ MUTANTS = [
     ("conv taps reversed", "acc += w[(size_t)c * 4 + j] * xv;", "acc += w[(size_t)c * 4 + (3 - j)] * xv;"),
     ("conv state read newest first", "conv_state[((size_t)n * 3 + (3 - back)) * C + c]",
      "conv_state[((size_t)n * 3 + (back - 1)) * C + c]"),
+    ("conv step: state rolled the wrong way", "s[c] = s1; s[C + c] = s2; s[2 * C + c] = xv;",
+     "s[c] = xv; s[C + c] = s1; s[2 * C + c] = s2;"),
+    ("conv step: current token on the oldest tap", "wc[0] * s0 + wc[1] * s1 + wc[2] * s2 + wc[3] * xv",
+     "wc[3] * s0 + wc[1] * s1 + wc[2] * s2 + wc[0] * xv"),
     ("norm mean over d dropped", "double inv = 1.0 / sqrt(ss / d + eps);", "double inv = 1.0 / sqrt(ss + eps);"),
     ("norm gate not SiLU", "* (w ? w[j] : 1.0) * silu(zrow[j]);", "* (w ? w[j] : 1.0) * zrow[j];"),
 ]
@@ -60,6 +64,7 @@ PINS = [
     ("conv step x T", lambda: P.test_conv_step_repeated_equals_sequence_conv(3)),
     ("conv no leak", P.test_conv_does_not_leak_across_sequences),
     ("norm vs torch", P.test_gated_rmsnorm_matches_torch_rms_norm),
+    ("decode steps = prefill", P.test_decode_steps_equal_prefill_of_the_same_tokens),
     ("norm closed forms", P.test_gated_rmsnorm_closed_forms),
 ]
 

@@ -12,6 +12,7 @@ import os
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 from oracle import oracle as O
 import gdr_inputs as GI
@@ -198,6 +199,19 @@ def test_chunked_form_equals_stepwise(lengths):
     np.testing.assert_allclose(h2, h1, rtol=1e-10, atol=1e-12)
 
 
+@settings(max_examples=12, deadline=None)
+@given(lengths=st.lists(st.integers(0, 150), min_size=1, max_size=4), seed=st.integers(0, 1000),
+       chunk=st.sampled_from([16, 64]))
+def test_chunked_form_equals_stepwise_on_random_packings(lengths, seed, chunk):
+    """Property form of the check above: random packings (empty sequences included), seeds and
+    chunk sizes."""
+    q, k, v, g, beta, cu, H0 = _core_case(seed, lengths, g_scale=0.5)
+    o1, h1 = O.gdr_stepwise(q, k, v, g, beta, cu, H0)
+    o2, h2 = O.gdr_chunked(q, k, v, g, beta, cu, H0, chunk=chunk)
+    np.testing.assert_allclose(o2, o1, rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(h2, h1, rtol=1e-9, atol=1e-11)
+
+
 @pytest.mark.parametrize("split", [1, 37, 64, 128, 129])
 def test_split_and_resume_equals_whole(split):
     q, k, v, g, beta, cu, H0 = _core_case(16, [200])
@@ -345,6 +359,15 @@ def test_prepare_chunks_brute_force(lengths):
     for s0, l0 in zip(st, ln):
         covered[s0:s0 + l0] += 1
     assert np.all(covered == 1)
+
+
+@settings(max_examples=40, deadline=None)
+@given(lengths=st.lists(st.integers(0, 400), min_size=0, max_size=12), chunk=st.integers(1, 130))
+def test_prepare_chunks_brute_force_on_random_offsets(lengths, chunk):
+    cu = GI.cu_seqlens_from_lengths(lengths) if lengths else np.array([0], np.int32)
+    seq, st_, ln = O.prepare_chunks(cu, chunk)
+    exp = [(n, int(cu[n]) + c0, min(chunk, L - c0)) for n, L in enumerate(lengths) for c0 in range(0, L, chunk)]
+    assert list(zip(seq.tolist(), st_.tolist(), ln.tolist())) == exp
 
 
 def test_prepare_chunks_rejects_bad_offsets():

@@ -6,6 +6,7 @@ import re
 
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 
 import gated_delta_rule_63_b200 as G
 from gated_delta_rule_63_b200 import build as B
@@ -52,6 +53,16 @@ def test_prepare_chunks_is_bit_exact_with_oracle(L, lengths):
     cu = GI.cu_seqlens_from_lengths(lengths)
     got = G.prepare_chunks(cu, 64)
     ref = O.prepare_chunks(cu, 64)
+    for g, r in zip(got, ref):
+        assert g.dtype == np.int32 and np.array_equal(g, r)
+
+
+@settings(max_examples=40, deadline=None)
+@given(lengths=st.lists(st.integers(0, 300), min_size=1, max_size=10), chunk=st.integers(1, 100))
+def test_prepare_chunks_bit_exact_on_random_offsets(L, lengths, chunk):
+    cu = GI.cu_seqlens_from_lengths(lengths)
+    got = G.prepare_chunks(cu, chunk)
+    ref = O.prepare_chunks(cu, chunk)
     for g, r in zip(got, ref):
         assert g.dtype == np.int32 and np.array_equal(g, r)
 

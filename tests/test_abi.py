@@ -181,7 +181,6 @@ def test_other_entry_points_reject_bad_arguments(L):
 
 
 def test_binding_fails_loudly_without_the_library(tmp_path):
-    import importlib
     import gated_delta_rule_63_b200 as mod
     saved = mod._lib
     try:

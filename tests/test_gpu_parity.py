@@ -367,6 +367,47 @@ def test_fused_conv_equals_separate_calls(fused_norm):
         assert rel_l2(bits_f64(y_f), bits_f64(ref["y"])) <= TOL_BF16
 
 
+def test_prefill_step_replays_from_a_cuda_graph():
+    """conv -> prefill -> gated norm captured once into a CUDA graph and replayed gives the
+    eager results bit for bit: the calls enqueue only kernels on the caller's stream."""
+    inp = GI.make_full_inputs(82, [300, 70], h0_std=0.02)
+    T, hk, hv = inp.T, inp.hk, inp.hv
+    cu_d = dev_i32(inp.cu_seqlens)
+    x, w = dev_bf16(inp.x), dev_bf16(inp.conv_w)
+    a, b = dev_bf16(inp.a), dev_bf16(inp.b)
+    Al, db, h0 = dev_f32(inp.A_log), dev_f32(inp.dt_bias), dev_f32(inp.h0)
+    z = dev_bf16(inp.z).reshape(T, hv, 128)
+    conv_y = torch.empty_like(x)
+    o = torch.empty((T, hv, 128), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty_like(o)
+    hT = torch.empty((inp.n_seqs, hv, 128, 128), device="cuda")
+    ws = G.prefill_workspace(inp.cu_seqlens, hv, "cuda")
+
+    def step():
+        G.causal_conv(x, w, cu_d, inp.cu_seqlens, None, None, conv_y)
+        q = conv_y[:, : hk * 128].view(T, hk, 128)
+        k = conv_y[:, hk * 128: 2 * hk * 128].view(T, hk, 128)
+        v = conv_y[:, 2 * hk * 128:].view(T, hv, 128)
+        G.chunk_prefill(q, k, v, a, b, Al, db, cu_d, inp.cu_seqlens, h0=h0, hT=hT, o=o, scale=inp.scale,
+                        workspace=ws)
+        G.gated_rmsnorm(o, z, None, inp.eps, y)
+
+    step()   # eager (also the library's one-time set-up)
+    torch.cuda.synchronize()
+    eager = (host_bits(o), host_bits(y), hT.cpu().numpy())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for t in (o, y, hT, conv_y):
+        t.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert G.get_device_error() == 0
+    assert np.array_equal(host_bits(o), eager[0])
+    assert np.array_equal(host_bits(y), eager[1])
+    assert np.array_equal(hT.cpu().numpy(), eager[2])
+
+
 def test_full_path_T4096_fused_norm():
     """The bench workload with the gated norm fused, against the oracle."""
     inp = GI.workload_full_T4096()

@@ -737,6 +737,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // soon as the products reading it are complete; Ut and the chunk scalars are
 // read into registers a chunk ahead; the output of a chunk is finished while
 // the next chunk's first products run.
+// The handoffs (mbarrier: who completes it -> what it allows):
+//   full_qw, full_k, full_mq (per stage): a chunk's copies landed -> its products may read them
+//   bar_p:   P and P2 done (commit)     -> U warps read W H0, output warps read Q H0
+//   u_ready: U, U' tiles written (4 W-row warps) -> K^T U' and O may be issued
+//   bar_h:   K^T U' done (commit)       -> every state warp updates its part of H
+//   h_ready: H tiles written (8 warps)  -> the next chunk's P (which overwrites P's region)
+//   bar_o:   O done (commit)            -> output warps read it; the U tiles may be rewritten
+//   o_free:  O read (4 output warps)    -> the next O may be issued, the Mq stage refilled
 
 // Bounded mbarrier wait that gives up at once after a timeout anywhere in the
 // CTA.  The waiting thread sleeps in try_wait (it takes no issue slots from

@@ -2,13 +2,16 @@
 """Benchmark of the gated delta-rule layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--part all|prefill|decode] [--decode-steps S] [--no-cpu-baseline]
+                    [--part all|prefill|decode] [--decode-steps S] [--decode-slots]
+                    [--no-cpu-baseline]
 
 A step of the default workload is one pass of the prefill path of one layer
 over B=1, T=4096 tokens: causal conv4+SiLU over the 10240 q|k|v channels ->
 chunk-64 gated delta rule (16 key / 48 value heads, dim 128) -> gated RMSNorm.
 The decode path (B=64 sequences, one token each, 1000 consecutive steps) is
-measured in the same run and reported under "decode".  Inputs are seeded
+measured in the same run and reported under "decode", and again in its
+slot-indexed form (64 rows on a pool of 128 cached states) under
+"decode_slots".  Inputs are seeded
 synthetic tensors (gdr_inputs) with the layer's shapes; there are no weights.
 
 `--part prefill` / `--part decode` run one of the two paths alone (for
@@ -220,6 +223,8 @@ def bench_ours(args, rank, world, device):
         torch.cuda.synchronize()
         # decode: B=64, 1000 consecutive steps, state updated in place
         dec_res = bench_decode(torch, G, device, args, steps=args.decode_steps) if args.part == "all" else None
+        slot_res = (bench_decode(torch, G, device, args, steps=args.decode_steps, slots=True)
+                    if args.part == "all" else None)
     if world > 1:
         torch.distributed.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -252,15 +257,18 @@ def bench_ours(args, rank, world, device):
                           "bytes_per_token_fused": B_FUSED,
                           "frac_of_fused_hbm_roofline": (T * B_FUSED + STATE_BYTES) / (ms * 1e-3) / 1e9 / hbm_peak},
         "decode": dec_res,
+        "decode_slots": slot_res,
         "e2e": e2e,
         # conv, prep, chain, norm per step, in the step pass and the prefill-timing pass
-        "gpu_launches": 8 * args.steps + (dec_res["launches"] if dec_res else 0),
+        "gpu_launches": 8 * args.steps + sum(r["launches"] for r in (dec_res, slot_res) if r),
         "clocks": clk.summary(),
     }
     return res
 
 
-def bench_decode(torch, G, device, args, steps=1000):
+def bench_decode(torch, G, device, args, steps=1000, slots=False):
+    """B=64 decode, `steps` consecutive steps.  slots=True runs the slot-indexed form on a
+    pool of 128 entries (the 64 rows name a seeded random half of them)."""
     hbm_peak, _, _ = measured_peaks()
     dec = GI.make_decode_inputs(2, 64, 8)       # 8 distinct token batches, reused round robin
     xs = to_dev(torch, dec.x, device)
@@ -272,23 +280,45 @@ def bench_decode(torch, G, device, args, steps=1000):
     Al = torch.from_numpy(dec.A_log).to(device)
     db = torch.from_numpy(dec.dt_bias).to(device)
     o = torch.empty((64, dec.hv, 128), dtype=torch.bfloat16, device=device)
+    kernel = "gdr_decode_step"
+    if slots:
+        kernel = "gdr_decode_step_slots"
+        n_slots = 128
+        slot = torch.from_numpy(GI.make_slot_table(7, 64, n_slots)).to(device)
+        idx = slot.long()
+        st_pool = torch.zeros((n_slots,) + tuple(st.shape[1:]), dtype=st.dtype, device=device)
+        cs_pool = torch.zeros((n_slots,) + tuple(cs.shape[1:]), dtype=cs.dtype, device=device)
+        st_pool[idx] = st
+        cs_pool[idx] = cs
+        del st, cs
+
+        def step(s):
+            G.decode_step_slots(xs[s % 8], cw, cs_pool, as_[s % 8], bs[s % 8], Al, db, st_pool, slot, o)
+    else:
+        def step(s):
+            G.decode_step(xs[s % 8], cw, cs, as_[s % 8], bs[s % 8], Al, db, st, o)
     for s in range(5):
-        G.decode_step(xs[s % 8], cw, cs, as_[s % 8], bs[s % 8], Al, db, st, o)
+        step(s)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for s in range(steps):
-        G.decode_step(xs[s % 8], cw, cs, as_[s % 8], bs[s % 8], Al, db, st, o)
+        step(s)
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     bytes_step = 64 * STATE_BYTES * 2
     achieved = bytes_step / (ms * 1e-3) / 1e9
-    return {"metric": METRIC_DECODE, "value": 1e3 / ms, "unit": "steps/s", "ms_per_step": ms,
-            "steps": steps, "launches": steps,
-            "roofline": {"kernel": "gdr_decode_step", "bound": "hbm", "achieved": achieved,
-                         "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                         "algorithmic_bytes_per_launch": bytes_step, "traffic": TRAFFIC_DECODE if TRAFFIC_DECODE else None}}
+    res = {"metric": METRIC_DECODE, "value": 1e3 / ms, "unit": "steps/s", "ms_per_step": ms,
+           "steps": steps, "launches": steps,
+           "roofline": {"kernel": kernel, "bound": "hbm", "achieved": achieved,
+                        "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                        "algorithmic_bytes_per_launch": bytes_step,
+                        "traffic": TRAFFIC_DECODE if TRAFFIC_DECODE and not slots else None}}
+    if slots:
+        res["config"] = {"workload": "decode_B64 on a pool of 128 cached states (rows name a seeded "
+                                     "random 64 of them)"}
+    return res
 
 
 def bench_e2e(torch, G, inp, device, args):
@@ -510,6 +540,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--part", choices=["all", "prefill", "decode"], default="all")
     ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--decode-slots", action="store_true",
+                    help="with --part decode: the slot-indexed form on a pool of 128 cached states")
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the bench line: the kernels over other sizes, one JSON line each")
     args = ap.parse_args()
@@ -542,7 +574,7 @@ def main():
         torch.cuda.set_device(device)
         import gated_delta_rule_63_b200 as G
         G.lib()
-        res = bench_decode(torch, G, device, args, steps=args.decode_steps)
+        res = bench_decode(torch, G, device, args, steps=args.decode_steps, slots=args.decode_slots)
         if rank == 0:
             print(json.dumps(res), flush=True)
         return

@@ -17,7 +17,7 @@ import numpy as np
 __all__ = [
     "GdrError", "lib", "status_string", "prepare_chunks", "causal_conv", "chunk_prefill",
     "chunk_prefill_noalloc", "prefill_workspace", "prefill_fused_workspace", "prefill_window",
-    "decode_step", "gated_rmsnorm", "get_device_error", "HEAD_DIM", "CHUNK",
+    "decode_step", "decode_step_slots", "gated_rmsnorm", "get_device_error", "HEAD_DIM", "CHUNK",
 ]
 
 HEAD_DIM = 128
@@ -79,11 +79,13 @@ def lib(path: Optional[str] = None):
                                                    ctypes.c_int]
     L.gdr_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_int,
                                   ctypes.c_int, _vp, _vp, ctypes.c_int, _vp]
+    L.gdr_decode_step_slots.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_int,
+                                        ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp]
     L.gdr_gated_rmsnorm.argtypes = [_vp, _vp, _vp, ctypes.c_float, ctypes.c_int64, ctypes.c_int, _vp,
                                     _vp]
     L.gdr_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), _vp]
     for fn in ("gdr_prepare_chunks", "gdr_causal_conv", "gdr_chunk_prefill", "gdr_decode_step",
-               "gdr_gated_rmsnorm", "gdr_get_device_error"):
+               "gdr_decode_step_slots", "gdr_gated_rmsnorm", "gdr_get_device_error"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
     return L
@@ -299,6 +301,30 @@ def decode_step(x, conv_w, conv_state, a, b, A_log, dt_bias, state, o=None, scal
         _ptr(a, bf, "a"), _ptr(b, bf, "b"), _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"),
         float(scale), int(hk), int(hv), _ptr(state, f32, "state"), _ptr(o, bf, "o"), int(B),
         _stream(stream)))
+    return o
+
+
+def decode_step_slots(x, conv_w, conv_state_pool, a, b, A_log, dt_bias, state_pool, slot, o=None,
+                      scale: float = 1.0, hk: int = 16, stream=None):
+    """One token for each of B rows; row i updates pool entry slot[i] of both pools in place.
+
+    slot is an int32 CUDA tensor [B]; a slot outside [0, n_slots) is a padding row (zero o).
+    """
+    torch = _torch()
+    bf, f32 = torch.bfloat16, torch.float32
+    B, hv = a.shape
+    n_slots = int(state_pool.shape[0])
+    if tuple(slot.shape) != (B,):
+        raise ValueError(f"slot must have shape ({B},), got {tuple(slot.shape)}")
+    if int(conv_state_pool.shape[0]) != n_slots:
+        raise ValueError("conv_state_pool and state_pool must hold the same number of slots")
+    if o is None:
+        o = torch.empty((B, hv, HEAD_DIM), dtype=bf, device=a.device)
+    _check("gdr_decode_step_slots", lib().gdr_decode_step_slots(
+        _ptr(x, bf, "x"), _ptr(conv_w, bf, "conv_w"), _ptr(conv_state_pool, bf, "conv_state_pool"),
+        _ptr(a, bf, "a"), _ptr(b, bf, "b"), _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"),
+        float(scale), int(hk), int(hv), _ptr(state_pool, f32, "state_pool"), n_slots,
+        _ptr(slot, torch.int32, "slot"), _ptr(o, bf, "o"), int(B), _stream(stream)))
     return o
 
 

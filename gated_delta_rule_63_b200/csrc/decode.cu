@@ -22,6 +22,12 @@
 // share a key head form a thread-block cluster: the q/k conv state of that
 // key head is read by all of them, then (after a cluster barrier) rolled by
 // the first one, so the conv state can be updated in place.
+//
+// Slot-indexed form (a serving cache: "33B 只做 18 层 ...", §1.2 keeps the
+// recurrent and conv states of each request in a per-layer cache): row n of
+// the batch reads and writes pool entry slot[n] of the state and conv-state
+// pools; x, a, b and o stay indexed by the row.  A slot outside the pool is a
+// padding row: the pools are not touched and its o row is zero.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -47,6 +53,8 @@ struct DecodeParams {
   int hk, hv, group, channels;
   float *state;
   uint16_t *o;
+  const int32_t *slot;   // [batch] pool entry of each row (slot form only)
+  int n_slots;
   int *err;
 };
 
@@ -64,9 +72,10 @@ __device__ __forceinline__ void st_stream(float *p, float4 v) {
   __stcs(reinterpret_cast<float4 *>(p), v);
 }
 
+template <bool kSlots>
 __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   const int h = blockIdx.x;          // value head
-  const int n = blockIdx.y;          // sequence
+  const int n = blockIdx.y;          // batch row
   const int kh = h / p.group;        // key head shared by `group` value heads
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int C = p.channels;
@@ -80,12 +89,19 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   extern __shared__ float4 s_tile[];   // H, [D][D / 4] float4
 
   // 1. one bulk copy of the 64 KB state tile into shared memory
-  float *S = p.state + (static_cast<size_t>(n) * p.hv + h) * D * D;
   const int row0 = warp * 16;
   const uint32_t bar = smem_u32(&s_bar);
   grid_dep_wait();     // the previous step's state and conv state are complete
   grid_dep_launch();   // the next step's CTAs may take the SMs this grid frees
-  if (tid == 0) {
+  int ns = n;          // state / conv-state entry of this row
+  bool live = true;    // false: a padding row (the pools stay untouched)
+  if (kSlots) {
+    ns = __ldg(p.slot + n);
+    live = ns >= 0 && ns < p.n_slots;
+    if (!live) ns = 0;   // a padding row reads and writes neither pool
+  }
+  float *S = p.state + (static_cast<size_t>(ns) * p.hv + h) * D * D;
+  if (tid == 0 && live) {
     mbar_init(bar, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(bar, D * D * 4);
@@ -94,11 +110,11 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
 
   // 2. conv step of this head's q, k (key head kh) and v channels
   const size_t xoff = static_cast<size_t>(n) * C;
-  const size_t soff = static_cast<size_t>(n) * 3 * C;
+  const size_t soff = static_cast<size_t>(ns) * 3 * C;
   float vq = 0.f, vk = 0.f, vv = 0.f;
   uint16_t new_q = 0, new_k = 0, new_v = 0;   // new newest conv-state entries
   uint16_t keep_q[2] = {0, 0}, keep_k[2] = {0, 0}, keep_v[2] = {0, 0};
-  if (tid < D) {
+  if (tid < D && live) {
     const int cq = kh * D + tid;
     const int ck = p.hk * D + kh * D + tid;
     const int cv = 2 * p.hk * D + h * D + tid;
@@ -133,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     if (lane == 0) { s_sum[0][warp] = a2; s_sum[1][warp] = b2; s_sum[2][warp] = ab; }
   }
   if (tid == 0) {
-    s_ok = mbar_wait(bar, 0, p.err) ? 1 : 0;   // the tile has landed (bounded wait)
+    s_ok = live && mbar_wait(bar, 0, p.err) ? 1 : 0;   // the tile has landed (bounded wait)
     const float av = bf_bits2f(p.a[static_cast<size_t>(n) * p.hv + h]);
     const float bv = bf_bits2f(p.b[static_cast<size_t>(n) * p.hv + h]);
     const float g = -expf(p.A_log[h]) * softplus_f(av + p.dt_bias[h]);
@@ -177,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     s_u[tid] = u;
     const float ov = p.scale * (eg * hq_ + u * kq);
     if (ok) p.o[(static_cast<size_t>(n) * p.hv + h) * D + tid] = f2bf_bits(ov);
+    else if (!live) p.o[(static_cast<size_t>(n) * p.hv + h) * D + tid] = 0;
   }
   __syncthreads();
 
@@ -196,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   // 7. roll the conv state: v channels by this CTA, q/k channels by the first
   //    CTA of the cluster once every CTA has read them
   cluster_wait();
-  if (tid < D) {
+  if (tid < D && live) {
     const int cv = 2 * p.hk * D + h * D + tid;
     p.conv_state[soff + cv] = keep_v[0];
     p.conv_state[soff + C + cv] = keep_v[1];
@@ -218,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
 
 int launch_decode(const void *x, const void *conv_w, void *conv_state, const void *a, const void *b,
                   const float *A_log, const float *dt_bias, float scale, int hk, int hv,
-                  float *state, void *o, int batch, cudaStream_t s) {
+                  float *state, const int32_t *slot, int n_slots, void *o, int batch, cudaStream_t s) {
   if (batch > 65535) return GDR_ERR_SHAPE;
   DecodeParams p;
   p.x = static_cast<const uint16_t *>(x);
@@ -235,6 +252,8 @@ int launch_decode(const void *x, const void *conv_w, void *conv_state, const voi
   p.channels = 2 * hk * D + hv * D;
   p.state = state;
   p.o = static_cast<uint16_t *>(o);
+  p.slot = slot;
+  p.n_slots = n_slots;
   p.err = device_error_ptr();
 
   static bool smem_set[64] = {};
@@ -242,12 +261,17 @@ int launch_decode(const void *x, const void *conv_w, void *conv_state, const voi
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return launch_status(e, "decode: cudaGetDevice");
   if (dev >= 0 && dev < 64 && !smem_set[dev]) {
-    e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileBytes);
+    e = cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileBytes);
     if (e != cudaSuccess) return launch_status(e, "decode: shared memory opt-in");
     smem_set[dev] = true;
   }
-  return launch_status(launch_pdl(decode_kernel, dim3(hv, batch, 1), dim3(kThreads), kTileBytes, s,
-                                  static_cast<unsigned>(p.group), p),
+  const unsigned cluster = static_cast<unsigned>(p.group);
+  return launch_status(slot ? launch_pdl(decode_kernel<true>, dim3(hv, batch, 1), dim3(kThreads), kTileBytes, s,
+                                         cluster, p)
+                            : launch_pdl(decode_kernel<false>, dim3(hv, batch, 1), dim3(kThreads), kTileBytes, s,
+                                         cluster, p),
                        "decode: kernel launch");
 }
 

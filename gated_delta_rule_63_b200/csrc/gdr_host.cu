@@ -76,7 +76,7 @@ const char *gdr_status_string(int status) {
   }
 }
 
-int gdr_abi_version(void) { return 2; }
+int gdr_abi_version(void) { return 3; }
 
 const char *gdr_last_error_string(void) { return gdr::t_last_error_ptr(); }
 
@@ -171,8 +171,27 @@ int gdr_decode_step(const void *x, const void *conv_w, void *conv_state, const v
   if (!aligned16(x) || !aligned16(conv_w) || !aligned16(conv_state) || !aligned16(state) ||
       !aligned16(o))
     return GDR_ERR_ALIGN;
-  return launch_decode(x, conv_w, conv_state, a, b, A_log, dt_bias, scale, hk, hv, state, o, batch,
-                       static_cast<cudaStream_t>(stream));
+  return launch_decode(x, conv_w, conv_state, a, b, A_log, dt_bias, scale, hk, hv, state, nullptr, 0, o,
+                       batch, static_cast<cudaStream_t>(stream));
+}
+
+int gdr_decode_step_slots(const void *x, const void *conv_w, void *conv_state_pool, const void *a,
+                          const void *b, const float *A_log, const float *dt_bias, float scale, int hk,
+                          int hv, float *state_pool, int n_slots, const int32_t *slot, void *o, int batch,
+                          void *stream) {
+  clear_last_error();
+  int st = check_heads(hk, hv);
+  if (st) return st;
+  if (batch < 0 || n_slots < 0) return GDR_ERR_SHAPE;
+  if (batch == 0) return GDR_OK;
+  if (!x || !conv_w || !a || !b || !A_log || !dt_bias || !slot || !o) return GDR_ERR_NULL;
+  // an empty pool makes every row a padding row; the pool pointers are then never read
+  if (n_slots > 0 && (!conv_state_pool || !state_pool)) return GDR_ERR_NULL;
+  if (!aligned16(x) || !aligned16(conv_w) || !aligned16(conv_state_pool) || !aligned16(state_pool) ||
+      !aligned16(o) || (reinterpret_cast<uintptr_t>(slot) & 3u) != 0)
+    return GDR_ERR_ALIGN;
+  return launch_decode(x, conv_w, conv_state_pool, a, b, A_log, dt_bias, scale, hk, hv, state_pool, slot,
+                       n_slots, o, batch, static_cast<cudaStream_t>(stream));
 }
 
 size_t gdr_chunk_prefill_workspace_size(int n_seqs, int hv, int window_chunks, int has_final_state) {

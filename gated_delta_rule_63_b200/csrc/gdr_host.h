@@ -73,7 +73,7 @@ int launch_gated_rmsnorm(const void *o, const void *z, const float *w, float eps
                          void *y, cudaStream_t s);
 int launch_decode(const void *x, const void *conv_w, void *conv_state, const void *a, const void *b,
                   const float *A_log, const float *dt_bias, float scale, int hk, int hv,
-                  float *state, void *o, int batch, cudaStream_t s);
+                  float *state, const int32_t *slot, int n_slots, void *o, int batch, cudaStream_t s);
 int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_stride,
                          int64_t v_stride, const void *a, const void *b,
                          const float *A_log, const float *dt_bias, float scale, int hk, int hv,

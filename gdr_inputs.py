@@ -269,6 +269,16 @@ def make_decode_inputs(seed: int, batch: int, steps: int, hk=HK, hv=HV, dk=DK, d
                         hk, hv, dk, dv, scale)
 
 
+def make_slot_table(seed: int, batch: int, n_slots: int, n_padding: int = 0) -> np.ndarray:
+    """Distinct pool entries for `batch` rows drawn from `n_slots`, int32; the last
+    `n_padding` rows get -1 (padding).  Indices only: no arithmetic of the layer."""
+    if batch - n_padding > n_slots:
+        raise ValueError("more live rows than pool entries")
+    slot = np.full(batch, -1, dtype=np.int32)
+    slot[: batch - n_padding] = _rng(seed).permutation(n_slots)[: batch - n_padding]
+    return slot
+
+
 # ---------------------------------------------------------------------------
 # the five workloads of the layer (sizes and seeds)
 # ---------------------------------------------------------------------------

@@ -75,7 +75,7 @@ GDR_API const char *gdr_status_string(int status);
 
 /* ABI version of this header, bumped whenever a signature or what a call does
  * changes (2: the conv fused into gdr_chunk_prefill,
- * gdr_chunk_prefill_fused_workspace_size). */
+ * gdr_chunk_prefill_fused_workspace_size; 3: gdr_decode_step_slots). */
 GDR_API int gdr_abi_version(void);
 
 /*
@@ -262,6 +262,30 @@ GDR_API size_t gdr_chunk_prefill_noalloc_scratch_bytes(void);
 GDR_API int gdr_decode_step(const void *x, const void *conv_w, void *conv_state, const void *a, const void *b,
                     const float *A_log, const float *dt_bias, float scale, int hk, int hv,
                     float *state, void *o, int batch, void *stream);
+
+/*
+ * gdr_decode_step_slots -- gdr_decode_step on a pool of cached states
+ * ("33B 只做 18 层 ...", §1.2: the layer keeps each request's recurrent state
+ * and conv state in a per-layer cache and resumes from it for the next token).
+ * Row i of the batch reads and writes pool entry slot[i] of both pools; x, a,
+ * b and o stay indexed by the row.  The arithmetic is that of gdr_decode_step,
+ * so a row gives the bits that gdr_decode_step gives on the same inputs.
+ *   conv_state_pool: bf16 [n_slots][3][channels], in/out
+ *   state_pool:      fp32 [n_slots][hv][128][128], in/out
+ *   slot:            int32 [batch], DEVICE memory, 4-byte aligned; read by the
+ *                    kernel, so it may be written by earlier work on the stream
+ *   other arguments as gdr_decode_step.
+ * A slot outside [0, n_slots) (e.g. -1) marks a padding row: neither pool is
+ * read or written for it and its o row is set to zero.  n_slots == 0 (both
+ * pools may then be NULL) makes every row a padding row.  Two rows naming the
+ * same slot in one call race: their results are undefined (every access stays
+ * inside the pools).  Returns GDR_ERR_NULL for a NULL slot array or a NULL
+ * pool with n_slots > 0, GDR_ERR_SHAPE for a negative batch or n_slots.
+ */
+GDR_API int gdr_decode_step_slots(const void *x, const void *conv_w, void *conv_state_pool, const void *a,
+                                  const void *b, const float *A_log, const float *dt_bias, float scale,
+                                  int hk, int hv, float *state_pool, int n_slots, const int32_t *slot,
+                                  void *o, int batch, void *stream);
 
 /*
  * gdr_gated_rmsnorm -- gated RMSNorm over rows of d values

@@ -285,3 +285,42 @@ def decode_steps(inp, steps: Optional[int] = None, heads=None, nthreads=None, ke
         if s in keep_o or (s - steps) in keep_o:
             kept[s] = round_bf16(o)
     return kept, H, cs
+
+
+def decode_step_slots(x, a, b, conv_w, A_log, dt_bias, conv_pool, state_pool, slot, hk, hv,
+                      scale=1.0, dk=128, dv=128, heads=None, nthreads=None):
+    """One decode step on pools of cached states ("33B 只做 18 层 ...", §1.2: each request's
+    recurrent and conv states live in a per-layer cache and the next token resumes from them).
+
+    Row i of the batch (x [B,C], a, b [B,hv] bf16 bits) reads and writes entry slot[i] of
+    conv_pool [S,3,C] and state_pool [S,hv,dk,dv]; a slot outside [0, S) is a padding row
+    whose o row is zero and which touches no entry.  Rows must name distinct slots.  The
+    step itself is the decode step above on the gathered rows.  Returns (o bits [B,hv,dv],
+    new conv pool fp64, new state pool fp64).
+    """
+    slot = np.asarray(slot, dtype=np.int64)
+    S = state_pool.shape[0]
+    live = np.nonzero((slot >= 0) & (slot < S))[0]
+    ids = slot[live]
+    if len(np.unique(ids)) != len(ids):
+        raise ValueError("rows name the same slot twice")
+    cpool = _d(conv_pool).copy()
+    spool = _d(state_pool).copy()
+    B = x.shape[0]
+    o_bits = np.zeros((B, hv, dv), dtype=np.uint16)
+    if len(live) == 0:
+        return o_bits, cpool, spool
+    y, cs = conv_step(bf16_to_f64(x[live]), bf16_to_f64(conv_w), cpool[ids])
+    y = round_bf16_f64(y)
+    q, k, v = split_qkv(y, hk, hv, dk, dv)
+    g, beta = gates(bf16_to_f64(a[live]), bf16_to_f64(b[live]), A_log, dt_bias)
+    cu = np.arange(len(live) + 1, dtype=np.int32)
+    o, Hn = gdr_stepwise(q, k, v, g, beta, cu, h0=spool[ids], scale=scale, heads=heads,
+                         nthreads=nthreads)
+    if heads is not None:
+        keep = np.zeros(hv, bool); keep[list(heads)] = True
+        Hn[:, ~keep] = spool[ids][:, ~keep]
+    o_bits[live] = round_bf16(o)
+    cpool[ids] = cs
+    spool[ids] = Hn
+    return o_bits, cpool, spool

@@ -44,7 +44,7 @@ def test_status_strings(L):
     for code in range(1, 10):
         assert G.status_string(code).startswith("GDR_ERR_")
     assert "UNKNOWN" in G.status_string(12345)
-    assert L.gdr_abi_version() == 2
+    assert L.gdr_abi_version() == 3
 
 
 @pytest.mark.parametrize("lengths", [[0], [1], [64], [65, 0, 128, 1, 63], [5000, 3, 64 * 7 + 1],
@@ -178,6 +178,22 @@ def test_other_entry_points_reject_bad_arguments(L):
     assert L.gdr_decode_step(None, None, None, None, None, None, None, ctypes.c_float(1.0), 16, 48,
                              None, None, 0, None) == 0
     assert L.gdr_gated_rmsnorm(None, None, None, ctypes.c_float(1e-6), 0, 128, None, None) == 0
+
+
+def test_decode_slots_rejects_bad_arguments_on_host(L):
+    f1 = ctypes.c_float(1.0)
+    dec = L.gdr_decode_step_slots
+    # heads, null slot array, null pool with slots, negative sizes, misaligned slot array
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f1, 16, 50, FAKE, 4, FAKE, FAKE, 4, None) == 5
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f1, 16, 48, FAKE, 4, None, FAKE, 4, None) == 1
+    assert dec(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, f1, 16, 48, FAKE, 4, FAKE, FAKE, 4, None) == 1
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f1, 16, 48, None, 4, FAKE, FAKE, 4, None) == 1
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f1, 16, 48, FAKE, -1, FAKE, FAKE, 4, None) == 2
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f1, 16, 48, FAKE, 4, FAKE, FAKE, -1, None) == 2
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f1, 16, 48, FAKE, 4, FAKE + 2, FAKE, 4, None) == 3
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f1, 16, 48, ODD, 4, FAKE, FAKE, 4, None) == 3
+    # an empty batch is accepted without touching the device
+    assert dec(None, None, None, None, None, None, None, f1, 16, 48, None, 0, None, None, 0, None) == 0
 
 
 def test_binding_fails_loudly_without_the_library(tmp_path):

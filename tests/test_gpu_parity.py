@@ -169,6 +169,66 @@ def test_decode_full_batch_sampled_heads():
     assert np.array_equal(cs, O.round_bf16(ref_cs))
 
 
+def test_decode_slots_match_oracle_and_plain_decode():
+    """Decode on pools of cached states: live rows agree with the oracle's slot step and, bit
+    for bit, with the plain decode of the same rows; padding rows are zero; entries no row
+    names keep their bits; an empty pool turns every row into padding."""
+    steps, S = 3, 9
+    dec = GI.make_decode_inputs(55, 5, steps)
+    slot = np.array([7, -1, 0, 3, S + 2], np.int32)
+    live = [0, 2, 3]
+    r = np.random.default_rng(56)
+    C = dec.x.shape[2]
+    cpool = GI.f32_to_bf16_bits(r.standard_normal((S, 3, C)).astype(np.float32))
+    spool = (r.standard_normal((S, dec.hv, 128, 128)) * 0.02).astype(np.float32)
+    for row in live:
+        cpool[slot[row]] = dec.conv_state[row]
+        spool[slot[row]] = dec.state[row]
+    cw = dev_bf16(dec.conv_w)
+    Al, db = dev_f32(dec.A_log), dev_f32(dec.dt_bias)
+    xs, as_, bs = dev_bf16(dec.x), dev_bf16(dec.a), dev_bf16(dec.b)
+    cp_d, sp_d, slot_d = dev_bf16(cpool), dev_f32(spool), dev_i32(slot)
+    outs = []
+    for s in range(steps):
+        o = torch.full((5, dec.hv, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+        G.decode_step_slots(xs[s], cw, cp_d, as_[s], bs[s], Al, db, sp_d, slot_d, o=o, scale=dec.scale)
+        outs.append(host_bits(o))
+    torch.cuda.synchronize()
+    sp_got, cp_got = sp_d.cpu().numpy(), host_bits(cp_d)
+
+    # the oracle's slot step, carried over the steps
+    cp_ref, sp_ref = O.bf16_to_f64(cpool), spool.astype(np.float64)
+    for s in range(steps):
+        o_ref, cp_ref, sp_ref = O.decode_step_slots(dec.x[s], dec.a[s], dec.b[s], dec.conv_w, dec.A_log,
+                                                    dec.dt_bias, cp_ref, sp_ref, slot, dec.hk, dec.hv,
+                                                    scale=dec.scale)
+        assert rel_l2(bits_f64(outs[s][live]), bits_f64(o_ref[live])) <= TOL_BF16, s
+        assert not outs[s][[1, 4]].any(), s
+    ids = slot[live]
+    assert rel_l2(sp_got[ids], sp_ref[ids]) <= TOL_STATE
+    assert np.array_equal(cp_got, O.round_bf16(cp_ref))
+    untouched = [e for e in range(S) if e not in ids]
+    assert np.array_equal(sp_got[untouched], spool[untouched])
+
+    # the plain decode of the live rows gives the same bits
+    plain = GI.DecodeInputs(dec.x[:, live], dec.a[:, live], dec.b[:, live], dec.conv_w,
+                            dec.conv_state[live], dec.state[live], dec.A_log, dec.dt_bias,
+                            dec.hk, dec.hv, scale=dec.scale)
+    p_outs, p_st, p_cs = run_gpu_decode(plain, steps, keep=range(steps))
+    for s in range(steps):
+        assert np.array_equal(outs[s][live], p_outs[s]), s
+    assert np.array_equal(sp_got[ids], p_st)
+    assert np.array_equal(cp_got[ids], p_cs)
+
+    # an empty pool: every row is padding
+    o = torch.full((2, dec.hv, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    G.decode_step_slots(xs[0][:2], cw, torch.empty((0, 3, C), dtype=torch.bfloat16, device="cuda"),
+                        as_[0][:2], bs[0][:2], Al, db,
+                        torch.empty((0, dec.hv, 128, 128), dtype=torch.float32, device="cuda"),
+                        dev_i32(np.array([-1, 0], np.int32)), o=o)
+    assert not host_bits(o).any()
+
+
 # ---------------------------------------------------------------------------
 # chunked prefill
 # ---------------------------------------------------------------------------

@@ -405,6 +405,61 @@ def test_decode_steps_equal_prefill_of_the_same_tokens():
         np.testing.assert_array_equal(kept[s], ob[:, s])
 
 
+def test_decode_slots_reduce_to_the_plain_step_on_gathered_rows():
+    # The slot form is indexing around the decode step: on a pool laid out in any order,
+    # each live row must give exactly what the plain step gives on that row's own state,
+    # write it back to its own entry, leave every other entry bit for bit as it was and
+    # give zeros on padding rows (slot -1 and slot past the pool).
+    hk, hv = 2, 6
+    dec = GI.make_decode_inputs(44, 4, 1, hk=hk, hv=hv)
+    S = 6
+    slot = np.array([4, -1, 1, S + 1], dtype=np.int32)
+    live = [0, 2]
+    r = rng(45)
+    cpool = GI.f32_to_bf16_bits(r.standard_normal((S, 3, dec.x.shape[2])).astype(np.float32))
+    spool = (r.standard_normal((S, hv, 128, 128)) * 0.02).astype(np.float32)
+    for row in live:
+        cpool[slot[row]] = dec.conv_state[row]
+        spool[slot[row]] = dec.state[row]
+    o, cp, sp = O.decode_step_slots(dec.x[0], dec.a[0], dec.b[0], dec.conv_w, dec.A_log, dec.dt_bias,
+                                    O.bf16_to_f64(cpool), spool, slot, hk, hv)
+    plain = GI.DecodeInputs(dec.x[:, live], dec.a[:, live], dec.b[:, live], dec.conv_w,
+                            dec.conv_state[live], dec.state[live], dec.A_log, dec.dt_bias, hk, hv)
+    kept, H, cs = O.decode_steps(plain, keep_o=(0,))
+    np.testing.assert_array_equal(o[live], kept[0])
+    assert not o[[1, 3]].any()
+    np.testing.assert_array_equal(sp[slot[live]], H)
+    np.testing.assert_array_equal(cp[slot[live]], cs)
+    untouched = [e for e in range(S) if e not in slot[live]]
+    np.testing.assert_array_equal(sp[untouched], spool[untouched].astype(np.float64))
+    np.testing.assert_array_equal(cp[untouched], O.bf16_to_f64(cpool[untouched]))
+
+
+def test_decode_slots_identity_is_the_plain_step_and_duplicates_are_rejected():
+    hk, hv = 2, 6
+    dec = GI.make_decode_inputs(46, 3, 1, hk=hk, hv=hv)
+    o, cp, sp = O.decode_step_slots(dec.x[0], dec.a[0], dec.b[0], dec.conv_w, dec.A_log, dec.dt_bias,
+                                    O.bf16_to_f64(dec.conv_state), dec.state, np.arange(3), hk, hv)
+    kept, H, cs = O.decode_steps(dec, keep_o=(0,))
+    np.testing.assert_array_equal(o, kept[0])
+    np.testing.assert_array_equal(sp, H)
+    np.testing.assert_array_equal(cp, cs)
+    with pytest.raises(ValueError):
+        O.decode_step_slots(dec.x[0], dec.a[0], dec.b[0], dec.conv_w, dec.A_log, dec.dt_bias,
+                            O.bf16_to_f64(dec.conv_state), dec.state, np.array([1, 0, 1]), hk, hv)
+
+
+def test_slot_table_generator():
+    slot = GI.make_slot_table(3, 10, 16, n_padding=2)
+    assert slot.dtype == np.int32 and slot.shape == (10,)
+    assert (slot[-2:] == -1).all()
+    live = slot[:-2]
+    assert len(set(live.tolist())) == 8 and live.min() >= 0 and live.max() < 16
+    np.testing.assert_array_equal(slot, GI.make_slot_table(3, 10, 16, n_padding=2))
+    with pytest.raises(ValueError):
+        GI.make_slot_table(3, 10, 4)
+
+
 def test_full_path_shapes_and_rounding():
     inp = GI.make_full_inputs(41, [5, 66], hk=2, hv=6, h0_std=0.02, conv_state_std=1.0,
                               norm_w_std=0.1)

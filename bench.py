@@ -53,9 +53,10 @@ STATE_BYTES = GI.HV * GI.DK * GI.DV * 4                  # one sequence's fp32 s
 
 # DRAM bytes (read + written) per launch from one ncu capture of the current kernels:
 # prefill = prep + state chain on full_T4096 (283.5 + 327.3 MB), decode = one B=64 step
-# (a replayed launch, partly served from L2)
+# (a replayed launch, partly served from L2), and the same step in the slot-indexed form
 TRAFFIC_PREFILL = 610_779_392
 TRAFFIC_DECODE = 355_618_304
+TRAFFIC_DECODE_SLOTS = 354_019_840
 
 
 def measured_peaks():
@@ -314,7 +315,7 @@ def bench_decode(torch, G, device, args, steps=1000, slots=False):
            "roofline": {"kernel": kernel, "bound": "hbm", "achieved": achieved,
                         "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
                         "algorithmic_bytes_per_launch": bytes_step,
-                        "traffic": TRAFFIC_DECODE if TRAFFIC_DECODE and not slots else None}}
+                        "traffic": TRAFFIC_DECODE_SLOTS if slots else TRAFFIC_DECODE}}
     if slots:
         res["config"] = {"workload": "decode_B64 on a pool of 128 cached states (rows name a seeded "
                                      "random 64 of them)"}

@@ -132,10 +132,30 @@ def _tok_stride(t):
     return 0 if t is None else int(t.stride(0))
 
 
-def _stream(stream=None):
+def _device_of(*tensors):
+    """The one device of the given tensors (None skipped); tensors on two devices raise.
+
+    Each call runs on that device with its stream, so no kernel is handed a pointer into
+    another GPU's memory."""
+    dev = None
+    for t in tensors:
+        d = getattr(t, "device", None)
+        if d is None or d.type != "cuda":
+            continue   # not a CUDA tensor: _ptr rejects it by name
+        if dev is None:
+            dev = d
+        elif d != dev:
+            raise ValueError(f"tensors on {dev} and {d}: all tensors of a call must be on one device")
+    return dev
+
+
+def _stream(stream=None, device=None):
     torch = _torch()
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return s.cuda_stream
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if device is not None and getattr(stream, "device", device) != device:
+        raise ValueError(f"stream on {stream.device}, tensors on {device}")
+    return stream.cuda_stream
 
 
 def _host_cu(cu_host):
@@ -171,10 +191,12 @@ def causal_conv(x, w, cu_seqlens, cu_seqlens_host, conv_state_in=None, conv_stat
     if y is None:
         y = torch.empty_like(x)
     C = x.shape[1]
-    _check("gdr_causal_conv", lib().gdr_causal_conv(
-        _ptr(x, bf, "x"), _ptr(w, bf, "w"), _ptr(conv_state_in, bf, "conv_state_in"),
-        _ptr(conv_state_out, bf, "conv_state_out"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup,
-        cu.shape[0] - 1, C, _ptr(y, bf, "y"), _stream(stream)))
+    dev = _device_of(x, w, conv_state_in, conv_state_out, cu_seqlens, y)
+    with torch.cuda.device(dev):
+        _check("gdr_causal_conv", lib().gdr_causal_conv(
+            _ptr(x, bf, "x"), _ptr(w, bf, "w"), _ptr(conv_state_in, bf, "conv_state_in"),
+            _ptr(conv_state_out, bf, "conv_state_out"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup,
+            cu.shape[0] - 1, C, _ptr(y, bf, "y"), _stream(stream, dev)))
     return y
 
 
@@ -255,14 +277,18 @@ def chunk_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_host, h0
             workspace = prefill_fused_workspace(cu_seqlens_host, hk, hv, a.device, window, hT is not None)
         else:
             workspace = prefill_workspace(cu_seqlens_host, hv, a.device, window, hT is not None)
-    _check("gdr_chunk_prefill", lib().gdr_chunk_prefill(
-        _ptr(q, bf, "q", rows=True), _ptr(k, bf, "k", rows=True), _ptr(v, bf, "v", rows=True),
-        _tok_stride(q), _tok_stride(v), _ptr(a, bf, "a"), _ptr(b, bf, "b"),
-        _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"), float(scale), int(hk), int(hv),
-        _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup, cu.shape[0] - 1,
-        _ptr(h0, f32, "h0"), _ptr(hT, f32, "hT"), _ptr(o, bf, "o"),
-        ctypes.byref(fz) if fz is not None else None, _ptr(workspace, torch.uint8, "workspace"),
-        int(workspace.numel()), _stream(stream)))
+    fuse_tensors = [fuse.get(n) for n in ("x", "conv_w", "conv_state_in", "conv_state_out", "z", "y",
+                                          "norm_w")] if fuse is not None else []
+    dev = _device_of(q, k, v, a, b, A_log, dt_bias, cu_seqlens, h0, hT, o, workspace, *fuse_tensors)
+    with torch.cuda.device(dev):
+        _check("gdr_chunk_prefill", lib().gdr_chunk_prefill(
+            _ptr(q, bf, "q", rows=True), _ptr(k, bf, "k", rows=True), _ptr(v, bf, "v", rows=True),
+            _tok_stride(q), _tok_stride(v), _ptr(a, bf, "a"), _ptr(b, bf, "b"),
+            _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"), float(scale), int(hk), int(hv),
+            _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup, cu.shape[0] - 1,
+            _ptr(h0, f32, "h0"), _ptr(hT, f32, "hT"), _ptr(o, bf, "o"),
+            ctypes.byref(fz) if fz is not None else None, _ptr(workspace, torch.uint8, "workspace"),
+            int(workspace.numel()), _stream(stream, dev)))
     return o
 
 
@@ -279,12 +305,14 @@ def chunk_prefill_noalloc(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_
     hv = a.shape[1]
     if o is None:
         o = torch.empty((a.shape[0], hv, HEAD_DIM), dtype=bf, device=a.device)
-    _check("gdr_chunk_prefill_noalloc", lib().gdr_chunk_prefill_noalloc(
-        _ptr(q, bf, "q", rows=True), _ptr(k, bf, "k", rows=True), _ptr(v, bf, "v", rows=True),
-        _tok_stride(q), _tok_stride(v), _ptr(a, bf, "a"), _ptr(b, bf, "b"),
-        _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"), float(scale), int(q.shape[1]),
-        int(hv), _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup, cu.shape[0] - 1,
-        _ptr(h0, f32, "h0"), _ptr(hT, f32, "hT"), _ptr(o, bf, "o"), _stream(stream)))
+    dev = _device_of(q, k, v, a, b, A_log, dt_bias, cu_seqlens, h0, hT, o)
+    with torch.cuda.device(dev):
+        _check("gdr_chunk_prefill_noalloc", lib().gdr_chunk_prefill_noalloc(
+            _ptr(q, bf, "q", rows=True), _ptr(k, bf, "k", rows=True), _ptr(v, bf, "v", rows=True),
+            _tok_stride(q), _tok_stride(v), _ptr(a, bf, "a"), _ptr(b, bf, "b"),
+            _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"), float(scale), int(q.shape[1]),
+            int(hv), _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup, cu.shape[0] - 1,
+            _ptr(h0, f32, "h0"), _ptr(hT, f32, "hT"), _ptr(o, bf, "o"), _stream(stream, dev)))
     return o
 
 
@@ -296,11 +324,13 @@ def decode_step(x, conv_w, conv_state, a, b, A_log, dt_bias, state, o=None, scal
     B, hv = a.shape
     if o is None:
         o = torch.empty((B, hv, HEAD_DIM), dtype=bf, device=a.device)
-    _check("gdr_decode_step", lib().gdr_decode_step(
-        _ptr(x, bf, "x"), _ptr(conv_w, bf, "conv_w"), _ptr(conv_state, bf, "conv_state"),
-        _ptr(a, bf, "a"), _ptr(b, bf, "b"), _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"),
-        float(scale), int(hk), int(hv), _ptr(state, f32, "state"), _ptr(o, bf, "o"), int(B),
-        _stream(stream)))
+    dev = _device_of(x, conv_w, conv_state, a, b, A_log, dt_bias, state, o)
+    with torch.cuda.device(dev):
+        _check("gdr_decode_step", lib().gdr_decode_step(
+            _ptr(x, bf, "x"), _ptr(conv_w, bf, "conv_w"), _ptr(conv_state, bf, "conv_state"),
+            _ptr(a, bf, "a"), _ptr(b, bf, "b"), _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"),
+            float(scale), int(hk), int(hv), _ptr(state, f32, "state"), _ptr(o, bf, "o"), int(B),
+            _stream(stream, dev)))
     return o
 
 
@@ -320,11 +350,13 @@ def decode_step_slots(x, conv_w, conv_state_pool, a, b, A_log, dt_bias, state_po
         raise ValueError("conv_state_pool and state_pool must hold the same number of slots")
     if o is None:
         o = torch.empty((B, hv, HEAD_DIM), dtype=bf, device=a.device)
-    _check("gdr_decode_step_slots", lib().gdr_decode_step_slots(
-        _ptr(x, bf, "x"), _ptr(conv_w, bf, "conv_w"), _ptr(conv_state_pool, bf, "conv_state_pool"),
-        _ptr(a, bf, "a"), _ptr(b, bf, "b"), _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"),
-        float(scale), int(hk), int(hv), _ptr(state_pool, f32, "state_pool"), n_slots,
-        _ptr(slot, torch.int32, "slot"), _ptr(o, bf, "o"), int(B), _stream(stream)))
+    dev = _device_of(x, conv_w, conv_state_pool, a, b, A_log, dt_bias, state_pool, slot, o)
+    with torch.cuda.device(dev):
+        _check("gdr_decode_step_slots", lib().gdr_decode_step_slots(
+            _ptr(x, bf, "x"), _ptr(conv_w, bf, "conv_w"), _ptr(conv_state_pool, bf, "conv_state_pool"),
+            _ptr(a, bf, "a"), _ptr(b, bf, "b"), _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"),
+            float(scale), int(hk), int(hv), _ptr(state_pool, f32, "state_pool"), n_slots,
+            _ptr(slot, torch.int32, "slot"), _ptr(o, bf, "o"), int(B), _stream(stream, dev)))
     return o
 
 
@@ -336,9 +368,11 @@ def gated_rmsnorm(o, z, w=None, eps: float = 1e-6, y=None, stream=None):
         y = torch.empty_like(o)
     d = o.shape[-1]
     rows = o.numel() // d
-    _check("gdr_gated_rmsnorm", lib().gdr_gated_rmsnorm(
-        _ptr(o, bf, "o"), _ptr(z, bf, "z"), _ptr(w, torch.float32, "w"), float(eps), int(rows), int(d),
-        _ptr(y, bf, "y"), _stream(stream)))
+    dev = _device_of(o, z, w, y)
+    with torch.cuda.device(dev):
+        _check("gdr_gated_rmsnorm", lib().gdr_gated_rmsnorm(
+            _ptr(o, bf, "o"), _ptr(z, bf, "z"), _ptr(w, torch.float32, "w"), float(eps), int(rows), int(d),
+            _ptr(y, bf, "y"), _stream(stream, dev)))
     return y
 
 

@@ -31,6 +31,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "gdr_common.cuh"
 #include "gdr_host.h"
 
@@ -256,16 +258,19 @@ int launch_decode(const void *x, const void *conv_w, void *conv_state, const voi
   p.n_slots = n_slots;
   p.err = device_error_ptr();
 
-  static bool smem_set[64] = {};
+  // the shared-memory opt-in, once per device (a bit per device; threads may race to set it,
+  // which only repeats the idempotent calls)
+  static std::atomic<uint64_t> attr_done{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return launch_status(e, "decode: cudaGetDevice");
-  if (dev >= 0 && dev < 64 && !smem_set[dev]) {
+  const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (!bit || !(attr_done.load(std::memory_order_acquire) & bit)) {
     e = cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileBytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileBytes);
     if (e != cudaSuccess) return launch_status(e, "decode: shared memory opt-in");
-    smem_set[dev] = true;
+    attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
   const unsigned cluster = static_cast<unsigned>(p.group);
   return launch_status(slot ? launch_pdl(decode_kernel<true>, dim3(hv, batch, 1), dim3(kThreads), kTileBytes, s,

@@ -205,3 +205,19 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
             mod.lib(str(tmp_path / "missing.so"))
     finally:
         mod._lib = saved
+
+
+def test_binding_refuses_tensors_on_two_devices():
+    """A call runs on its tensors' one device; a mix never reaches a kernel (no GPU needed:
+    the check reads only the tensors' device attributes)."""
+    import types
+    import torch
+    d0 = types.SimpleNamespace(device=torch.device("cuda", 0))
+    d1 = types.SimpleNamespace(device=torch.device("cuda", 1))
+    host = types.SimpleNamespace(device=torch.device("cpu"))
+    assert G._device_of(None, d0, host, d0) == torch.device("cuda", 0)
+    assert G._device_of(None, host) is None
+    with pytest.raises(ValueError):
+        G._device_of(d0, None, d1)
+    with pytest.raises(ValueError):
+        G._stream(types.SimpleNamespace(device=torch.device("cuda", 1), cuda_stream=0), torch.device("cuda", 0))

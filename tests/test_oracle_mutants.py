@@ -43,6 +43,19 @@ MUTANTS = [
      "wc[3] * s0 + wc[1] * s1 + wc[2] * s2 + wc[0] * xv"),
     ("norm mean over d dropped", "double inv = 1.0 / sqrt(ss / d + eps);", "double inv = 1.0 / sqrt(ss + eps);"),
     ("norm gate not SiLU", "* (w ? w[j] : 1.0) * silu(zrow[j]);", "* (w ? w[j] : 1.0) * zrow[j];"),
+    ("delta read from the undecayed state", "u[j] = bt * (vt[j] - acc[j]);", "u[j] = bt * (vt[j] - acc[j] / decay);"),
+    ("write strength of the key head", "const double bt = c->beta[(size_t)t * hv + h];",
+     "const double bt = c->beta[(size_t)t * hv + kh];"),
+    ("chunked: diagonal dropped from the output mask", "for (int j = 0; j <= i; ++j) {", "for (int j = 0; j < i; ++j) {"),
+    ("chunked: forward substitution sign", "x -= A[i * C + j] * Tm[j * C + col];", "x += A[i * C + j] * Tm[j * C + col];"),
+    ("chunked: W H0 added to U", "sacc -= W[i * dk + x] * H[x * dv + y];", "sacc += W[i * dk + x] * H[x * dv + y];"),
+    ("chunked: carried state not decayed", "double sacc = eL * H[x * dv + y];", "double sacc = H[x * dv + y];"),
+    ("chunked: state update without in-chunk decay", "exp(gam[L - 1] - gam[j]) * U[j * dv + y]", "U[j * dv + y]"),
+    ("chunked: output from the carried state undecayed", "double ei = exp(gam[i]);", "double ei = 1.0;"),
+    ("chunked: beta missing in Ut", "sacc += Tm[i * C + j] * bt[j] * V[j * dv + y];",
+     "sacc += Tm[i * C + j] * V[j * dv + y];"),
+    ("chunked: intra-chunk output decay reversed", "intra += qk * exp(gam[i] - gam[j]) * U[j * dv + y];",
+     "intra += qk * exp(gam[j] - gam[i]) * U[j * dv + y];"),
 ]
 
 # the pins, as (name, call)

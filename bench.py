@@ -500,9 +500,16 @@ def cpu_baseline(inp=None):
     t0 = time.perf_counter()
     oracle_step(O, inp)
     dt = time.perf_counter() - t0
+    # the core_T128 workload (recurrence alone, 48 heads) on one thread, for scale
+    small = GI.workload_core_T128()
+    t1 = time.perf_counter()
+    O.core_path(small, nthreads=1)
+    dt1 = time.perf_counter() - t1
     return {"value": inp.T / dt, "unit": "tokens/s", "cores": O.default_threads(), "kind": "oracle",
             "sample": f"one full_T4096 step (all 48 heads, T={inp.T}), fp64 stepwise, "
-                      f"{dt:.2f} s wall"}
+                      f"{dt:.2f} s wall",
+            "one_thread_core_T128": {"value": small.T / dt1, "unit": "tokens/s", "cores": 1,
+                                     "sample": f"core_T128 recurrence, all 48 heads, {dt1:.2f} s wall"}}
 
 
 def bench_reference(args, rank, world):

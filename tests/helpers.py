@@ -47,3 +47,23 @@ def ulp_diff_bf16(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
         x = x.astype(np.int32)
         return np.where(x & 0x8000, 0x8000 - (x & 0x7FFF), x + 0x8000)
     return np.abs(ordered(a_bits) - ordered(b_bits))
+
+
+def restrict_decode_heads(dec, heads):
+    """The decode inputs of the value heads `heads` alone, as a layer with hk = hv = len(heads).
+
+    Value head h reads the q and k channels of key head h // (hv / hk), its own v channels, a,
+    b, A_log, dt_bias and state; nothing else enters its recurrence, so the oracle run on the
+    restriction gives exactly its results on those heads (indexing only).
+    """
+    import gdr_inputs as GI
+    d = dec.dk
+    khs = [h // (dec.hv // dec.hk) for h in heads]
+    chans = np.concatenate([np.arange(kh * d, (kh + 1) * d) for kh in khs]
+                           + [dec.hk * d + np.arange(kh * d, (kh + 1) * d) for kh in khs]
+                           + [2 * dec.hk * d + np.arange(h * d, (h + 1) * d) for h in heads])
+    return GI.DecodeInputs(np.ascontiguousarray(dec.x[:, :, chans]), np.ascontiguousarray(dec.a[:, :, heads]),
+                           np.ascontiguousarray(dec.b[:, :, heads]), np.ascontiguousarray(dec.conv_w[chans]),
+                           np.ascontiguousarray(dec.conv_state[:, :, chans]),
+                           np.ascontiguousarray(dec.state[:, heads]), dec.A_log[heads].copy(),
+                           dec.dt_bias[heads].copy(), len(heads), len(heads), dec.dk, dec.dv, dec.scale)

@@ -449,6 +449,22 @@ def test_decode_slots_identity_is_the_plain_step_and_duplicates_are_rejected():
                             O.bf16_to_f64(dec.conv_state), dec.state, np.array([1, 0, 1]), hk, hv)
 
 
+def test_decode_on_sampled_heads_equals_the_full_layer_on_them():
+    # The parity tests run the oracle on a few value heads of a large decode workload by
+    # cutting out their channels; that cut must give exactly the full layer's results.
+    from tests.helpers import restrict_decode_heads
+    dec = GI.make_decode_inputs(47, 2, 4)
+    heads = [0, 23, 25, 47]            # 23 and 25 share no key head, 0 and 47 are the ends
+    kept, H, cs = O.decode_steps(dec, keep_o=(0, 3))
+    sub = restrict_decode_heads(dec, heads)
+    kept_s, H_s, _ = O.decode_steps(sub, keep_o=(0, 3))
+    for s in (0, 3):
+        np.testing.assert_array_equal(kept_s[s], kept[s][:, heads])
+    np.testing.assert_array_equal(H_s, H[:, heads])
+    # after three or more steps the conv state is the last three inputs, oldest first
+    np.testing.assert_array_equal(O.round_bf16(cs), np.transpose(dec.x[1:], (1, 0, 2)))
+
+
 def test_slot_table_generator():
     slot = GI.make_slot_table(3, 10, 16, n_padding=2)
     assert slot.dtype == np.int32 and slot.shape == (10,)

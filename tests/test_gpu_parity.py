@@ -63,7 +63,8 @@ def check_core(inp, heads=None, h0_inplace=False):
         s, e = int(cu[n]), int(cu[n + 1])
         if e > s:
             assert rel_l2(bits_f64(o_bits[s:e]), bits_f64(ref_bits[s:e])) <= TOL_BF16
-        assert rel_l2(hT[n], ref_hT[n]) <= TOL_STATE or np.linalg.norm(ref_hT[n]) == 0
+        # (a state the oracle leaves exactly zero, e.g. an empty sequence without h0, must be zero)
+        assert rel_l2(hT[n], ref_hT[n]) <= TOL_STATE, n
     return eo, eh
 
 

@@ -150,6 +150,29 @@ def test_beta1_unit_key_overwrites():
     np.testing.assert_allclose(hT[0, 0].T @ k[0, 0], v[0, 0], rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("form", ["stepwise", "chunked"])
+def test_repeated_unit_key_with_full_write_closed_form(form):
+    # One exactly unit key repeated for every token, beta = 1: each token overwrites the
+    # k direction and decays the rest, so H_t = e^gamma_t (I - k k^T) H0 + k v_t^T and
+    # o_t = s (e^gamma_t H0^T (I - k k^T) q_t + v_t (k . q_t)).  In the chunked form every
+    # A entry of a chunk then carries k.k = 1, the most correlated keys can be.
+    q, k, v, g, beta, cu, H0 = _core_case(17, [150], hk=1, hv=1, dk=32, dv=16)
+    kk = unit(rng(18).standard_normal(32))
+    k[:, 0] = kk
+    beta[:] = 1.0
+    g *= 0.05
+    scale = 0.7
+    fn = O.gdr_stepwise if form == "stepwise" else O.gdr_chunked
+    o, hT = fn(q, k, v, g, beta, cu, H0, scale=scale, use_l2norm=False)
+    P = np.eye(32) - np.outer(kk, kk)
+    gam = np.cumsum(g[:, 0])
+    for t in range(150):
+        ref = scale * (math.exp(gam[t]) * H0[0, 0].T @ (P @ q[t, 0]) + v[t, 0] * (kk @ q[t, 0]))
+        np.testing.assert_allclose(o[t, 0], ref, rtol=1e-9, atol=1e-11)
+    Href = math.exp(gam[-1]) * P @ H0[0, 0] + np.outer(kk, v[-1, 0])
+    np.testing.assert_allclose(hT[0, 0], Href, rtol=1e-9, atol=1e-11)
+
+
 def test_large_negative_gate_resets_state():
     q, k, v, g, beta, cu, H0 = _core_case(12, [1], hk=1, hv=1, dk=16, dv=8)
     g[:] = -1e30

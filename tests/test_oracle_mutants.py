@@ -79,6 +79,8 @@ PINS = [
     ("norm vs torch", P.test_gated_rmsnorm_matches_torch_rms_norm),
     ("decode steps = prefill", P.test_decode_steps_equal_prefill_of_the_same_tokens),
     ("norm closed forms", P.test_gated_rmsnorm_closed_forms),
+    ("repeated unit key, stepwise", lambda: P.test_repeated_unit_key_with_full_write_closed_form("stepwise")),
+    ("repeated unit key, chunked", lambda: P.test_repeated_unit_key_with_full_write_closed_form("chunked")),
 ]
 
 

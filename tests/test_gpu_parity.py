@@ -11,7 +11,7 @@ import gated_delta_rule_63_b200 as G
 import gdr_inputs as GI
 from oracle import oracle as O
 from tests.helpers import (TOL_BF16, TOL_STATE, bits_f64, dev_bf16, dev_f32, dev_i32, host_bits,
-                           rel_l2, restrict_decode_heads, ulp_diff_bf16)
+                           rel_l2, ulp_diff_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -504,23 +504,3 @@ def test_prefill_varlen8_full_path_sampled_heads():
     got_y = host_bits(out)[:, heads]
     assert rel_l2(bits_f64(got_y), bits_f64(ref["y"][:, heads])) <= TOL_BF16
     assert rel_l2(hT.cpu().numpy()[:, heads], ref["hT"][:, heads]) <= TOL_STATE
-
-
-# ---------------------------------------------------------------------------
-# the decode workload at its measured length (last: the longest decode test)
-# ---------------------------------------------------------------------------
-
-def test_decode_workload_1000_steps_sampled_heads():
-    """The decode workload as measured: B = 64, 1000 consecutive steps on one state, compared
-    with the oracle run over all 1000 steps at the first and the last step's output and the
-    final state of three sampled value heads; the conv state, all channels, bit for bit."""
-    dec = GI.workload_decode_B64()
-    heads = [0, 23, 47]
-    S = dec.steps
-    outs, st, cs = run_gpu_decode(dec, S, keep=(0, S - 1))
-    kept, H, _ = O.decode_steps(restrict_decode_heads(dec, heads), keep_o=(0, -1))
-    for s in (0, S - 1):
-        assert rel_l2(bits_f64(outs[s][:, heads]), bits_f64(kept[s])) <= TOL_BF16, s
-    assert rel_l2(st[:, heads], H) <= TOL_STATE
-    # after three or more steps the conv state holds the last three inputs, oldest first
-    assert np.array_equal(cs, np.transpose(dec.x[S - 3:], (1, 0, 2)))

@@ -117,7 +117,8 @@ def sigmoid(x: float) -> float:
 
 
 def gates(a: np.ndarray, b: np.ndarray, A_log: np.ndarray, dt_bias: np.ndarray):
-    """g, beta from fp64 a, b of shape [T, hv]."""
+    """g, beta from fp64 a, b of shape [T, hv] ("33B 只做 18 层 ..." (yfxerp.com) §1.2:
+    g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b))."""
     a = _d(a); b = _d(b)
     T, hv = a.shape
     A_log = np.ascontiguousarray(A_log, dtype=np.float32)
@@ -152,20 +153,23 @@ def _core(fn, q, k, v, g, beta, cu, h0, scale, use_l2norm, l2eps, heads, nthread
 
 def gdr_stepwise(q, k, v, g, beta, cu, h0=None, scale=1.0, use_l2norm=True, l2eps=1e-6,
                  heads: Optional[Sequence[int]] = None, nthreads=None):
-    """Token-by-token recurrence in fp64.  Returns (o [T,hv,dv], hT [N,hv,dk,dv])."""
+    """Token-by-token recurrence in fp64 ("Sapiens AI 发布 Agnes-3.0-Flash", delta 规则循环层究竟怎么
+    运作, with the forget gate of "33B 只做 18 层 ..." §1.2).  Returns (o [T,hv,dv], hT [N,hv,dk,dv])."""
     return _core(lib().oracle_gdr_stepwise, q, k, v, g, beta, cu, h0, scale, use_l2norm, l2eps,
                  heads, nthreads)
 
 
 def gdr_chunked(q, k, v, g, beta, cu, h0=None, scale=1.0, use_l2norm=True, l2eps=1e-6,
                 chunk=64, heads=None, nthreads=None):
-    """Chunked form (self-check of the stepwise form)."""
+    """Chunked form, a self-check of the stepwise form ("33B 只做 18 层 ..." §1.2 names a
+    chunk-64 path interchangeable with the per-token one; the algebra is in gdr_oracle.c)."""
     return _core(lib().oracle_gdr_chunked, q, k, v, g, beta, cu, h0, scale, use_l2norm, l2eps,
                  heads, nthreads, extra=(int(chunk),))
 
 
 def causal_conv(x, w, cu, conv_state=None, round_y=True):
-    """Returns (y [T,C], conv_state_out [N,3,C])."""
+    """Kernel-4 causal conv + SiLU over packed sequences ("Agnes-3.0-Flash 深度解析",
+    注意力层的细节).  Returns (y [T,C], conv_state_out [N,3,C])."""
     x = _d(x); w = _d(w)
     T, C = x.shape
     cu = np.ascontiguousarray(cu, dtype=np.int32)
@@ -178,7 +182,8 @@ def causal_conv(x, w, cu, conv_state=None, round_y=True):
 
 
 def conv_step(x, w, conv_state):
-    """One decode step of the conv; returns (y [B,C] fp64 unrounded, new state)."""
+    """One decode step of the conv ("33B 只做 18 层 ..." (mhpq.cn) §2.1, the single-step
+    causal conv); returns (y [B,C] fp64 unrounded, new state)."""
     x = _d(x); w = _d(w)
     st = _d(conv_state).copy()
     B, C = x.shape
@@ -188,6 +193,9 @@ def conv_step(x, w, conv_state):
 
 
 def gated_rmsnorm(o, z, w=None, eps=1e-6):
+    """y = o / sqrt(mean(o^2) + eps) * w * SiLU(z) per row of d ("Agnes-3.0-Flash 深度解析",
+    注意力层的细节: gated RMS-norm; z of width 48 x 128 in the parameter table of "33B 只做 18 层 ..."
+    §2), in fp64, unrounded."""
     o = _d(o); z = _d(z)
     d = o.shape[-1]
     rows = o.size // d
@@ -199,6 +207,8 @@ def gated_rmsnorm(o, z, w=None, eps=1e-6):
 
 
 def prepare_chunks(cu, chunk=64):
+    """Chunk table (chunk_seq, chunk_start, chunk_len) of packed sequences: chunks of `chunk`
+    tokens restarting at every sequence start ("33B 只做 18 层 ..." §1.2, the chunk-64 walk)."""
     cu = np.ascontiguousarray(cu, dtype=np.int32)
     n = cu.shape[0] - 1
     total = int(cu[-1]) if n > 0 else 0

@@ -488,6 +488,42 @@ def test_decode_on_sampled_heads_equals_the_full_layer_on_them():
     np.testing.assert_array_equal(O.round_bf16(cs), np.transpose(dec.x[1:], (1, 0, 2)))
 
 
+@settings(max_examples=12, deadline=None)
+@given(st.integers(1, 5), st.integers(0, 3), st.integers(0, 2**31 - 1))
+def test_decode_slots_on_random_pools_match_the_plain_step(batch, extra_slots, seed):
+    # Any slot table (distinct live entries, padding as -1 or past the pool) gives, row by
+    # row, the plain step on that row's own state, and leaves every other entry as it was.
+    hk, hv = 1, 2
+    r = rng(seed)
+    n_pad = int(r.integers(0, batch + 1))
+    n_slots = batch - n_pad + extra_slots
+    slot = GI.make_slot_table(seed, batch, max(n_slots, 1), n_pad) if n_slots > 0 else np.full(batch, -1, np.int32)
+    if n_pad:
+        slot[batch - n_pad:] = r.choice([-1, n_slots, n_slots + 7], n_pad)
+    dec = GI.make_decode_inputs(seed % 1000, batch, 1, hk=hk, hv=hv)
+    C = dec.x.shape[2]
+    cpool = GI.f32_to_bf16_bits(r.standard_normal((n_slots, 3, C)).astype(np.float32))
+    spool = (r.standard_normal((n_slots, hv, 128, 128)) * 0.02).astype(np.float32)
+    live = [i for i in range(batch) if 0 <= slot[i] < n_slots]
+    for i in live:
+        cpool[slot[i]] = dec.conv_state[i]
+        spool[slot[i]] = dec.state[i]
+    o, cp, sp = O.decode_step_slots(dec.x[0], dec.a[0], dec.b[0], dec.conv_w, dec.A_log, dec.dt_bias,
+                                    O.bf16_to_f64(cpool), spool, slot, hk, hv)
+    pad = [i for i in range(batch) if i not in live]
+    assert not o[pad].any()
+    if live:
+        plain = GI.DecodeInputs(dec.x[:, live], dec.a[:, live], dec.b[:, live], dec.conv_w,
+                                dec.conv_state[live], dec.state[live], dec.A_log, dec.dt_bias, hk, hv)
+        kept, H, cs = O.decode_steps(plain, keep_o=(0,))
+        np.testing.assert_array_equal(o[live], kept[0])
+        np.testing.assert_array_equal(sp[slot[live]], H)
+        np.testing.assert_array_equal(cp[slot[live]], cs)
+    others = [e for e in range(n_slots) if e not in set(slot[live].tolist())]
+    np.testing.assert_array_equal(sp[others], spool[others].astype(np.float64))
+    np.testing.assert_array_equal(cp[others], O.bf16_to_f64(cpool[others]))
+
+
 def test_slot_table_generator():
     slot = GI.make_slot_table(3, 10, 16, n_padding=2)
     assert slot.dtype == np.int32 and slot.shape == (10,)

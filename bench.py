@@ -226,6 +226,7 @@ def bench_ours(args, rank, world, device):
         dec_res = bench_decode(torch, G, device, args, steps=args.decode_steps) if args.part == "all" else None
         slot_res = (bench_decode(torch, G, device, args, steps=args.decode_steps, slots=True)
                     if args.part == "all" else None)
+        other = bench_long_and_varlen(torch, G, device) if args.part == "all" else None
     if world > 1:
         torch.distributed.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -259,19 +260,33 @@ def bench_ours(args, rank, world, device):
                           "frac_of_fused_hbm_roofline": (T * B_FUSED + STATE_BYTES) / (ms * 1e-3) / 1e9 / hbm_peak},
         "decode": dec_res,
         "decode_slots": slot_res,
+        "long_context": other["long_context"] if other else None,
+        "varlen8": other["varlen8"] if other else None,
         "e2e": e2e,
         # conv, prep, chain, norm per step, in the step pass and the prefill-timing pass
-        "gpu_launches": 8 * args.steps + sum(r["launches"] for r in (dec_res, slot_res) if r),
+        "gpu_launches": 8 * args.steps + sum(r["launches"] for r in (dec_res, slot_res, other) if r),
         "clocks": clk.summary(),
     }
     return res
 
 
+_DECODE = {}
+
+
+def decode_workload(steps):
+    """The decode_B64 workload (fresh seeded x, a, b for every step), drawn once per run."""
+    if steps not in _DECODE:
+        _DECODE.clear()
+        _DECODE[steps] = GI.workload_decode_B64(steps=steps)
+    return _DECODE[steps]
+
+
 def bench_decode(torch, G, device, args, steps=1000, slots=False):
-    """B=64 decode, `steps` consecutive steps.  slots=True runs the slot-indexed form on a
-    pool of 128 entries (the 64 rows name a seeded random half of them)."""
+    """B=64 decode, `steps` consecutive steps, each on its own seeded x, a, b (the decode_B64
+    workload).  slots=True runs the slot-indexed form on a pool of 128 entries (the 64 rows
+    name a seeded random half of them)."""
     hbm_peak, _, _ = measured_peaks()
-    dec = GI.make_decode_inputs(2, 64, 8)       # 8 distinct token batches, reused round robin
+    dec = decode_workload(steps)
     xs = to_dev(torch, dec.x, device)
     as_ = to_dev(torch, dec.a, device)
     bs = to_dev(torch, dec.b, device)
@@ -291,16 +306,19 @@ def bench_decode(torch, G, device, args, steps=1000, slots=False):
         cs_pool = torch.zeros((n_slots,) + tuple(cs.shape[1:]), dtype=cs.dtype, device=device)
         st_pool[idx] = st
         cs_pool[idx] = cs
-        del st, cs
+        warm = (st_pool.clone(), cs_pool.clone())
 
-        def step(s):
-            G.decode_step_slots(xs[s % 8], cw, cs_pool, as_[s % 8], bs[s % 8], Al, db, st_pool, slot, o)
+        def step(s, pools=(st_pool, cs_pool)):
+            G.decode_step_slots(xs[s], cw, pools[1], as_[s], bs[s], Al, db, pools[0], slot, o)
     else:
-        def step(s):
-            G.decode_step(xs[s % 8], cw, cs, as_[s % 8], bs[s % 8], Al, db, st, o)
-    for s in range(5):
-        step(s)
+        warm = (st.clone(), cs.clone())
+
+        def step(s, pools=(st, cs)):
+            G.decode_step(xs[s], cw, pools[1], as_[s], bs[s], Al, db, pools[0], o)
+    for s in range(max(3, args.warmup)):      # warm-up on copies of the states
+        step(s % steps, warm)
     torch.cuda.synchronize()
+    del warm
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for s in range(steps):
@@ -312,6 +330,7 @@ def bench_decode(torch, G, device, args, steps=1000, slots=False):
     achieved = bytes_step / (ms * 1e-3) / 1e9
     res = {"metric": METRIC_DECODE, "value": 1e3 / ms, "unit": "steps/s", "ms_per_step": ms,
            "steps": steps, "launches": steps,
+           "inputs": "fresh seeded x, a, b for every step (decode_B64 workload)",
            "roofline": {"kernel": kernel, "bound": "hbm", "achieved": achieved,
                         "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
                         "algorithmic_bytes_per_launch": bytes_step,
@@ -320,6 +339,78 @@ def bench_decode(torch, G, device, args, steps=1000, slots=False):
         res["config"] = {"workload": "decode_B64 on a pool of 128 cached states (rows name a seeded "
                                      "random 64 of them)"}
     return res
+
+
+def n_windows(G, cu_host, hv):
+    """Chunk windows (each a prep and a chain launch) of one prefill call with the default workspace."""
+    longest = int(max(1, ((np.diff(np.asarray(cu_host, dtype=np.int64)) + 63) // 64).max()))
+    win = G.prefill_window(cu_host, hv)
+    return -(-longest // win)
+
+
+def bench_long_and_varlen(torch, G, device, reps=3):
+    """The two other prefill workloads on their seeded inputs, timed with CUDA events on the
+    launching stream (median of `reps` calls after one untimed call; inputs are far larger
+    than L2): long_context = the recurrence alone over B=1, T=262144 (core_T262144);
+    varlen8 = conv -> prefill -> gated norm over 8 packed sequences of U{1024..32768} tokens
+    with initial states (full_varlen8)."""
+    hbm_peak, _, _ = measured_peaks()
+    out = {}
+    hk, hv, d = GI.HK, GI.HV, GI.DK
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    inp = GI.workload_core_T262144()
+    T = inp.T
+    q, k, v = to_dev(torch, inp.q, device), to_dev(torch, inp.k, device), to_dev(torch, inp.v, device)
+    a, b = to_dev(torch, inp.a, device), to_dev(torch, inp.b, device)
+    Al, db = f32(inp.A_log), f32(inp.dt_bias)
+    cu_host = inp.cu_seqlens
+    cu = torch.from_numpy(cu_host).to(device)
+    o = torch.empty((T, hv, d), dtype=torch.bfloat16, device=device)
+    hT = torch.empty((1, hv, d, d), dtype=torch.float32, device=device)
+    ws = G.prefill_workspace(cu_host, hv, device)
+    launches = 2 * n_windows(G, cu_host, hv)
+    ms = timed(lambda: G.chunk_prefill(q, k, v, a, b, Al, db, cu, cu_host, hT=hT, o=o, workspace=ws))
+    byts = T * B_CORE + STATE_BYTES
+    out["long_context"] = {
+        "workload": "core_T262144: B=1 T=262144, recurrence alone, zero initial state, final state out",
+        "metric": METRIC_PREFILL, "value": T / (ms * 1e-3), "unit": "tokens/s", "ms": ms,
+        "algorithmic_bytes": byts, "launches_per_call": launches,
+        "roofline": {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": byts / (ms * 1e-3) / 1e9 / hbm_peak}}
+    del q, k, v, a, b, o, hT, ws, inp
+
+    inp = GI.workload_full_varlen8()
+    T, N = inp.T, inp.n_seqs
+    run = PrefillRunner(torch, G, inp, device)
+    launches8 = 2 + 2 * n_windows(G, inp.cu_seqlens, hv)
+    ms = timed(run.step)
+    fused = T * B_FUSED + 2 * N * STATE_BYTES
+    unfused = T * (B_CONV + B_CORE + B_NORM) + 2 * N * STATE_BYTES
+    out["varlen8"] = {
+        "workload": "full_varlen8: 8 packed sequences, lengths U{1024..32768} (seed 4), initial states, "
+                    "conv4+SiLU -> chunk-64 GDR -> gated RMSNorm",
+        "lengths": [int(x) for x in np.diff(inp.cu_seqlens)],
+        "metric": METRIC_PREFILL, "value": T / (ms * 1e-3), "unit": "tokens/s", "ms": ms,
+        "algorithmic_bytes_fused": fused, "algorithmic_bytes_unfused": unfused, "launches_per_call": launches8,
+        "roofline": {"bound": "hbm", "achieved": fused / (ms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": fused / (ms * 1e-3) / 1e9 / hbm_peak,
+                     "frac_of_unfused_bytes": unfused / (ms * 1e-3) / 1e9 / hbm_peak}}
+    out["launches"] = (1 + reps) * (launches + launches8)
+    return out
 
 
 def bench_e2e(torch, G, inp, device, args):

@@ -17,7 +17,8 @@ import numpy as np
 __all__ = [
     "GdrError", "lib", "status_string", "prepare_chunks", "causal_conv", "chunk_prefill",
     "chunk_prefill_noalloc", "prefill_workspace", "prefill_fused_workspace", "prefill_window",
-    "decode_step", "decode_step_slots", "gated_rmsnorm", "get_device_error", "HEAD_DIM", "CHUNK",
+    "decode_step", "decode_step_slots", "gated_rmsnorm", "get_device_error", "debug_wait_timeout",
+    "HEAD_DIM", "CHUNK",
 ]
 
 HEAD_DIM = 128
@@ -84,8 +85,10 @@ def lib(path: Optional[str] = None):
     L.gdr_gated_rmsnorm.argtypes = [_vp, _vp, _vp, ctypes.c_float, ctypes.c_int64, ctypes.c_int, _vp,
                                     _vp]
     L.gdr_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), _vp]
+    L.gdr_debug_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_ulonglong, _vp, _vp]
     for fn in ("gdr_prepare_chunks", "gdr_causal_conv", "gdr_chunk_prefill", "gdr_decode_step",
-               "gdr_decode_step_slots", "gdr_gated_rmsnorm", "gdr_get_device_error"):
+               "gdr_decode_step_slots", "gdr_gated_rmsnorm", "gdr_get_device_error",
+               "gdr_debug_wait_timeout"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
     return L
@@ -381,3 +384,17 @@ def get_device_error(stream=None) -> int:
     v = ctypes.c_int(0)
     _check("gdr_get_device_error", lib().gdr_get_device_error(ctypes.byref(v), _stream(stream)))
     return v.value
+
+
+def debug_wait_timeout(kind: int, limit: int, device=None, stream=None) -> int:
+    """Run the bounded-wait self-test kernel (gdr_debug_wait_timeout): one CTA waits on an
+    mbarrier nothing arrives at until `limit` runs out (kind 0: polls, kind 1: SM cycles).
+    Returns the kernel's own verdict (0 = the wait gave up); the device error word then holds
+    GDR_ERR_TIMEOUT (read it with get_device_error)."""
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        res = torch.full((1,), -1, dtype=torch.int32, device=dev)
+        _check("gdr_debug_wait_timeout", lib().gdr_debug_wait_timeout(int(kind), int(limit), res.data_ptr(),
+                                                                      _stream(stream, dev)))
+        return int(res.item())

@@ -213,9 +213,10 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   }
 
   // 7. roll the conv state: v channels by this CTA, q/k channels by the first
-  //    CTA of the cluster once every CTA has read them
+  //    CTA of the cluster once every CTA has read them; a CTA whose state tile
+  //    never arrived (bounded wait ran out) leaves its channels as they were
   cluster_wait();
-  if (tid < D && live) {
+  if (tid < D && live && ok) {
     const int cv = 2 * p.hk * D + h * D + tid;
     p.conv_state[soff + cv] = keep_v[0];
     p.conv_state[soff + C + cv] = keep_v[1];

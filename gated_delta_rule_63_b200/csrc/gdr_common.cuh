@@ -376,6 +376,26 @@ __device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t pa
       : "memory");
   return ok != 0;
 }
+// Bounded mbarrier wait that gives up at once after a timeout anywhere in the
+// CTA (`abort` is a shared-memory flag every waiter of the CTA polls).  The
+// waiting thread sleeps in try_wait (it takes no issue slots from the warps
+// that share its scheduler) and gives up after `limit_cycles` SM clock cycles
+// (about 2.2 s by default), setting `abort` and recording GDR_ERR_TIMEOUT.
+__device__ __forceinline__ bool chain_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort, int *err,
+                                           long long limit_cycles = (1LL << 32)) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const long long start = clock64();
+  while (!*abort) {
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (clock64() - start > limit_cycles) {
+      *abort = 1u;
+      raise_device_error(err, GDR_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return false;
+}
+
 // every thread of every CTA of the cluster
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");

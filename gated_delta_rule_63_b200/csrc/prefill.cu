@@ -746,23 +746,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 //   bar_o:   O done (commit)            -> output warps read it; the U tiles may be rewritten
 //   o_free:  O read (4 output warps)    -> the next O may be issued, the Mq stage refilled
 
-// Bounded mbarrier wait that gives up at once after a timeout anywhere in the
-// CTA.  The waiting thread sleeps in try_wait (it takes no issue slots from
-// the warps that share its scheduler) and gives up after about 2^32 cycles.
-__device__ __forceinline__ bool chain_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort, int *err) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const long long start = clock64();
-  while (!*abort) {
-    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
-    if (clock64() - start > (1LL << 32)) {
-      *abort = 1u;
-      raise_device_error(err, GDR_ERR_TIMEOUT);
-      return false;
-    }
-  }
-  return false;
-}
-
 // the same for an mbarrier that another CTA of the cluster arrives on; it polls
 // (with a short back-off) instead of sleeping in try_wait
 __device__ __forceinline__ bool chain_wait_cluster(uint32_t bar, uint32_t parity, volatile uint32_t *abort, int *err) {

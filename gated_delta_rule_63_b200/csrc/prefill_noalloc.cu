@@ -26,26 +26,39 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t{32} << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// device address of the scratch on each device, looked up once per device
+// device address of the scratch on each device, as last looked up
 std::atomic<void *> g_scratch_addr[64];
 std::mutex g_scratch_mutex;
 
-int scratch_for_current_device(void **out) {
+// The address is looked up again on every call made outside stream capture (the
+// lookup is cheap, and a device reset or a new primary context may move the
+// module); a call made while the stream is being captured uses the address of
+// the last call made outside capture, since capture forbids the lookup.
+int scratch_for_current_device(cudaStream_t stream, void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return launch_status(e, "prefill (no-alloc): cudaGetDevice");
   if (dev < 0 || dev >= 64) return GDR_ERR_UNSUPPORTED;
-  void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!p) {
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    p = g_scratch_addr[dev].load(std::memory_order_relaxed);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(stream, &cap);
+  if (e != cudaSuccess) return launch_status(e, "prefill (no-alloc): cudaStreamIsCapturing");
+  if (cap != cudaStreamCaptureStatusNone) {
+    void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
     if (!p) {
-      // the symbol's name is a host stand-in; the device address comes from here
-      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-      if (e != cudaSuccess || !p) return launch_status(e, "prefill (no-alloc): cudaGetSymbolAddress");
-      g_scratch_addr[dev].store(p, std::memory_order_release);
+      set_last_error("prefill (no-alloc): first call on this device made during stream capture; "
+                     "make one call outside capture first",
+                     cudaSuccess);
+      return GDR_ERR_UNSUPPORTED;
     }
+    *out = p;
+    return GDR_OK;
   }
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  void *p = nullptr;
+  // the symbol's name is a host stand-in; the device address comes from here
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p) return launch_status(e, "prefill (no-alloc): cudaGetSymbolAddress");
+  g_scratch_addr[dev].store(p, std::memory_order_release);
   *out = p;
   return GDR_OK;
 }
@@ -73,7 +86,7 @@ int gdr_chunk_prefill_noalloc(const void *q, const void *k, const void *v, int64
     return GDR_ERR_WORKSPACE;
   }
   void *scratch = nullptr;
-  int st = scratch_for_current_device(&scratch);
+  int st = scratch_for_current_device(static_cast<cudaStream_t>(stream), &scratch);
   if (st) return st;
   // the scratch needs no initialisation: every record is written before it is read
   return gdr_chunk_prefill(q, k, v, qk_token_stride, v_token_stride, a, b, A_log, dt_bias, scale, hk,

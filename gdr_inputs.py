@@ -20,11 +20,18 @@ notes):
 
 The generator is numpy's PCG64 seeded with the workload's seed; draws happen
 in a fixed documented order so that a workload is reproducible bit for bit.
+A normal tensor of more than 2^24 elements is drawn in blocks of 2^22
+elements, block i from its own PCG64 whose seed is the i-th of a list of
+63-bit integers drawn from the workload's generator at that point of the
+order; the blocks are filled on all host cores.  Smaller tensors come straight
+from the workload's generator.
 """
 
 from __future__ import annotations
 
 import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Optional
 
 import numpy as np
@@ -41,15 +48,38 @@ CHUNK = 64       # chunk length of the prefill
 # bf16 bit handling (input preparation only)
 # ---------------------------------------------------------------------------
 
+_PAR_MIN = 1 << 24      # tensors above this many elements are processed in blocks
+_PAR_BLOCK = 1 << 22    # elements per block
+
+
+def _blocks(n):
+    return [slice(i, min(n, i + _PAR_BLOCK)) for i in range(0, n, _PAR_BLOCK)]
+
+
+def _each_block(fn, n):
+    """fn(slice) over the blocks of n elements on all host cores (numpy releases the GIL)."""
+    with ThreadPoolExecutor(max(1, os.cpu_count() or 1)) as ex:
+        list(ex.map(fn, _blocks(n)))
+
+
+def _f32_to_bf16_flat(u, out):
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    out[...] = ((u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)).astype(np.uint16)
+
+
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 values to bf16 (round to nearest, ties to even).
 
     Returns the bf16 bit patterns as uint16.  Inputs are finite.
     """
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    lsb = (u >> np.uint32(16)) & np.uint32(1)
-    r = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
-    return r.astype(np.uint16)
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.reshape(-1).view(np.uint32)
+    out = np.empty(u.shape, dtype=np.uint16)
+    if u.size <= _PAR_MIN:
+        _f32_to_bf16_flat(u, out)
+    else:
+        _each_block(lambda s: _f32_to_bf16_flat(u[s], out[s]), u.size)
+    return out.reshape(x.shape)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -69,8 +99,26 @@ def _rng(seed: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(seed))
 
 
+def _standard_normal_f32(rng, shape) -> np.ndarray:
+    """N(0, 1) float32 draws of the given shape (large tensors in seeded blocks, see above)."""
+    n = int(np.prod(shape))
+    if n <= _PAR_MIN:
+        return rng.standard_normal(size=shape, dtype=np.float32)
+    blocks = _blocks(n)
+    seeds = rng.integers(0, 2 ** 63, size=len(blocks), dtype=np.int64)
+    out = np.empty(n, dtype=np.float32)
+    index = {b.start: i for i, b in enumerate(blocks)}
+
+    def fill(s):
+        g = np.random.Generator(np.random.PCG64(int(seeds[index[s.start]])))
+        g.standard_normal(dtype=np.float32, out=out[s])
+
+    _each_block(fill, n)
+    return out.reshape(shape)
+
+
 def _normal_bf16(rng, shape, std=1.0) -> np.ndarray:
-    x = rng.standard_normal(size=shape, dtype=np.float32)
+    x = _standard_normal_f32(rng, shape)
     if std != 1.0:
         x *= np.float32(std)
     return f32_to_bf16_bits(x)
@@ -81,9 +129,21 @@ def _unit_rows_bf16(rng, shape) -> np.ndarray:
 
     This is the input recipe "q and k L2-normalised per head".
     """
-    x = rng.standard_normal(size=shape, dtype=np.float32)
-    n = np.sqrt(np.sum(x.astype(np.float64) ** 2, axis=-1, keepdims=True))
-    return f32_to_bf16_bits((x / n).astype(np.float32))
+    x = _standard_normal_f32(rng, shape)
+    d = shape[-1]
+    flat = x.reshape(-1, d)
+    out = np.empty_like(flat)
+
+    def unit(s):
+        rows = slice(s.start // d, s.stop // d)
+        n = np.sqrt(np.sum(flat[rows].astype(np.float64) ** 2, axis=-1, keepdims=True))
+        out[rows] = (flat[rows] / n).astype(np.float32)
+
+    if x.size <= _PAR_MIN or _PAR_BLOCK % d:
+        unit(slice(0, x.size))
+    else:
+        _each_block(unit, x.size)
+    return f32_to_bf16_bits(out.reshape(shape))
 
 
 def _head_params(rng, hv):
@@ -250,7 +310,8 @@ class DecodeInputs:
 
 def make_decode_inputs(seed: int, batch: int, steps: int, hk=HK, hv=HV, dk=DK, dv=DV,
                        state_std=0.02, conv_state_std=1.0, scale: float = 1.0) -> DecodeInputs:
-    """Draw order: state, conv_state, conv_w, A_log/dt_bias, then per step x, a, b."""
+    """Draw order: state, conv_state, conv_w, A_log/dt_bias, then x, a, b of every step
+    (each one tensor [steps, batch, ...])."""
     rng = _rng(seed)
     C = hk * dk * 2 + hv * dv
     state = (rng.standard_normal(size=(batch, hv, dk, dv), dtype=np.float32)
@@ -258,13 +319,9 @@ def make_decode_inputs(seed: int, batch: int, steps: int, hk=HK, hv=HV, dk=DK, d
     conv_state = _normal_bf16(rng, (batch, CONV_K - 1, C), std=conv_state_std)
     conv_w = _normal_bf16(rng, (C, CONV_K), std=0.5)
     A_log, dt_bias = _head_params(rng, hv)
-    x = np.empty((steps, batch, C), dtype=np.uint16)
-    a = np.empty((steps, batch, hv), dtype=np.uint16)
-    b = np.empty((steps, batch, hv), dtype=np.uint16)
-    for s in range(steps):
-        x[s] = _normal_bf16(rng, (batch, C))
-        a[s] = _normal_bf16(rng, (batch, hv))
-        b[s] = _normal_bf16(rng, (batch, hv))
+    x = _normal_bf16(rng, (steps, batch, C))
+    a = _normal_bf16(rng, (steps, batch, hv))
+    b = _normal_bf16(rng, (steps, batch, hv))
     return DecodeInputs(x, a, b, conv_w, conv_state, state, A_log, dt_bias,
                         hk, hv, dk, dv, scale)
 

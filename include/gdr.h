@@ -222,9 +222,13 @@ GDR_API size_t gdr_chunk_prefill_fused_workspace_size(int n_seqs, int hk, int hv
  *    returns GDR_ERR_WORKSPACE and launches nothing (for 48 value heads:
  *    up to 8 sequences with hT given).  Longer sequences are processed in
  *    more windows, i.e. more kernel launches.
- *  - The first call on a device looks up the scratch's device address with
- *    cudaGetSymbolAddress (once per device, with that device current); make
- *    that first call before any stream capture.
+ *  - Every call made outside stream capture looks up the scratch's device
+ *    address with cudaGetSymbolAddress on the current device (a device reset
+ *    or a new primary context can move it).  A call made while `stream` is
+ *    being captured cannot do the lookup and uses the address found by the
+ *    last call outside capture on that device: make one call on the device
+ *    before capturing, and none across a device reset during capture.  A
+ *    first call made during capture returns GDR_ERR_UNSUPPORTED.
  *  - All calls share the one scratch array, which keeps whatever the last
  *    call left in it (no call relies on its contents: every part is written
  *    before it is read).  Calls whose work overlaps on the GPU -- on two
@@ -258,6 +262,11 @@ GDR_API size_t gdr_chunk_prefill_noalloc_scratch_bytes(void);
  *   A_log, dt_bias: fp32 [hv]
  *   state:      fp32 [batch][hv][128][128], in/out (updated in place)
  *   o:          bf16 [batch][hv][128]
+ * If the bounded wait for a (sequence, value head)'s state tile runs out (the
+ * device error word then reads GDR_ERR_TIMEOUT), that head writes neither its
+ * state, its o row nor its v channels of the conv state; the q and k channels
+ * of its key head roll only if the key head's first value head completed.
+ * Treat the results of such a step as invalid.
  */
 GDR_API int gdr_decode_step(const void *x, const void *conv_w, void *conv_state, const void *a, const void *b,
                     const float *A_log, const float *dt_bias, float scale, int hk, int hv,
@@ -312,6 +321,22 @@ GDR_API const char *gdr_last_error_string(void);
  * This call synchronises `stream`.
  */
 GDR_API int gdr_get_device_error(int *error_out, void *stream);
+
+/*
+ * gdr_debug_wait_timeout -- self-test of the kernels' bounded waits (no
+ * counterpart in the pages: a diagnostic of this library).
+ * Launches one CTA that allocates tensor memory and then waits, with the
+ * wait helpers the kernels use, on an mbarrier that nothing arrives at:
+ *   kind 0: the poll-count bound of the prep, conv and decode kernels;
+ *   kind 1: the clock bound of the prefill's state chain (all warps wait).
+ * `limit` is the bound (polls for kind 0, SM clock cycles for kind 1; at most
+ * 2^31).  When it runs out the kernel records GDR_ERR_TIMEOUT in the device
+ * error word, releases its tensor memory and returns; it writes 0 to
+ * result_dev[0] (1 would mean the wait completed).  No copy or MMA is in
+ * flight while it waits.  Returns GDR_ERR_SHAPE for another kind or a limit
+ * of 0 or above 2^31, GDR_ERR_NULL without result_dev.
+ */
+GDR_API int gdr_debug_wait_timeout(int kind, unsigned long long limit, int *result_dev, void *stream);
 
 #ifdef __cplusplus
 }

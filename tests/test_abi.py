@@ -163,6 +163,14 @@ def test_fused_workspace_size(L):
     assert L.gdr_chunk_prefill_fused_workspace_size(2, 16, 48, -1, 1, 1) == 0
 
 
+def test_wait_self_test_rejects_bad_arguments(L):
+    L.gdr_debug_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_ulonglong, ctypes.c_void_p, ctypes.c_void_p]
+    assert L.gdr_debug_wait_timeout(2, 10, FAKE, None) == 2          # unknown kind
+    assert L.gdr_debug_wait_timeout(0, 0, FAKE, None) == 2           # no bound
+    assert L.gdr_debug_wait_timeout(0, 1 << 40, FAKE, None) == 2     # bound above 2^31
+    assert L.gdr_debug_wait_timeout(0, 10, None, None) == 1          # no result word
+
+
 def test_other_entry_points_reject_bad_arguments(L):
     cu, cup = _cu([4])
     assert L.gdr_causal_conv(FAKE, FAKE, None, None, FAKE, cup, 1, 10, FAKE, None) == 2   # C % 8

@@ -5,6 +5,7 @@ invariant of the recurrence, a library routine or brute force, chosen so that
 a dropped term, a wrong sign, a wrong index or a transposed operand in the
 oracle fails at least one of them.
 """
+import dataclasses
 import json
 import math
 import os
@@ -545,3 +546,70 @@ def test_full_path_shapes_and_rounding():
     # the conv state out is made of the raw inputs: the last 3 tokens of each sequence
     np.testing.assert_array_equal(out["conv_state_out"][1], inp.x[71 - 3:71])
     np.testing.assert_array_equal(out["conv_state_out"][0], inp.x[2:5])
+
+
+# ---------------------------------------------------------------------------
+# composition of the full path: channel order of the conv output and the
+# rounding points between the kernels
+# ---------------------------------------------------------------------------
+
+def _perturb_channels(inp, lo, hi, seed):
+    x = inp.x.copy()
+    x[:, lo:hi] = GI.f32_to_bf16_bits(rng(seed).standard_normal((x.shape[0], hi - lo)).astype(np.float32))
+    return dataclasses.replace(inp, x=x)
+
+
+def test_full_path_reads_q_k_v_from_their_channel_blocks():
+    """The conv runs over the channels [q | k | v] (hk*128 q channels, hk*128 k channels, then
+    hv*128 v channels, value head h in block h).  The conv is depthwise, so a channel of x
+    reaches only the same channel of the conv output.  q enters only the output: new values
+    in the q channels change o and leave the final state identical bit for bit.  New values
+    in the k channels of key head 1 change the state of value heads 3..5 only (heads group
+    contiguously, three per key head).  New values in the v channels of value head 4 change
+    that head's state and output alone."""
+    hk, hv, d = 2, 6, 128
+    inp = GI.make_full_inputs(42, [40, 70], hk=hk, hv=hv, h0_std=0.02)
+    base = O.full_path(inp)
+    heads_changed = lambda out, key: [h for h in range(hv)
+                                      if not np.array_equal(out[key][..., h, :] if key == "o" else out[key][:, h],
+                                                            base[key][..., h, :] if key == "o" else base[key][:, h])]
+    pq = O.full_path(_perturb_channels(inp, 0, hk * d, 1))
+    assert np.array_equal(pq["hT"], base["hT"])
+    assert heads_changed(pq, "o") == list(range(hv))
+    pk = O.full_path(_perturb_channels(inp, hk * d + d, 2 * hk * d, 2))
+    assert heads_changed(pk, "hT") == [3, 4, 5]
+    pv = O.full_path(_perturb_channels(inp, 2 * hk * d + 4 * d, 2 * hk * d + 5 * d, 3))
+    assert heads_changed(pv, "hT") == [4]
+    assert heads_changed(pv, "o") == [4]
+
+
+def test_full_path_is_the_recurrence_on_the_rounded_conv_output():
+    """The recurrence of the full path runs on the conv output as the bf16 tensor the conv
+    emits, split at the channel offsets of the [q | k | v] layout (written out here), with
+    the gates of a and b: the full path's o and final state equal those of the pinned
+    stepwise recurrence run on those slices."""
+    hk, hv, d = 2, 6, 128
+    inp = GI.make_full_inputs(45, [33, 66], hk=hk, hv=hv, h0_std=0.02, conv_state_std=1.0)
+    out = O.full_path(inp)
+    yc, _ = O.causal_conv(O.bf16_to_f64(inp.x), O.bf16_to_f64(inp.conv_w), inp.cu_seqlens,
+                          O.bf16_to_f64(inp.conv_state), round_y=False)
+    assert np.array_equal(out["conv_y"], O.round_bf16(yc))
+    y = O.bf16_to_f64(out["conv_y"])
+    T = y.shape[0]
+    q = y[:, 0:256].reshape(T, hk, d)
+    k = y[:, 256:512].reshape(T, hk, d)
+    v = y[:, 512:1280].reshape(T, hv, d)
+    g, beta = O.gates(O.bf16_to_f64(inp.a), O.bf16_to_f64(inp.b), inp.A_log, inp.dt_bias)
+    o, hT = O.gdr_stepwise(q, k, v, g, beta, inp.cu_seqlens, h0=inp.h0)
+    assert np.array_equal(out["o"], O.round_bf16(o))
+    assert np.array_equal(out["hT"], hT)
+
+
+def test_full_path_norm_reads_the_bf16_output():
+    """The gated norm of the full path reads o as the bf16 tensor the recurrence emits: y is
+    the pinned gated norm of the returned o bits, rounded to bf16, exactly.  (On this input
+    the unrounded o gives a different y in many places, so the rounding point is seen.)"""
+    inp = GI.make_full_inputs(44, [50, 30], hk=2, hv=6, h0_std=0.02, norm_w_std=0.1)
+    out = O.full_path(inp)
+    y = O.round_bf16(O.gated_rmsnorm(O.bf16_to_f64(out["o"]), O.bf16_to_f64(inp.z), inp.norm_w, inp.eps))
+    assert np.array_equal(out["y"], y)

@@ -7,6 +7,7 @@ tests/test_oracle.py and requires that at least one of them fails.  The real ora
 restored afterwards.  Mutants apply to every occurrence of the pattern, so the stepwise and
 chunked forms carry the same slip where both have the line.
 """
+import inspect
 import os
 import subprocess
 
@@ -120,4 +121,47 @@ def test_pins_pass_on_the_real_oracle(restore_oracle):
     assert os.path.exists(O.build())
     O._lib = None
     for _, pin in PINS:
+        pin()
+
+
+# Slips in the Python composition of the oracle (oracle/oracle.py): (name, function, pattern,
+# replacement).  The mutated function replaces the real one in the module for the test.
+COMPOSITION_MUTANTS = [
+    ("q and k channel blocks swapped", "split_qkv",
+     "q = y[:, : hk * dk].reshape(T, hk, dk)\n    k = y[:, hk * dk: 2 * hk * dk].reshape(T, hk, dk)",
+     "k = y[:, : hk * dk].reshape(T, hk, dk)\n    q = y[:, hk * dk: 2 * hk * dk].reshape(T, hk, dk)"),
+    ("v read from the k channels on", "split_qkv", "v = y[:, 2 * hk * dk:].reshape(T, hv, dv)",
+     "v = y[:, hk * dk: hk * dk + hv * dv].reshape(T, hv, dv)"),
+    ("o not rounded before the gated norm", "full_path", "y = gated_rmsnorm(bf16_to_f64(o_bits),",
+     "y = gated_rmsnorm(o,"),
+    ("conv output not rounded", "full_path", "causal_conv(x, w, inp.cu_seqlens, cs, round_y=True)",
+     "causal_conv(x, w, inp.cu_seqlens, cs, round_y=False)"),
+]
+
+COMPOSITION_PINS = PINS + [
+    ("channel blocks", P.test_full_path_reads_q_k_v_from_their_channel_blocks),
+    ("recurrence on the rounded conv output", P.test_full_path_is_the_recurrence_on_the_rounded_conv_output),
+    ("norm reads the bf16 o", P.test_full_path_norm_reads_the_bf16_output),
+]
+
+
+@pytest.mark.parametrize("name,func,pattern,replacement", COMPOSITION_MUTANTS,
+                         ids=[m[0] for m in COMPOSITION_MUTANTS])
+def test_planted_composition_mistake_fails_a_pin(name, func, pattern, replacement, monkeypatch):
+    src = inspect.getsource(getattr(O, func))
+    assert pattern in src, f"pattern of mutant '{name}' not found"
+    ns = dict(vars(O))
+    exec(compile(src.replace(pattern, replacement), O.__file__, "exec"), ns)
+    monkeypatch.setattr(O, func, ns[func])
+    failed = []
+    for pin_name, pin in COMPOSITION_PINS:
+        try:
+            pin()
+        except Exception:
+            failed.append(pin_name)
+    assert failed, f"no pin catches the planted mistake '{name}'"
+
+
+def test_composition_pins_pass_on_the_real_oracle():
+    for _, pin in COMPOSITION_PINS[len(PINS):]:
         pin()

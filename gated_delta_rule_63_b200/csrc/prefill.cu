@@ -1079,7 +1079,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           tmem_ld16(tl + C_COL_H + 64 + 16 * hh, hb);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) hreg[16 * hh + j] = eL * hreg[16 * hh + j] + (ha[j] + hb[j]);
+          for (int j = 0; j < 8; ++j) {
+            const float2 hn = __ffma2_rn(make_float2(eL, eL), make_float2(hreg[16 * hh + 2 * j], hreg[16 * hh + 2 * j + 1]),
+                                         __fadd2_rn(make_float2(ha[2 * j], ha[2 * j + 1]), make_float2(hb[2 * j], hb[2 * j + 1])));
+            hreg[16 * hh + 2 * j] = hn.x;
+            hreg[16 * hh + 2 * j + 1] = hn.y;
+          }
         }
         write_h();
       }

@@ -227,6 +227,7 @@ def bench_ours(args, rank, world, device):
         slot_res = (bench_decode(torch, G, device, args, steps=args.decode_steps, slots=True)
                     if args.part == "all" else None)
         other = bench_long_and_varlen(torch, G, device) if args.part == "all" else None
+        mixed = bench_mixed(torch, G, device, args) if args.part == "all" else None
     if world > 1:
         torch.distributed.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -262,9 +263,10 @@ def bench_ours(args, rank, world, device):
         "decode_slots": slot_res,
         "long_context": other["long_context"] if other else None,
         "varlen8": other["varlen8"] if other else None,
+        "mixed_serving": mixed,
         "e2e": e2e,
         # conv, prep, chain, norm per step, in the step pass and the prefill-timing pass
-        "gpu_launches": 8 * args.steps + sum(r["launches"] for r in (dec_res, slot_res, other) if r),
+        "gpu_launches": 8 * args.steps + sum(r["launches"] for r in (dec_res, slot_res, other, mixed) if r),
         "clocks": clk.summary(),
     }
     return res
@@ -339,6 +341,82 @@ def bench_decode(torch, G, device, args, steps=1000, slots=False):
         res["config"] = {"workload": "decode_B64 on a pool of 128 cached states (rows name a seeded "
                                      "random 64 of them)"}
     return res
+
+
+def bench_mixed(torch, G, device, args, steps=20):
+    """A mixed serving step on one pool of 128 cached states (mixed_serving workload): 4 new
+    requests of U{256..4096} tokens prefilled into free entries (gdr_chunk_prefill_slots, from
+    zero), then one decode token for the 64 running rows from theirs (gdr_decode_step_slots,
+    fresh decode_B64 inputs each step).  Events on the launching stream around each call; the
+    pool (403 MB) and the step's inputs exceed L2."""
+    hbm_peak, _, _ = measured_peaks()
+    mix = GI.workload_mixed_serving()
+    inp = mix.prefill
+    dec = decode_workload(args.decode_steps)
+    hv, d = GI.HV, GI.DK
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    q, k, v = to_dev(torch, inp.q, device), to_dev(torch, inp.k, device), to_dev(torch, inp.v, device)
+    a, b = to_dev(torch, inp.a, device), to_dev(torch, inp.b, device)
+    Al, db = f32(inp.A_log), f32(inp.dt_bias)
+    cu_host = inp.cu_seqlens
+    cu = torch.from_numpy(cu_host).to(device)
+    T = inp.T
+    o = torch.empty((T, hv, d), dtype=torch.bfloat16, device=device)
+    ws = G.prefill_workspace(cu_host, hv, device, has_final_state=False)
+    new_slot = torch.from_numpy(mix.new_slot).to(device)
+    dslot = torch.from_numpy(mix.decode_slot).to(device)
+    st_pool = torch.zeros((mix.n_slots, hv, d, d), dtype=torch.float32, device=device)
+    st_pool[dslot.long()] = torch.from_numpy(dec.state).to(device)
+    cs_pool = torch.zeros((mix.n_slots,) + tuple(dec.conv_state.shape[1:]), dtype=torch.bfloat16, device=device)
+    cs_pool[dslot.long()] = to_dev(torch, dec.conv_state, device)
+    xs, as_, bs = to_dev(torch, dec.x, device), to_dev(torch, dec.a, device), to_dev(torch, dec.b, device)
+    cw = to_dev(torch, dec.conv_w, device)
+    dAl, ddb = f32(dec.A_log), f32(dec.dt_bias)
+    od = torch.empty((len(mix.decode_slot), hv, d), dtype=torch.bfloat16, device=device)
+    n_dec = xs.shape[0]
+
+    def prefill():
+        G.chunk_prefill_slots(q, k, v, a, b, Al, db, cu, cu_host, st_pool, new_slot, init_from_pool=False,
+                              o=o, workspace=ws)
+
+    def decode(s):
+        G.decode_step_slots(xs[s % n_dec], cw, cs_pool, as_[s % n_dec], bs[s % n_dec], dAl, ddb, st_pool,
+                            dslot, o=od)
+
+    for s in range(3):
+        prefill()
+        decode(s)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for s in range(steps):
+        ev[s][0].record()
+        prefill()
+        ev[s][1].record()
+        decode(3 + s)
+        ev[s][2].record()
+    torch.cuda.synchronize()
+    pre = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    dms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
+    step = statistics.median(e[0].elapsed_time(e[2]) for e in ev)
+    n_new, rows = len(mix.new_slot), len(mix.decode_slot)
+    pbytes = T * B_CORE + n_new * STATE_BYTES          # from zero: the entries are only written
+    dbytes = rows * STATE_BYTES * 2
+    launches = 2 * n_windows(G, cu_host, hv) + 1
+    return {"workload": f"mixed_serving: {n_new} new requests, lengths {[int(x) for x in np.diff(cu_host)]}, "
+                        f"prefilled into free entries of a {mix.n_slots}-entry pool; {rows} running rows "
+                        "decode one token from theirs (decode_B64 inputs)",
+            "metric": "tokens/s (prompt + decoded tokens per mixed step)",
+            "value": (T + rows) / (step * 1e-3), "unit": "tokens/s", "ms_per_step": step,
+            "prefill_slots": {"ms": pre, "tokens_per_s": T / (pre * 1e-3),
+                              "roofline": {"kernel": "gdr_chunk_prefill_slots", "bound": "hbm",
+                                           "achieved": pbytes / (pre * 1e-3) / 1e9, "peak": hbm_peak,
+                                           "unit": "GB/s", "frac": pbytes / (pre * 1e-3) / 1e9 / hbm_peak,
+                                           "algorithmic_bytes_per_launch": pbytes}},
+            "decode_slots": {"ms": dms,
+                             "roofline": {"kernel": "gdr_decode_step_slots", "bound": "hbm",
+                                          "achieved": dbytes / (dms * 1e-3) / 1e9, "peak": hbm_peak,
+                                          "unit": "GB/s", "frac": dbytes / (dms * 1e-3) / 1e9 / hbm_peak}},
+            "steps": steps, "launches": (3 + steps) * launches}
 
 
 def n_windows(G, cu_host, hv):

@@ -16,7 +16,7 @@ import numpy as np
 
 __all__ = [
     "GdrError", "lib", "status_string", "prepare_chunks", "causal_conv", "chunk_prefill",
-    "chunk_prefill_noalloc", "prefill_workspace", "prefill_fused_workspace", "prefill_window",
+    "chunk_prefill_noalloc", "chunk_prefill_slots", "prefill_workspace", "prefill_fused_workspace", "prefill_window",
     "decode_step", "decode_step_slots", "gated_rmsnorm", "get_device_error", "debug_wait_timeout",
     "HEAD_DIM", "CHUNK",
 ]
@@ -86,9 +86,12 @@ def lib(path: Optional[str] = None):
                                     _vp]
     L.gdr_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), _vp]
     L.gdr_debug_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_ulonglong, _vp, _vp]
+    L.gdr_chunk_prefill_slots.argtypes = [_vp, _vp, _vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp, _vp,
+                                          ctypes.c_float, ctypes.c_int, ctypes.c_int, _vp, _ip, ctypes.c_int,
+                                          _vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, ctypes.c_size_t, _vp]
     for fn in ("gdr_prepare_chunks", "gdr_causal_conv", "gdr_chunk_prefill", "gdr_decode_step",
                "gdr_decode_step_slots", "gdr_gated_rmsnorm", "gdr_get_device_error",
-               "gdr_debug_wait_timeout"):
+               "gdr_debug_wait_timeout", "gdr_chunk_prefill_slots"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
     return L
@@ -316,6 +319,32 @@ def chunk_prefill_noalloc(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_
             _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"), float(scale), int(q.shape[1]),
             int(hv), _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup, cu.shape[0] - 1,
             _ptr(h0, f32, "h0"), _ptr(hT, f32, "hT"), _ptr(o, bf, "o"), _stream(stream, dev)))
+    return o
+
+
+def chunk_prefill_slots(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_host, state_pool, slot,
+                        init_from_pool: bool = False, o=None, scale: float = 1.0, workspace=None, stream=None):
+    """gdr_chunk_prefill on a pool of cached states: sequence n starts from entry slot[n] of
+    state_pool (or from zero, init_from_pool=False) and leaves its final state there.  A slot
+    outside the pool is a sequence that starts from zero and keeps no state."""
+    torch = _torch()
+    bf, f32 = torch.bfloat16, torch.float32
+    cu, cup = _host_cu(cu_seqlens_host)
+    hv = a.shape[1]
+    if o is None:
+        o = torch.empty((a.shape[0], hv, HEAD_DIM), dtype=bf, device=a.device)
+    if workspace is None:
+        workspace = prefill_workspace(cu, hv, a.device, has_final_state=False)
+    dev = _device_of(q, k, v, a, b, A_log, dt_bias, cu_seqlens, state_pool, slot, o, workspace)
+    with torch.cuda.device(dev):
+        _check("gdr_chunk_prefill_slots", lib().gdr_chunk_prefill_slots(
+            _ptr(q, bf, "q", rows=True), _ptr(k, bf, "k", rows=True), _ptr(v, bf, "v", rows=True),
+            _tok_stride(q), _tok_stride(v), _ptr(a, bf, "a"), _ptr(b, bf, "b"),
+            _ptr(A_log, f32, "A_log"), _ptr(dt_bias, f32, "dt_bias"), float(scale), int(q.shape[1]),
+            int(hv), _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cup, cu.shape[0] - 1,
+            _ptr(state_pool, f32, "state_pool"), int(state_pool.shape[0]), _ptr(slot, torch.int32, "slot"),
+            int(bool(init_from_pool)), _ptr(o, bf, "o"), _ptr(workspace, torch.uint8, "workspace"),
+            workspace.numel(), _stream(stream, dev)))
     return o
 
 

@@ -76,7 +76,7 @@ const char *gdr_status_string(int status) {
   }
 }
 
-int gdr_abi_version(void) { return 3; }
+int gdr_abi_version(void) { return 4; }
 
 const char *gdr_last_error_string(void) { return gdr::t_last_error_ptr(); }
 
@@ -291,6 +291,46 @@ int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_st
   return launch_chunk_prefill(q, k, v, qk_stride, v_stride, a, b, A_log, dt_bias, scale, hk, hv,
                               cu_dev, cu_host, n_seqs, total, max_chunks, h0, hT, o, z, norm_w, eps, y, workspace,
                               workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int gdr_chunk_prefill_slots(const void *q, const void *k, const void *v, int64_t qk_stride, int64_t v_stride,
+                            const void *a, const void *b, const float *A_log, const float *dt_bias, float scale,
+                            int hk, int hv, const int32_t *cu_dev, const int32_t *cu_host, int n_seqs,
+                            float *state_pool, int n_slots, const int32_t *slot, int init_from_pool, void *o,
+                            void *workspace, size_t workspace_bytes, void *stream) {
+  clear_last_error();
+  int st = check_heads(hk, hv);
+  if (st) return st;
+  if (n_slots < 0 || (init_from_pool != 0 && init_from_pool != 1)) return GDR_ERR_SHAPE;
+  if (qk_stride == 0) qk_stride = static_cast<int64_t>(hk) * kHeadDim;
+  if (v_stride == 0) v_stride = static_cast<int64_t>(hv) * kHeadDim;
+  if (qk_stride < static_cast<int64_t>(hk) * kHeadDim || v_stride < static_cast<int64_t>(hv) * kHeadDim)
+    return GDR_ERR_SHAPE;
+  if (qk_stride % 8 != 0 || v_stride % 8 != 0) return GDR_ERR_ALIGN;
+  if (!cu_host) return GDR_ERR_NULL;
+  st = check_cu_seqlens(cu_host, n_seqs);
+  if (st) return st;
+  if (n_seqs == 0) return GDR_OK;
+  if (!cu_dev || !slot) return GDR_ERR_NULL;
+  if (n_slots > 0 && !state_pool) return GDR_ERR_NULL;
+  const int total = cu_host[n_seqs];
+  if (total > 0 && (!q || !k || !v || !a || !b || !A_log || !dt_bias || !o)) return GDR_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state_pool) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(slot) & 3u) != 0)
+    return GDR_ERR_ALIGN;
+  int max_chunks = 0;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int nc = (cu_host[i + 1] - cu_host[i] + kChunk - 1) / kChunk;
+    if (nc > max_chunks) max_chunks = nc;
+  }
+  // the records of a one-chunk window and the carry of sequences without an entry
+  const size_t rec_bytes = max_chunks > 0 ? chunk_prefill_workspace_bytes(n_seqs, hv, 1, true) : 0;
+  if (rec_bytes != 0 && (!workspace || workspace_bytes < rec_bytes)) return GDR_ERR_WORKSPACE;
+  if (n_slots == 0 && total == 0) return GDR_OK;   // no entry to write, nothing to compute
+  PrefillPool pool{state_pool, n_slots, slot, init_from_pool};
+  return launch_chunk_prefill(q, k, v, qk_stride, v_stride, a, b, A_log, dt_bias, scale, hk, hv, cu_dev, cu_host,
+                              n_seqs, total, max_chunks, nullptr, nullptr, o, nullptr, nullptr, 0.0f, nullptr,
+                              workspace, workspace_bytes, static_cast<cudaStream_t>(stream), &pool);
 }
 
 }  // extern "C"

@@ -74,12 +74,20 @@ int launch_gated_rmsnorm(const void *o, const void *z, const float *w, float eps
 int launch_decode(const void *x, const void *conv_w, void *conv_state, const void *a, const void *b,
                   const float *A_log, const float *dt_bias, float scale, int hk, int hv,
                   float *state, const int32_t *slot, int n_slots, void *o, int batch, cudaStream_t s);
+// pool of states for gdr_chunk_prefill_slots (see PrefillParams)
+struct PrefillPool {
+  float *pool;
+  int n_slots;
+  const int32_t *slot;
+  int init_from_pool;
+};
 int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_stride,
                          int64_t v_stride, const void *a, const void *b,
                          const float *A_log, const float *dt_bias, float scale, int hk, int hv,
                          const int32_t *cu_dev, const int32_t *cu_host, int n_seqs, int total, int max_chunks,
                          const float *h0, float *hT, void *o, const void *z, const float *norm_w,
-                         float eps, void *y, void *workspace, size_t ws_bytes, cudaStream_t s);
+                         float eps, void *y, void *workspace, size_t ws_bytes, cudaStream_t s,
+                         const PrefillPool *pool = nullptr);
 size_t chunk_prefill_workspace_bytes(int n_seqs, int hv, int window_chunks, bool need_carry);
 
 // Conv output of `total` tokens of `channels` bf16 kept in the workspace when the conv is

@@ -156,6 +156,15 @@ struct PrefillParams {
   int win_chunks;       // chunks per window (record stride)
   const float *state_in;
   float *state_out;
+  // state pool (gdr_chunk_prefill_slots): sequence n's state lives in entry slot[n] of
+  // `pool`; a slot outside [0, n_slots) is a sequence that starts from zero and keeps
+  // nothing (its state crosses windows in `carry`)
+  const int32_t *slot;   // null: the states are state_in / state_out, indexed by sequence
+  int n_slots;
+  int pool_init;         // 1: the first window reads the entry, 0: it starts from zero
+  float *pool;
+  float *carry;
+  int last_window;
   uint16_t *o;          // may be null when y is set
   // gated RMSNorm fused into the output (y != null): y = o / sqrt(mean o^2 + eps) w SiLU(z)
   const uint16_t *z;
@@ -847,12 +856,30 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
   // ---- the state: row `row`, columns 32 ch .. 32 ch + 31 of this dv slice --------------
   float hreg[32];
-  const size_t srow = (static_cast<size_t>(n) * p.hv + h) * D * D + static_cast<size_t>(row) * D + slice * N + 32 * ch;
+  // where this sequence's state comes from and goes to
+  const float *state_in = p.state_in;
+  float *state_out = p.state_out;
+  size_t sidx = n;
+  if (p.slot) {
+    const int e = __ldg(p.slot + n);
+    if (e >= 0 && e < p.n_slots) {   // a pool entry, updated in place window by window
+      sidx = static_cast<size_t>(e);
+      state_in = (p.win0 == 0 && !p.pool_init) ? nullptr : p.pool;
+      state_out = p.pool;
+    } else {                         // no entry: from zero, through the workspace carry, dropped
+      state_in = p.win0 == 0 ? nullptr : p.carry;
+      state_out = p.last_window ? nullptr : p.carry;
+    }
+  }
+  const size_t srow = (sidx * p.hv + h) * D * D + static_cast<size_t>(row) * D + slice * N + 32 * ch;
+  const size_t crow = (static_cast<size_t>(n) * p.hv + h) * D * D + static_cast<size_t>(row) * D + slice * N + 32 * ch;
+  const size_t in_row = (p.slot && state_in == p.carry) ? crow : srow;
+  const size_t out_row = (p.slot && state_out == p.carry) ? crow : srow;
   if (!ctrl) {
-    if (p.state_in) {
+    if (state_in) {
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {
-        const float4 v4 = *reinterpret_cast<const float4 *>(p.state_in + srow + j);
+        const float4 v4 = *reinterpret_cast<const float4 *>(state_in + in_row + j);
         hreg[j] = v4.x; hreg[j + 1] = v4.y; hreg[j + 2] = v4.z; hreg[j + 3] = v4.w;
       }
     } else {
@@ -1172,10 +1199,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   if (kNorm) cluster_sync_all();   // no remote arrivals target a CTA that has left
   tc_fence_before();
   __syncthreads();
-  if (!ctrl && p.state_out && *abort_flag == 0u) {
+  if (!ctrl && state_out && *abort_flag == 0u) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4)
-      *reinterpret_cast<float4 *>(p.state_out + srow + j) = make_float4(hreg[j], hreg[j + 1], hreg[j + 2], hreg[j + 3]);
+      *reinterpret_cast<float4 *>(state_out + out_row + j) = make_float4(hreg[j], hreg[j + 1], hreg[j + 2], hreg[j + 3]);
   }
   if (warp == 0) tmem_dealloc(tmem, C_TM_COLS);
 }
@@ -1229,12 +1256,13 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
                          const float *A_log, const float *dt_bias, float scale, int hk, int hv,
                          const int32_t *cu_dev, const int32_t *cu_host, int n_seqs, int total, int max_chunks,
                          const float *h0, float *hT, void *o, const void *z, const float *norm_w,
-                         float eps, void *y, void *workspace, size_t ws_bytes, cudaStream_t s) {
+                         float eps, void *y, void *workspace, size_t ws_bytes, cudaStream_t s,
+                         const PrefillPool *pool) {
   if (n_seqs > 65535 || hv > 65535) return GDR_ERR_SHAPE;
   int st = ensure_smem_attrs();
   if (st) return st;
-  // window: as many chunks as the workspace holds (the state crosses windows
-  // in hT, or in the workspace tail when the caller wants no final state)
+  // window: as many chunks as the workspace holds; the state crosses windows in hT, in the pool entries, or in the workspace tail (no final
+  // state asked for, or sequences of a pooled call that have no entry)
   const bool carry_in_ws = hT == nullptr;
   const size_t rec_per_chunk = static_cast<size_t>(n_seqs) * hv * WS_REC;
   const size_t carry = carry_in_ws ? chunk_prefill_workspace_bytes(n_seqs, hv, 0, true) : 0;
@@ -1250,6 +1278,7 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   const uint64_t rows = total > 0 ? static_cast<uint64_t>(total) : 1;
   // with no tokens no tile is ever loaded; any aligned device address serves as a base
   const void *any = v ? v : (hT ? static_cast<const void *>(hT) : static_cast<const void *>(h0));
+  if (!any && pool) any = pool->pool;
   if (!any) return GDR_OK;
   if (!tensor_map_encoder()) return launch_status(cudaErrorSymbolNotFound, "prefill: cuTensorMapEncodeTiled lookup");
   if (!make_map(&tq, q ? q : any, static_cast<uint64_t>(hk) * D, rows, static_cast<uint64_t>(qk_stride)) ||
@@ -1277,12 +1306,18 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   p.eps = eps;
   p.y = static_cast<uint16_t *>(y);
   p.err = device_error_ptr();
+  p.slot = pool ? pool->slot : nullptr;
+  p.n_slots = pool ? pool->n_slots : 0;
+  p.pool_init = pool ? pool->init_from_pool : 0;
+  p.pool = pool ? pool->pool : nullptr;
+  p.carry = carry_buf;
   const int n_windows = max_chunks > 0 ? (max_chunks + win - 1) / win : 1;
   for (int w = 0; w < n_windows; ++w) {
     p.win0 = w * win;
     const bool first = w == 0, last = w == n_windows - 1;
     p.state_in = first ? h0 : (carry_in_ws ? carry_buf : hT);
     p.state_out = last ? hT : (carry_in_ws ? carry_buf : hT);
+    p.last_window = last ? 1 : 0;
     const int nc = std::min(win, max_chunks - p.win0);
     if (nc > 0) {
       st = launch_status(launch_pdl(prep_kernel, dim3(nc, hv, n_seqs), dim3(kPrepThreads), P_SMEM, s, 1, tq, tk, tv, p),

@@ -367,3 +367,25 @@ def varlen8_lengths(seed=4):
 def workload_full_varlen8(seed=4):
     """8 packed sequences, lengths U{1024..32768}, h0 ~ N(0,0.02), full path."""
     return make_full_inputs(seed + 1000, varlen8_lengths(seed), h0_std=0.02)
+
+
+@dataclasses.dataclass
+class MixedServing:
+    """One mixed serving step on a pool of cached states: new requests prefilled into free
+    entries of the pool, running requests decoding one token from theirs."""
+    prefill: CoreInputs       # the new requests' recurrence inputs (packed, varlen)
+    new_slot: np.ndarray      # [n_new] int32 entries the new requests fill
+    decode_slot: np.ndarray   # [rows] int32 entries of the running requests
+    n_slots: int
+
+
+def workload_mixed_serving(seed=5, n_new=4, rows=64, n_slots=128):
+    """4 new requests of U{256..4096} tokens (recurrence inputs, q/k not normalised) into free
+    entries of a 128-entry pool, beside the 64 running rows of decode_B64 (their entries: the
+    same seeded half of the pool as make_slot_table(7, 64, 128))."""
+    decode_slot = make_slot_table(7, rows, n_slots)
+    free = np.setdiff1d(np.arange(n_slots, dtype=np.int32), decode_slot)
+    new_slot = _rng(seed).permutation(free)[:n_new].astype(np.int32)
+    lengths = varlen_lengths(seed, n_new, 256, 4096)
+    return MixedServing(make_core_inputs(seed + 1000, lengths, prenorm_qk=False), new_slot,
+                        decode_slot, n_slots)

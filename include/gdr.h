@@ -75,7 +75,8 @@ GDR_API const char *gdr_status_string(int status);
 
 /* ABI version of this header, bumped whenever a signature or what a call does
  * changes (2: the conv fused into gdr_chunk_prefill,
- * gdr_chunk_prefill_fused_workspace_size; 3: gdr_decode_step_slots). */
+ * gdr_chunk_prefill_fused_workspace_size; 3: gdr_decode_step_slots; 4:
+ * gdr_chunk_prefill_slots). */
 GDR_API int gdr_abi_version(void);
 
 /*
@@ -295,6 +296,43 @@ GDR_API int gdr_decode_step_slots(const void *x, const void *conv_w, void *conv_
                                   const void *b, const float *A_log, const float *dt_bias, float scale,
                                   int hk, int hv, float *state_pool, int n_slots, const int32_t *slot,
                                   void *o, int batch, void *stream);
+
+/*
+ * gdr_chunk_prefill_slots -- gdr_chunk_prefill on a pool of cached states
+ * ("33B 只做 18 层 ...", §1.2: each request's recurrent state lives in a
+ * per-layer cache; a prompt fills it and later calls resume from it).
+ * Sequence n reads its initial state from, and writes its final state to,
+ * entry slot[n] of state_pool, in place.  With the decode's pool form this
+ * serves mixed batches: new requests are prefilled into their entries and
+ * running ones decode from theirs, all on one pool.
+ *   q, k, v, strides, a, b, A_log, dt_bias, scale, hk, hv, cu_seqlens, o:
+ *                 as gdr_chunk_prefill (no fusion)
+ *   state_pool:   fp32 [n_slots][hv][128][128], in/out
+ *   slot:         int32 [n_seqs], DEVICE memory, 4-byte aligned; read by the
+ *                 kernels, so it may be written by earlier work on the stream
+ *   init_from_pool: 1 = a sequence starts from its entry's state (a prompt
+ *                 continued in a later call), 0 = from zero (a new request);
+ *                 the entry is overwritten with the final state either way
+ *   workspace:    at least gdr_chunk_prefill_workspace_size(n_seqs, hv, 1, 0)
+ *                 bytes (the form without a final state: sequences without an
+ *                 entry carry their state through the workspace)
+ * A slot outside [0, n_slots) (e.g. -1) marks a sequence without an entry: it
+ * starts from zero, its o rows are written, and its final state is dropped.
+ * An empty sequence with an entry leaves it as it was (init_from_pool = 1) or
+ * sets it to zero (0).  The arithmetic is gdr_chunk_prefill's, so o and the
+ * final states equal that call's on the same initial states bit for bit.  Two
+ * sequences naming the same entry in one call race (every access stays inside
+ * the pool).  Returns GDR_ERR_NULL for a NULL slot array, a NULL pool with
+ * n_slots > 0 or a NULL input with tokens to process, GDR_ERR_SHAPE for a
+ * negative n_slots or init_from_pool not 0 or 1, GDR_ERR_WORKSPACE for a
+ * workspace below the size above.
+ */
+GDR_API int gdr_chunk_prefill_slots(const void *q, const void *k, const void *v, int64_t qk_token_stride,
+                                    int64_t v_token_stride, const void *a, const void *b, const float *A_log,
+                                    const float *dt_bias, float scale, int hk, int hv,
+                                    const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int n_seqs,
+                                    float *state_pool, int n_slots, const int32_t *slot, int init_from_pool,
+                                    void *o, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * gdr_gated_rmsnorm -- gated RMSNorm over rows of d values

@@ -44,7 +44,7 @@ def test_status_strings(L):
     for code in range(1, 10):
         assert G.status_string(code).startswith("GDR_ERR_")
     assert "UNKNOWN" in G.status_string(12345)
-    assert L.gdr_abi_version() == 3
+    assert L.gdr_abi_version() == 4
 
 
 @pytest.mark.parametrize("lengths", [[0], [1], [64], [65, 0, 128, 1, 63], [5000, 3, 64 * 7 + 1],
@@ -169,6 +169,29 @@ def test_wait_self_test_rejects_bad_arguments(L):
     assert L.gdr_debug_wait_timeout(0, 0, FAKE, None) == 2           # no bound
     assert L.gdr_debug_wait_timeout(0, 1 << 40, FAKE, None) == 2     # bound above 2^31
     assert L.gdr_debug_wait_timeout(0, 10, None, None) == 1          # no result word
+
+
+def test_prefill_slots_rejects_bad_arguments_on_host(L):
+    f = L.gdr_chunk_prefill_slots
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 2 + [ctypes.c_void_p] * 4 + [
+        ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_size_t, ctypes.c_void_p]
+    cu, cup = _cu([70, 5])
+    ws = L.gdr_chunk_prefill_workspace_size(2, 48, 1, 0)
+
+    def call(slot=FAKE, pool=FAKE, n_slots=4, init=0, hv=48, wsb=ws, q=FAKE):
+        return f(q, FAKE, FAKE, 0, 0, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(1.0), 16, hv, FAKE, cup, 2,
+                 pool, n_slots, slot, init, FAKE, FAKE, wsb, None)
+    assert call(slot=None) == 1                   # no slot array
+    assert call(pool=None) == 1                   # entries without a pool
+    assert call(q=None) == 1                      # tokens without inputs
+    assert call(n_slots=-1) == 2
+    assert call(init=2) == 2
+    assert call(hv=50) == 5                       # grouping not supported
+    assert call(slot=FAKE + 2) == 3               # slot array not 4-byte aligned
+    assert call(wsb=ws - 16) == 6                 # workspace below one window plus the carry
+    assert ws == L.gdr_chunk_prefill_workspace_size(2, 48, 1, 1) + 2 * 48 * 128 * 128 * 4
 
 
 def test_other_entry_points_reject_bad_arguments(L):

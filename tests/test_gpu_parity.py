@@ -234,6 +234,95 @@ def test_decode_slots_match_oracle_and_plain_decode():
 # chunked prefill
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("window", [None, 1])
+def test_prefill_into_pool_entries_then_decode_from_the_pool(window):
+    """Mixed serving batch on one pool of cached states: new requests are prefilled into their
+    entries (from zero), a sequence without an entry keeps nothing, a second call continues two
+    entries from their states, then one decode step runs rows on prefilled and pre-existing
+    entries.  Against the oracle (recurrence from the entries' states, decode on the pool) and
+    bit for bit against the plain prefill on the same initial states; entries no call names
+    stay unchanged bit for bit.  window=1 makes every sequence cross windows (pool entries in
+    place, the entry-less sequence through the workspace carry)."""
+    S, hv = 6, 48
+    r = np.random.default_rng(57)
+    pool0 = (r.standard_normal((S, hv, 128, 128)) * 0.02).astype(np.float32)
+    pool = dev_f32(pool0)
+    # call 1: lengths 70, 0, 5, 130 into entries 4, 1, none, 2, from zero
+    inp = GI.make_core_inputs(94, [70, 0, 5, 130], prenorm_qk=False)
+    slot1 = np.array([4, 1, -1, 2], np.int32)
+    args = (dev_bf16(inp.q), dev_bf16(inp.k), dev_bf16(inp.v), dev_bf16(inp.a), dev_bf16(inp.b),
+            dev_f32(inp.A_log), dev_f32(inp.dt_bias), dev_i32(inp.cu_seqlens), inp.cu_seqlens)
+    ws = (G.prefill_workspace(inp.cu_seqlens, hv, "cuda", window=window, has_final_state=False)
+          if window else None)
+    o1 = G.chunk_prefill_slots(*args, pool, dev_i32(slot1), init_from_pool=False, workspace=ws)
+    torch.cuda.synchronize()
+    assert G.get_device_error() == 0
+    ref_bits, _, ref_h = O.core_path(inp)                  # from zero states
+    got = pool.cpu().numpy()
+    cu = inp.cu_seqlens
+    o1b = host_bits(o1)
+    for n in range(4):
+        s_, e_ = int(cu[n]), int(cu[n + 1])
+        if e_ > s_:
+            assert rel_l2(bits_f64(o1b[s_:e_]), bits_f64(ref_bits[s_:e_])) <= TOL_BF16, n
+    for n, e in ((0, 4), (3, 2)):
+        assert rel_l2(got[e], ref_h[n]) <= TOL_STATE, n
+    assert not got[1].any()                                 # an empty new request: zero state
+    for e in (0, 3, 5):                                     # entries no sequence names
+        assert np.array_equal(got[e], pool0[e]), e
+    # bit for bit the plain prefill from zero states
+    hT = torch.empty((4, hv, 128, 128), device="cuda")
+    o_plain = G.chunk_prefill(*args, hT=hT)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(o_plain), o1b)
+    hTn = hT.cpu().numpy()
+    assert np.array_equal(got[4], hTn[0]) and np.array_equal(got[2], hTn[3])
+
+    # call 2: continue entries 4 and 0 from their states (lengths 64, 33)
+    inp2 = GI.make_core_inputs(95, [64, 33], prenorm_qk=False)
+    slot2 = np.array([4, 0], np.int32)
+    before = pool.cpu().numpy()
+    inp2.h0 = np.ascontiguousarray(before[slot2])
+    args2 = (dev_bf16(inp2.q), dev_bf16(inp2.k), dev_bf16(inp2.v), dev_bf16(inp2.a), dev_bf16(inp2.b),
+             dev_f32(inp2.A_log), dev_f32(inp2.dt_bias), dev_i32(inp2.cu_seqlens), inp2.cu_seqlens)
+    ws2 = (G.prefill_workspace(inp2.cu_seqlens, hv, "cuda", window=window, has_final_state=False)
+           if window else None)
+    o2 = G.chunk_prefill_slots(*args2, pool, dev_i32(slot2), init_from_pool=True, workspace=ws2)
+    torch.cuda.synchronize()
+    assert G.get_device_error() == 0
+    ref2_bits, _, ref2_h = O.core_path(inp2)
+    got2 = pool.cpu().numpy()
+    o2b = host_bits(o2)
+    for n in range(2):
+        s_, e_ = int(inp2.cu_seqlens[n]), int(inp2.cu_seqlens[n + 1])
+        assert rel_l2(bits_f64(o2b[s_:e_]), bits_f64(ref2_bits[s_:e_])) <= TOL_BF16, n
+        assert rel_l2(got2[slot2[n]], ref2_h[n]) <= TOL_STATE, n
+    for e in (1, 2, 3, 5):
+        assert np.array_equal(got2[e], before[e]), e
+
+    # one decode step on rows naming a prefilled entry (2), a continued one (4), an untouched
+    # one (5) and a padding row, from the same pool
+    dec = GI.make_decode_inputs(96, 4, 1)
+    slot3 = np.array([2, 4, 5, -1], np.int32)
+    C = dec.x.shape[2]
+    cpool0 = GI.f32_to_bf16_bits(r.standard_normal((S, 3, C)).astype(np.float32))
+    cp_d = dev_bf16(cpool0)
+    od = torch.full((4, hv, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    G.decode_step_slots(dev_bf16(dec.x[0]), dev_bf16(dec.conv_w), cp_d, dev_bf16(dec.a[0]), dev_bf16(dec.b[0]),
+                        dev_f32(dec.A_log), dev_f32(dec.dt_bias), pool, dev_i32(slot3), o=od)
+    torch.cuda.synchronize()
+    o_ref, _, sp_ref = O.decode_step_slots(dec.x[0], dec.a[0], dec.b[0], dec.conv_w, dec.A_log, dec.dt_bias,
+                                           O.bf16_to_f64(cpool0), got2.astype(np.float64), slot3, dec.hk, dec.hv)
+    odb = host_bits(od)
+    assert rel_l2(bits_f64(odb[:3]), bits_f64(o_ref[:3])) <= TOL_BF16
+    assert not odb[3].any()
+    got3 = pool.cpu().numpy()
+    for e in (2, 4, 5):
+        assert rel_l2(got3[e], sp_ref[e]) <= TOL_STATE, e
+    for e in (0, 1, 3):
+        assert np.array_equal(got3[e], got2[e]), e
+
+
 @pytest.mark.parametrize("lengths", [[1], [63], [64], [65], [200], [1, 64, 65, 0, 130, 3]])
 def test_prefill_lengths_and_varlen(lengths):
     inp = GI.make_core_inputs(60 + len(lengths), lengths, prenorm_qk=False, h0_std=0.02)

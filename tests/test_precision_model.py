@@ -11,7 +11,11 @@ B200 kernels measure 3-5e-6.  Against the oracle: the scheme keeps every head's 
 state well inside the layer's 1e-4 bar; dropping the lo part of U' breaks the bar
 everywhere, and dropping one of the three terms of W H0 breaks it on the heads that decay
 slowest (their initial state persists through the sequence).  A 128-token chunk keeps the
-same accuracy.  The model is test scaffolding: it does not run on the GPU and shares no
+same accuracy.  The output side, o = e^gamma/|q| Q H0 + Mq U, keeps hi*hi + hi*lo + lo*hi
+in Mq U as well: o's bound (2e-3 on the bf16 output) is twenty times looser than the
+state's, but dropping either lo term of Mq U puts o at 2.6-2.7e-3; dropping H0's lo part
+from Q H0 stays inside (1.1e-3 with an initial state) but saves no work, since Q rides in
+the same tensor-core product as W's rows, which need it.  The model is test scaffolding: it does not run on the GPU and shares no
 code with the kernels or the oracle.
 """
 import numpy as np
@@ -20,7 +24,7 @@ import torch
 
 import gdr_inputs as GI
 from oracle import oracle as O
-from tests.helpers import TOL_STATE
+from tests.helpers import TOL_BF16, TOL_STATE
 
 
 def _bf16(x):
@@ -134,3 +138,72 @@ def test_two_term_w_h0_breaks_the_bar_on_slowly_decaying_heads(short):
 
 def test_a_128_token_chunk_is_as_accurate(long):
     assert _state_error(long, HEADS, chunk=128) < 0.1 * TOL_STATE
+
+
+def _output_model(inp, heads, mq_lo=True, u_lo=True, qh_lo=True, chunk=64):
+    """o [T, len(heads), 128] of the chunked form under the split-operand arithmetic (the state
+    path as in _state_model, three-term W H0, U' with its lo part)."""
+    q_heads = inp.q.shape[1]
+    q = O.bf16_to_f64(inp.q).astype(np.float32)
+    k = O.bf16_to_f64(inp.k).astype(np.float32)
+    v = O.bf16_to_f64(inp.v).astype(np.float32)
+    g, beta = O.gates(O.bf16_to_f64(inp.a), O.bf16_to_f64(inp.b), inp.A_log, inp.dt_bias)
+    g, beta = g.astype(np.float32), beta.astype(np.float32)
+    hv = v.shape[1]
+    cu = inp.cu_seqlens
+    o = np.zeros((inp.T, len(heads), 128), np.float32)
+    for n in range(len(cu) - 1):
+        for col, h in enumerate(heads):
+            kh = h // (hv // q_heads)
+            H = np.zeros((128, 128), np.float32) if inp.h0 is None else inp.h0[n, h].astype(np.float32)
+            for s in range(int(cu[n]), int(cu[n + 1]), chunk):
+                e = min(s + chunk, int(cu[n + 1]))
+                K, V, Q = k[s:e, kh], v[s:e, h], q[s:e, kh]
+                rk = (1.0 / np.sqrt((K * K).sum(1) + 1e-6)).astype(np.float32)
+                rq = (1.0 / np.sqrt((Q * Q).sum(1) + 1e-6)).astype(np.float32)
+                gam = np.cumsum(g[s:e, h]).astype(np.float32)
+                bt = beta[s:e, h]
+                decay = np.exp(np.minimum(gam[:, None] - gam[None, :], 0.0))
+                Kn = K * rk[:, None]
+                A = np.tril(bt[:, None] * decay * (Kn @ Kn.T), -1).astype(np.float32)
+                T = np.linalg.inv(np.eye(e - s, dtype=np.float32) + A).astype(np.float32)
+                Tw_hi, Tw_lo = _split(T * (bt * np.exp(gam) * rk)[None, :])
+                Tu_hi, Tu_lo = _split(T * bt[None, :])
+                W = _mm(Tw_hi, K) + _mm(Tw_lo, K)
+                Ut = _mm(Tu_hi, V) + _mm(Tu_lo, V)
+                W_hi, W_lo = _split(W)
+                H_hi, H_lo = _split(H)
+                U = (Ut - (_mm(W_hi, H_hi) + _mm(W_hi, H_lo) + _mm(W_lo, H_hi))).astype(np.float32)
+                # Mq = (Q K^T) e^(gamma_i - gamma_j) / (|q_i| |k_j|), j <= i; raw Q exact
+                Mq = (np.tril(_mm(Q, K.T) * decay) * rq[:, None] * rk[None, :]).astype(np.float32)
+                Mq_hi, Mq_lo = _split(Mq)
+                U_hi, U_lo = _split(U)
+                MU = _mm(Mq_hi, U_hi)
+                if u_lo:
+                    MU = MU + _mm(Mq_hi, U_lo)
+                if mq_lo:
+                    MU = MU + _mm(Mq_lo, U_hi)
+                QH = _mm(Q, H_hi) + (_mm(Q, H_lo) if qh_lo else 0.0)
+                o[s:e, col] = (np.exp(gam) * rq)[:, None] * QH + MU
+                Us_hi, Us_lo = _split(U * (np.exp(gam[-1] - gam) * rk)[:, None])
+                H = (np.exp(gam[-1]) * H + _mm(K.T, Us_hi) + _mm(K.T, Us_lo)).astype(np.float32)
+    return o
+
+
+def _output_error(inp, heads, **kw):
+    """rel-L2 of the model's bf16 o against the oracle's bf16 o (what the GPU tests compare)."""
+    bits, _, _ = O.core_path(inp, heads=heads)
+    ref = O.bf16_to_f64(bits)[:, heads]
+    got = O.bf16_to_f64(O.round_bf16(_output_model(inp, heads, **kw).astype(np.float64)))
+    return float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+
+
+def test_the_output_needs_both_lo_terms_of_mq_u(short):
+    assert _output_error(short, HEADS) < 0.15 * TOL_BF16
+    assert _output_error(short, HEADS, mq_lo=False) > TOL_BF16
+    assert _output_error(short, HEADS, u_lo=False) > TOL_BF16
+
+
+def test_q_h0_without_its_lo_part_stays_inside_the_bar_but_uses_half_of_it(short):
+    e = _output_error(short, HEADS, qh_lo=False)
+    assert 0.4 * TOL_BF16 < e < TOL_BF16

@@ -238,7 +238,7 @@ def prefill_workspace(cu_seqlens_host, hv: int, device, window: Optional[int] = 
 
 def prefill_fused_workspace(cu_seqlens_host, hk: int, hv: int, device, window: Optional[int] = None,
                             has_final_state: bool = True):
-    """Workspace for gdr_chunk_prefill with the conv fused: the conv output, then the records."""
+    """Workspace for gdr_chunk_prefill running the conv in the same call: the conv output, then the records."""
     torch = _torch()
     cu = np.asarray(cu_seqlens_host)
     n = len(cu) - 1
@@ -256,7 +256,7 @@ def chunk_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, cu_seqlens_host, h0
     """Chunk-64 prefill.  q, k [T, hk, 128], v [T, hv, 128], a, b [T, hv] bf16.
 
     q, k, v may be token-strided views (e.g. slices of the [T, q|k|v] conv output); with the
-    conv fused (``fuse`` holding "x", "conv_w" and "hk") they are None.
+    conv run by the same call (``fuse`` holding "x", "conv_w" and "hk") they are None.
 
     Returns o [T, hv, 128] bf16 (and writes hT [N, hv, 128, 128] fp32 when given).
     ``fuse`` (optional) maps gdr_prefill_fuse_t field names to tensors.

@@ -118,21 +118,27 @@ GDR_API int gdr_causal_conv(const void *x, const void *w, const void *conv_state
                     int channels, void *y, void *stream);
 
 /*
- * Optional fusion around the prefill (pass NULL to gdr_chunk_prefill to run
+ * Optional work around the prefill (pass NULL to gdr_chunk_prefill to run
  * the recurrence alone).
- *  - Gated RMSNorm (`z` set): y receives o / sqrt(mean(o^2) + eps) * w * SiLU(z)
- *    row by row, computed from the bf16-rounded o inside the prefill (the two
- *    64-column halves of a head run as a thread-block cluster and exchange their
- *    row sums of squares); o is written as well only when gdr_chunk_prefill's o
- *    is not NULL.  y must not overlap o (GDR_ERR_ALIAS).
- *  - Conv (`x` set): the call runs the causal conv of gdr_causal_conv on x
- *    (with conv_w and the optional conv states) into the head of the
- *    workspace and reads q, k, v from that output; q, k and v must then be
- *    NULL (GDR_ERR_SHAPE otherwise) and the workspace must hold
- *    gdr_chunk_prefill_fused_workspace_size(...) bytes.  conv_state_out
- *    receives the last three inputs of every sequence (empty ones included),
- *    as from gdr_causal_conv.  The results equal the separate calls bit for
- *    bit: the same kernels run, one after the other on the stream.
+ *  - Gated RMSNorm (`z` set), a fusion: y receives o / sqrt(mean(o^2) + eps) *
+ *    w * SiLU(z) row by row, computed from the bf16-rounded o inside the
+ *    prefill's state kernel (the two 64-column halves of a head run as a
+ *    thread-block cluster and exchange their row sums of squares), so o need not
+ *    go through memory; o is written as well only when gdr_chunk_prefill's o is
+ *    not NULL.  y must not overlap o (GDR_ERR_ALIAS).  It saves the o round
+ *    trip but lengthens the state kernel's per-chunk path, and at one sequence
+ *    it runs slower than the separate gdr_gated_rmsnorm call.
+ *  - Conv (`x` set), a convenience, not a fusion: the call runs the kernel of
+ *    gdr_causal_conv on x (with conv_w and the optional conv states) into the
+ *    head of the workspace and the prefill reads q, k, v from there, so the
+ *    caller needs no conv output buffer.  The conv output is still written to
+ *    and read back from device memory: the bytes moved are those of the two
+ *    separate calls.  q, k and v must then be NULL (GDR_ERR_SHAPE otherwise)
+ *    and the workspace must hold gdr_chunk_prefill_fused_workspace_size(...)
+ *    bytes.  conv_state_out receives the last three inputs of every sequence
+ *    (empty ones included), as from gdr_causal_conv.  The results equal the
+ *    separate calls bit for bit: the same kernels run, one after the other on
+ *    the stream.
  */
 typedef struct gdr_prefill_fuse {
   const void *x;             /* bf16 [T][hk*128*2 + hv*128] conv input, or NULL */

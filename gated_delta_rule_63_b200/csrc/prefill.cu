@@ -36,6 +36,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 
 #include "gdr_common.cuh"
 #include "gdr_host.h"
@@ -1243,6 +1244,51 @@ int ensure_smem_attrs() {
   return GDR_OK;
 }
 
+// ---- pipelined windows -------------------------------------------------------
+// When the chains of a call leave SMs idle (fewer than one chain CTA per SM) and the
+// sequences span several windows, the prep of window w + 1 runs beside the chain of
+// window w: chains on a high-priority stream, preps on a low-priority one, records in two
+// buffers used alternately.  The prep CTAs take the SMs the chains leave free and spread
+// to all of them once a chain window ends.  Both streams belong to the library (one pair
+// per device), fork from the caller's stream and join it again before the call returns,
+// so stream order and graph capture see one piece of work.
+constexpr int kPipeMinChunks = 16;   // below this the extra chain start-ups cost more than the overlap
+constexpr int kPipeEvents = 64;
+
+struct PipeStreams {
+  cudaStream_t hi = nullptr, lo = nullptr;
+  cudaEvent_t ev[kPipeEvents] = {};
+  int next = 0;
+  int sms = 0;
+  std::mutex lock;   // one call at a time issues on a device's pair
+};
+
+int pipe_streams(PipeStreams **out) {
+  static PipeStreams per_dev[64];
+  static std::mutex init_lock;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return launch_status(e, "prefill: cudaGetDevice");
+  if (dev < 0 || dev >= 64) return GDR_ERR_UNSUPPORTED;
+  PipeStreams &ps = per_dev[dev];
+  std::lock_guard<std::mutex> g(init_lock);
+  if (!ps.hi) {
+    int least = 0, greatest = 0;
+    cudaStream_t hi = nullptr, lo = nullptr;
+    e = cudaDeviceGetAttribute(&ps.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&hi, cudaStreamNonBlocking, greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&lo, cudaStreamNonBlocking, least);
+    for (int i = 0; i < kPipeEvents && e == cudaSuccess; ++i)
+      e = cudaEventCreateWithFlags(&ps.ev[i], cudaEventDisableTiming);
+    if (e != cudaSuccess) return launch_status(e, "prefill: pipeline streams");
+    ps.lo = lo;
+    ps.hi = hi;
+  }
+  *out = &ps;
+  return GDR_OK;
+}
+
 }  // namespace
 
 size_t chunk_prefill_workspace_bytes(int n_seqs, int hv, int window_chunks, bool need_carry) {
@@ -1271,8 +1317,23 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   if (max_chunks > 0)
     win = static_cast<int>(std::min<size_t>((ws_bytes - carry) / rec_per_chunk, static_cast<size_t>(max_chunks)));
   if (win > 65535) win = 65535;
+  // pipelined windows (see PipeStreams): two record buffers of `win2` chunks each
+  PipeStreams *ps = nullptr;
+  bool pipelined = false;
+  if (max_chunks > 2 * kPipeMinChunks) {
+    const size_t fit2 = (ws_bytes - carry) / (2 * rec_per_chunk);
+    if (fit2 >= static_cast<size_t>(kPipeMinChunks) && max_chunks > win) {
+      st = pipe_streams(&ps);
+      if (st) return st;
+      if (static_cast<long long>(n_seqs) * hv * NS < ps->sms) {
+        win = static_cast<int>(std::min<size_t>({fit2, static_cast<size_t>(max_chunks), size_t{65535}}));
+        pipelined = (max_chunks + win - 1) / win >= 3;
+      }
+    }
+  }
+  const size_t buf_bytes = rec_per_chunk * win;
   float *carry_buf = carry_in_ws && max_chunks > 0
-                         ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + rec_per_chunk * win)
+                         ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + buf_bytes * (pipelined ? 2 : 1))
                          : nullptr;
   CUtensorMap tq, tk, tv;
   const uint64_t rows = total > 0 ? static_cast<uint64_t>(total) : 1;
@@ -1312,28 +1373,64 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   p.pool = pool ? pool->pool : nullptr;
   p.carry = carry_buf;
   const int n_windows = max_chunks > 0 ? (max_chunks + win - 1) / win : 1;
-  for (int w = 0; w < n_windows; ++w) {
-    p.win0 = w * win;
+  auto window_params = [&](int w) {
+    PrefillParams pw = p;
+    pw.win0 = w * win;
     const bool first = w == 0, last = w == n_windows - 1;
-    p.state_in = first ? h0 : (carry_in_ws ? carry_buf : hT);
-    p.state_out = last ? hT : (carry_in_ws ? carry_buf : hT);
-    p.last_window = last ? 1 : 0;
-    const int nc = std::min(win, max_chunks - p.win0);
-    if (nc > 0) {
-      st = launch_status(launch_pdl(prep_kernel, dim3(nc, hv, n_seqs), dim3(kPrepThreads), P_SMEM, s, 1, tq, tk, tv, p),
+    pw.state_in = first ? h0 : (carry_in_ws ? carry_buf : hT);
+    pw.state_out = last ? hT : (carry_in_ws ? carry_buf : hT);
+    pw.last_window = last ? 1 : 0;
+    if (pipelined) pw.ws = static_cast<uint8_t *>(workspace) + (w & 1) * buf_bytes;
+    return pw;
+  };
+  auto launch_prep = [&](int w, cudaStream_t stream) -> int {
+    const PrefillParams pw = window_params(w);
+    const int nc = std::min(win, max_chunks - pw.win0);
+    if (nc <= 0) return GDR_OK;
+    return launch_status(launch_pdl(prep_kernel, dim3(nc, hv, n_seqs), dim3(kPrepThreads), P_SMEM, stream, 1, tq, tk,
+                                    tv, pw),
                          "prefill: prep kernel launch");
-      if (st) return st;
-    }
+  };
+  auto launch_chain = [&](int w, cudaStream_t stream) -> int {
+    const PrefillParams pw = window_params(w);
     // with the fused norm the two dv slices of a head form a cluster and exchange row sums
-    st = y ? launch_status(launch_pdl(chain_kernel<true>, dim3(NS, hv, n_seqs), dim3(kChainThreads), C_SMEM, s,
-                                      static_cast<unsigned>(NS), tq, tk, p),
-                           "prefill: chain kernel launch")
-           : launch_status(launch_pdl(chain_kernel<false>, dim3(NS, hv, n_seqs), dim3(kChainThreads), C_SMEM, s, 1,
-                                      tq, tk, p),
-                           "prefill: chain kernel launch");
-    if (st) return st;
+    return y ? launch_status(launch_pdl(chain_kernel<true>, dim3(NS, hv, n_seqs), dim3(kChainThreads), C_SMEM, stream,
+                                        static_cast<unsigned>(NS), tq, tk, pw),
+                             "prefill: chain kernel launch")
+             : launch_status(launch_pdl(chain_kernel<false>, dim3(NS, hv, n_seqs), dim3(kChainThreads), C_SMEM, stream,
+                                        1, tq, tk, pw),
+                             "prefill: chain kernel launch");
+  };
+  if (!pipelined) {
+    for (int w = 0; w < n_windows; ++w) {
+      if ((st = launch_prep(w, s)) || (st = launch_chain(w, s))) return st;
+    }
+    return GDR_OK;
   }
-  return GDR_OK;
+  // pipelined: chain w on `hi` after prep w; prep w + 1 on `lo` beside chain w, once chain
+  // w - 1 has released the buffer it reuses
+  std::lock_guard<std::mutex> g(ps->lock);
+  auto record = [&](cudaStream_t from, cudaEvent_t *e) -> int {   // mark `from`'s work so far
+    *e = ps->ev[ps->next];
+    ps->next = (ps->next + 1) % kPipeEvents;
+    return launch_status(cudaEventRecord(*e, from), "prefill: stream ordering");
+  };
+  auto wait = [&](cudaStream_t to, cudaEvent_t e) -> int {
+    return launch_status(cudaStreamWaitEvent(to, e, 0), "prefill: stream ordering");
+  };
+  cudaEvent_t e = nullptr, chain_prev = nullptr, chain_cur = nullptr;
+  if ((st = record(s, &e)) || (st = wait(ps->hi, e)) || (st = wait(ps->lo, e))) return st;
+  if ((st = launch_prep(0, ps->lo))) return st;
+  for (int w = 0; w < n_windows; ++w) {
+    if ((st = record(ps->lo, &e)) || (st = wait(ps->hi, e))) return st;   // prep w is done
+    if ((st = launch_chain(w, ps->hi)) || (st = record(ps->hi, &chain_cur))) return st;
+    if (w + 1 < n_windows) {
+      if (w >= 1 && (st = wait(ps->lo, chain_prev))) return st;   // chain w - 1 read the buffer
+      if ((st = launch_prep(w + 1, ps->lo))) return st;
+    }
+    chain_prev = chain_cur;
+  }
+  return wait(s, chain_prev);   // the last prep precedes the last chain
 }
 
 }  // namespace gdr

@@ -354,6 +354,38 @@ def test_prefill_windows_carry_state(window, final_state):
         assert rel_l2(hT.cpu().numpy(), ref_hT) <= TOL_STATE
 
 
+@pytest.mark.parametrize("final_state", [True, False])
+def test_prefill_pipelined_windows_equal_one_window(final_state):
+    """One sequence (96 chain CTAs: SMs left idle) over 41 chunks with a workspace for 32
+    chunks: the call runs three windows of 16 chunks on two record buffers, the prep of window
+    w + 1 beside the chain of window w on the library's own pair of streams, joined back to the
+    caller's stream.  o and the final state equal a one-window call's bit for bit (the state
+    crosses windows in fp32), and o matches the oracle on three heads."""
+    T = 64 * 40 + 17
+    inp = GI.make_core_inputs(97, [T], prenorm_qk=False, h0_std=0.02)
+    hv = inp.v.shape[1]
+    args = (dev_bf16(inp.q), dev_bf16(inp.k), dev_bf16(inp.v), dev_bf16(inp.a), dev_bf16(inp.b),
+            dev_f32(inp.A_log), dev_f32(inp.dt_bias), dev_i32(inp.cu_seqlens), inp.cu_seqlens)
+    h0 = dev_f32(inp.h0)
+    outs = []
+    for window in (None, 32):
+        hT = torch.full((1, hv, 128, 128), float("nan"), device="cuda") if final_state else None
+        ws = G.prefill_workspace(inp.cu_seqlens, hv, "cuda", window=window, has_final_state=final_state)
+        o = torch.full((T, hv, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+        G.chunk_prefill(*args, h0=h0, hT=hT, o=o, scale=inp.scale, workspace=ws)
+        torch.cuda.synchronize()
+        assert G.get_device_error() == 0
+        outs.append((host_bits(o), None if hT is None else hT.cpu().numpy()))
+    assert np.array_equal(outs[0][0], outs[1][0])
+    if final_state:
+        assert np.array_equal(outs[0][1], outs[1][1])
+    heads = [0, 25, 47]
+    ref_bits, _, ref_hT = O.core_path(inp, heads=heads)
+    assert rel_l2(bits_f64(outs[1][0][:, heads]), bits_f64(ref_bits[:, heads])) <= TOL_BF16
+    if final_state:
+        assert rel_l2(outs[1][1][:, heads], ref_hT[:, heads]) <= TOL_STATE
+
+
 @pytest.mark.parametrize("case", ["no_decay", "instant_decay", "no_write", "full_write"])
 def test_prefill_degenerate_gates(case):
     """Limits of the gates on the GPU path: g = 0 (exp(A_log) = 0), g far below zero (the

@@ -1251,7 +1251,8 @@ int ensure_smem_attrs() {
 // buffers used alternately.  The prep CTAs take the SMs the chains leave free and spread
 // to all of them once a chain window ends.  Both streams belong to the library (one pair
 // per device), fork from the caller's stream and join it again before the call returns,
-// so stream order and graph capture see one piece of work.
+// so the caller's stream order sees one piece of work.  A call whose stream is being
+// captured into a graph keeps the serial schedule.
 constexpr int kPipeMinChunks = 16;   // below this the extra chain start-ups cost more than the overlap
 constexpr int kPipeEvents = 64;
 
@@ -1320,7 +1321,14 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   // pipelined windows (see PipeStreams): two record buffers of `win2` chunks each
   PipeStreams *ps = nullptr;
   bool pipelined = false;
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
   if (max_chunks > 2 * kPipeMinChunks) {
+    const cudaError_t ce = cudaStreamIsCapturing(s, &capture);
+    if (ce != cudaSuccess) return launch_status(ce, "prefill: cudaStreamIsCapturing");
+  }
+  // (under stream capture the call keeps to the caller's stream: the library's streams are
+  // shared by all calls on the device and must not join one caller's graph)
+  if (max_chunks > 2 * kPipeMinChunks && capture == cudaStreamCaptureStatusNone) {
     const size_t fit2 = (ws_bytes - carry) / (2 * rec_per_chunk);
     if (fit2 >= static_cast<size_t>(kPipeMinChunks) && max_chunks > win) {
       st = pipe_streams(&ps);

@@ -179,6 +179,16 @@ typedef struct gdr_prefill_fuse {
  *             bytes (GDR_ERR_WORKSPACE otherwise); the window is the largest
  *             number of chunks that fits.
  * Empty sequences copy h0 (or zeros) to hT.
+ * Long sequences on a GPU that the state kernels leave partly idle (n_seqs *
+ * hv * 2 below the SM count, e.g. one sequence of 48 value heads): when the
+ * workspace holds two windows of at least 16 chunks and the sequences need at
+ * least three such windows, the call splits the workspace into two record
+ * buffers and builds window w + 1 while window w's state walk runs, on a pair
+ * of streams the library creates once per device (high and low priority).
+ * The work forks from `stream` and joins it before the call returns; the
+ * results equal the one-buffer schedule bit for bit.  Calls that pipeline on
+ * one device take turns issuing (a lock).  A call made while `stream` is
+ * being captured into a graph keeps the one-buffer schedule on `stream`.
  */
 GDR_API int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk_token_stride,
                               int64_t v_token_stride, const void *a, const void *b,

@@ -384,6 +384,21 @@ def test_prefill_pipelined_windows_equal_one_window(final_state):
     assert rel_l2(bits_f64(outs[1][0][:, heads]), bits_f64(ref_bits[:, heads])) <= TOL_BF16
     if final_state:
         assert rel_l2(outs[1][1][:, heads], ref_hT[:, heads]) <= TOL_STATE
+    # the same call captured into a graph keeps to the caller's stream (one buffer at a time)
+    # and replays the eager bits
+    hT = torch.empty((1, hv, 128, 128), device="cuda") if final_state else None
+    ws = G.prefill_workspace(inp.cu_seqlens, hv, "cuda", window=32, has_final_state=final_state)
+    o = torch.empty((T, hv, 128), dtype=torch.bfloat16, device="cuda")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        G.chunk_prefill(*args, h0=h0, hT=hT, o=o, scale=inp.scale, workspace=ws)
+    o.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert G.get_device_error() == 0
+    assert np.array_equal(host_bits(o), outs[0][0])
+    if final_state:
+        assert np.array_equal(hT.cpu().numpy(), outs[0][1])
 
 
 @pytest.mark.parametrize("case", ["no_decay", "instant_decay", "no_write", "full_write"])

@@ -401,7 +401,7 @@ def bench_mixed(torch, G, device, args, steps=20):
     n_new, rows = len(mix.new_slot), len(mix.decode_slot)
     pbytes = T * B_CORE + n_new * STATE_BYTES          # from zero: the entries are only written
     dbytes = rows * STATE_BYTES * 2
-    launches = 2 * n_windows(G, cu_host, hv) + 1
+    launches = 2 * n_windows(G, cu_host, hv, ws, False)[0] + 1
     return {"workload": f"mixed_serving: {n_new} new requests, lengths {[int(x) for x in np.diff(cu_host)]}, "
                         f"prefilled into free entries of a {mix.n_slots}-entry pool; {rows} running rows "
                         "decode one token from theirs (decode_B64 inputs)",
@@ -419,11 +419,10 @@ def bench_mixed(torch, G, device, args, steps=20):
             "steps": steps, "launches": (3 + steps) * launches}
 
 
-def n_windows(G, cu_host, hv):
-    """Chunk windows (each a prep and a chain launch) of one prefill call with the default workspace."""
-    longest = int(max(1, ((np.diff(np.asarray(cu_host, dtype=np.int64)) + 63) // 64).max()))
-    win = G.prefill_window(cu_host, hv)
-    return -(-longest // win)
+def n_windows(G, cu_host, hv, ws, has_final_state=True):
+    """Chunk windows (each a prep and a chain launch) of one prefill call on workspace `ws`, and
+    whether the call pipelines them (the library's own schedule query)."""
+    return G.prefill_schedule(cu_host, hv, ws.numel(), has_final_state)
 
 
 def bench_long_and_varlen(torch, G, device, reps=3):
@@ -460,13 +459,15 @@ def bench_long_and_varlen(torch, G, device, reps=3):
     o = torch.empty((T, hv, d), dtype=torch.bfloat16, device=device)
     hT = torch.empty((1, hv, d, d), dtype=torch.float32, device=device)
     ws = G.prefill_workspace(cu_host, hv, device)
-    launches = 2 * n_windows(G, cu_host, hv)
+    windows, pipelined = n_windows(G, cu_host, hv, ws)
+    launches = 2 * windows
     ms = timed(lambda: G.chunk_prefill(q, k, v, a, b, Al, db, cu, cu_host, hT=hT, o=o, workspace=ws))
     byts = T * B_CORE + STATE_BYTES
     out["long_context"] = {
         "workload": "core_T262144: B=1 T=262144, recurrence alone, zero initial state, final state out",
         "metric": METRIC_PREFILL, "value": T / (ms * 1e-3), "unit": "tokens/s", "ms": ms,
         "algorithmic_bytes": byts, "launches_per_call": launches,
+        "schedule": {"windows": windows, "pipelined": pipelined, "workspace_bytes": int(ws.numel())},
         "roofline": {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                      "frac": byts / (ms * 1e-3) / 1e9 / hbm_peak}}
     del q, k, v, a, b, o, hT, ws, inp
@@ -474,7 +475,7 @@ def bench_long_and_varlen(torch, G, device, reps=3):
     inp = GI.workload_full_varlen8()
     T, N = inp.T, inp.n_seqs
     run = PrefillRunner(torch, G, inp, device)
-    launches8 = 2 + 2 * n_windows(G, inp.cu_seqlens, hv)
+    launches8 = 2 + 2 * n_windows(G, inp.cu_seqlens, hv, run.ws)[0]
     ms = timed(run.step)
     fused = T * B_FUSED + 2 * N * STATE_BYTES
     unfused = T * (B_CONV + B_CORE + B_NORM) + 2 * N * STATE_BYTES

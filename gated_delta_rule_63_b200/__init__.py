@@ -16,7 +16,7 @@ import numpy as np
 
 __all__ = [
     "GdrError", "lib", "status_string", "prepare_chunks", "causal_conv", "chunk_prefill",
-    "chunk_prefill_noalloc", "chunk_prefill_slots", "prefill_workspace", "prefill_fused_workspace", "prefill_window",
+    "chunk_prefill_noalloc", "chunk_prefill_slots", "prefill_schedule", "prefill_workspace", "prefill_fused_workspace", "prefill_window",
     "decode_step", "decode_step_slots", "gated_rmsnorm", "get_device_error", "debug_wait_timeout",
     "HEAD_DIM", "CHUNK",
 ]
@@ -89,9 +89,11 @@ def lib(path: Optional[str] = None):
     L.gdr_chunk_prefill_slots.argtypes = [_vp, _vp, _vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp, _vp,
                                           ctypes.c_float, ctypes.c_int, ctypes.c_int, _vp, _ip, ctypes.c_int,
                                           _vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, ctypes.c_size_t, _vp]
+    L.gdr_chunk_prefill_schedule.argtypes = [_ip, ctypes.c_int, ctypes.c_int, ctypes.c_size_t, ctypes.c_int,
+                                             ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     for fn in ("gdr_prepare_chunks", "gdr_causal_conv", "gdr_chunk_prefill", "gdr_decode_step",
                "gdr_decode_step_slots", "gdr_gated_rmsnorm", "gdr_get_device_error",
-               "gdr_debug_wait_timeout", "gdr_chunk_prefill_slots"):
+               "gdr_debug_wait_timeout", "gdr_chunk_prefill_slots", "gdr_chunk_prefill_schedule"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
     return L
@@ -221,6 +223,18 @@ def prefill_window(cu_seqlens_host, hv: int, max_bytes: int = DEFAULT_WORKSPACE_
     carry = lib().gdr_chunk_prefill_workspace_size(n, hv, 1, int(has_final_state)) - per_chunk
     fit = max(1, (max_bytes - carry) // per_chunk)
     return int(min(max_chunks, fit))
+
+
+def prefill_schedule(cu_seqlens_host, hv: int, workspace_bytes: int, has_final_state: bool = True):
+    """(windows, pipelined) of gdr_chunk_prefill for these sequences and workspace size on the
+    current CUDA device: the number of windows (one operand launch and one state launch each)
+    and whether the next window is built beside the current one's state walk."""
+    cu, cup = _host_cu(cu_seqlens_host)
+    w, pl = ctypes.c_int(0), ctypes.c_int(0)
+    _check("gdr_chunk_prefill_schedule", lib().gdr_chunk_prefill_schedule(
+        cup, cu.shape[0] - 1, int(hv), int(workspace_bytes), int(bool(has_final_state)), ctypes.byref(w),
+        ctypes.byref(pl)))
+    return w.value, bool(pl.value)
 
 
 def prefill_workspace(cu_seqlens_host, hv: int, device, window: Optional[int] = None,

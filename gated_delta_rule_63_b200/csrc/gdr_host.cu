@@ -76,7 +76,7 @@ const char *gdr_status_string(int status) {
   }
 }
 
-int gdr_abi_version(void) { return 4; }
+int gdr_abi_version(void) { return 5; }
 
 const char *gdr_last_error_string(void) { return gdr::t_last_error_ptr(); }
 
@@ -197,6 +197,26 @@ int gdr_decode_step_slots(const void *x, const void *conv_w, void *conv_state_po
 size_t gdr_chunk_prefill_workspace_size(int n_seqs, int hv, int window_chunks, int has_final_state) {
   if (n_seqs <= 0 || hv <= 0 || window_chunks <= 0) return 0;
   return chunk_prefill_workspace_bytes(n_seqs, hv, window_chunks, has_final_state == 0);
+}
+
+int gdr_chunk_prefill_schedule(const int32_t *cu_host, int n_seqs, int hv, size_t workspace_bytes,
+                               int has_final_state, int *windows, int *pipelined) {
+  clear_last_error();
+  if (!cu_host || !windows || !pipelined) return GDR_ERR_NULL;
+  if (hv <= 0 || n_seqs < 0 || (has_final_state != 0 && has_final_state != 1)) return GDR_ERR_SHAPE;
+  int st = check_cu_seqlens(cu_host, n_seqs);
+  if (st) return st;
+  int max_chunks = 0;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int nc = (cu_host[i + 1] - cu_host[i] + kChunk - 1) / kChunk;
+    if (nc > max_chunks) max_chunks = nc;
+  }
+  int win = 1;
+  bool pl = false;
+  st = plan_chunk_prefill(n_seqs, hv, max_chunks, workspace_bytes, has_final_state == 0, false, windows, &win, &pl);
+  if (st) return st;
+  *pipelined = pl ? 1 : 0;
+  return GDR_OK;
 }
 
 size_t gdr_chunk_prefill_fused_workspace_size(int n_seqs, int hk, int hv, int total_tokens, int window_chunks,

@@ -89,6 +89,11 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
                          float eps, void *y, void *workspace, size_t ws_bytes, cudaStream_t s,
                          const PrefillPool *pool = nullptr);
 size_t chunk_prefill_workspace_bytes(int n_seqs, int hv, int window_chunks, bool need_carry);
+// window schedule of a prefill call on the current device (windows, chunks per window,
+// whether the next window's prep runs beside the current chain); GDR_ERR_WORKSPACE when
+// not even one chunk per sequence fits
+int plan_chunk_prefill(int n_seqs, int hv, int max_chunks, size_t ws_bytes, bool carry_in_ws, bool capturing,
+                       int *windows, int *win_chunks, bool *pipelined);
 
 // Conv output of `total` tokens of `channels` bf16 kept in the workspace when the conv is
 // fused into the prefill (a whole number of KiB, so the records after it stay aligned).

@@ -1260,7 +1260,6 @@ struct PipeStreams {
   cudaStream_t hi = nullptr, lo = nullptr;
   cudaEvent_t ev[kPipeEvents] = {};
   int next = 0;
-  int sms = 0;
   std::mutex lock;   // one call at a time issues on a device's pair
 };
 
@@ -1276,8 +1275,7 @@ int pipe_streams(PipeStreams **out) {
   if (!ps.hi) {
     int least = 0, greatest = 0;
     cudaStream_t hi = nullptr, lo = nullptr;
-    e = cudaDeviceGetAttribute(&ps.sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&hi, cudaStreamNonBlocking, greatest);
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&lo, cudaStreamNonBlocking, least);
     for (int i = 0; i < kPipeEvents && e == cudaSuccess; ++i)
@@ -1290,7 +1288,59 @@ int pipe_streams(PipeStreams **out) {
   return GDR_OK;
 }
 
+int device_sms(int *sms) {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return launch_status(e, "prefill: cudaGetDevice");
+  if (dev < 0 || dev >= 64) return GDR_ERR_UNSUPPORTED;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return launch_status(e, "prefill: SM count");
+    cached[dev].store(n, std::memory_order_relaxed);
+  }
+  *sms = n;
+  return GDR_OK;
+}
+
 }  // namespace
+
+// The window schedule of a call: as many chunks per window as the workspace holds (the
+// state crosses windows in hT, in the pool entries, or in the workspace tail), or, pipelined
+// (see PipeStreams), two record buffers when the chains leave SMs idle, each buffer at least
+// kPipeMinChunks chunks, and at least three windows result.
+int plan_chunk_prefill(int n_seqs, int hv, int max_chunks, size_t ws_bytes, bool carry_in_ws, bool capturing,
+                       int *windows, int *win_chunks, bool *pipelined) {
+  const size_t rec_per_chunk = static_cast<size_t>(n_seqs) * hv * WS_REC;
+  const size_t carry = carry_in_ws ? chunk_prefill_workspace_bytes(n_seqs, hv, 0, true) : 0;
+  *pipelined = false;
+  if (max_chunks <= 0) {
+    *windows = 1;
+    *win_chunks = 1;
+    return GDR_OK;
+  }
+  if (rec_per_chunk == 0 || ws_bytes < carry + rec_per_chunk) return GDR_ERR_WORKSPACE;
+  int win = static_cast<int>(std::min<size_t>({(ws_bytes - carry) / rec_per_chunk, static_cast<size_t>(max_chunks),
+                                               size_t{65535}}));
+  const size_t fit2 = (ws_bytes - carry) / (2 * rec_per_chunk);
+  if (!capturing && max_chunks > 2 * kPipeMinChunks && fit2 >= static_cast<size_t>(kPipeMinChunks) &&
+      max_chunks > win) {
+    int sms = 0;
+    const int st = device_sms(&sms);
+    if (st) return st;
+    if (static_cast<long long>(n_seqs) * hv * NS < sms) {
+      const int win2 = static_cast<int>(std::min<size_t>({fit2, static_cast<size_t>(max_chunks), size_t{65535}}));
+      if ((max_chunks + win2 - 1) / win2 >= 3) {
+        win = win2;
+        *pipelined = true;
+      }
+    }
+  }
+  *win_chunks = win;
+  *windows = (max_chunks + win - 1) / win;
+  return GDR_OK;
+}
 
 size_t chunk_prefill_workspace_bytes(int n_seqs, int hv, int window_chunks, bool need_carry) {
   size_t b = static_cast<size_t>(n_seqs) * hv * window_chunks * WS_REC;
@@ -1308,37 +1358,23 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   if (n_seqs > 65535 || hv > 65535) return GDR_ERR_SHAPE;
   int st = ensure_smem_attrs();
   if (st) return st;
-  // window: as many chunks as the workspace holds; the state crosses windows in hT, in the pool entries, or in the workspace tail (no final
-  // state asked for, or sequences of a pooled call that have no entry)
   const bool carry_in_ws = hT == nullptr;
   const size_t rec_per_chunk = static_cast<size_t>(n_seqs) * hv * WS_REC;
-  const size_t carry = carry_in_ws ? chunk_prefill_workspace_bytes(n_seqs, hv, 0, true) : 0;
-  if (max_chunks > 0 && (!workspace || ws_bytes < carry + rec_per_chunk)) return GDR_ERR_WORKSPACE;
-  int win = 1;
-  if (max_chunks > 0)
-    win = static_cast<int>(std::min<size_t>((ws_bytes - carry) / rec_per_chunk, static_cast<size_t>(max_chunks)));
-  if (win > 65535) win = 65535;
-  // pipelined windows (see PipeStreams): two record buffers of `win2` chunks each
-  PipeStreams *ps = nullptr;
-  bool pipelined = false;
+  if (max_chunks > 0 && !workspace) return GDR_ERR_WORKSPACE;
+  // under stream capture the call keeps to the caller's stream: the library's streams are
+  // shared by all calls on the device and must not join one caller's graph
   cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
   if (max_chunks > 2 * kPipeMinChunks) {
     const cudaError_t ce = cudaStreamIsCapturing(s, &capture);
     if (ce != cudaSuccess) return launch_status(ce, "prefill: cudaStreamIsCapturing");
   }
-  // (under stream capture the call keeps to the caller's stream: the library's streams are
-  // shared by all calls on the device and must not join one caller's graph)
-  if (max_chunks > 2 * kPipeMinChunks && capture == cudaStreamCaptureStatusNone) {
-    const size_t fit2 = (ws_bytes - carry) / (2 * rec_per_chunk);
-    if (fit2 >= static_cast<size_t>(kPipeMinChunks) && max_chunks > win) {
-      st = pipe_streams(&ps);
-      if (st) return st;
-      if (static_cast<long long>(n_seqs) * hv * NS < ps->sms) {
-        win = static_cast<int>(std::min<size_t>({fit2, static_cast<size_t>(max_chunks), size_t{65535}}));
-        pipelined = (max_chunks + win - 1) / win >= 3;
-      }
-    }
-  }
+  int n_windows = 1, win = 1;
+  bool pipelined = false;
+  st = plan_chunk_prefill(n_seqs, hv, max_chunks, ws_bytes, carry_in_ws, capture != cudaStreamCaptureStatusNone,
+                          &n_windows, &win, &pipelined);
+  if (st) return st;
+  PipeStreams *ps = nullptr;
+  if (pipelined && (st = pipe_streams(&ps))) return st;
   const size_t buf_bytes = rec_per_chunk * win;
   float *carry_buf = carry_in_ws && max_chunks > 0
                          ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + buf_bytes * (pipelined ? 2 : 1))
@@ -1380,7 +1416,6 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
   p.pool_init = pool ? pool->init_from_pool : 0;
   p.pool = pool ? pool->pool : nullptr;
   p.carry = carry_buf;
-  const int n_windows = max_chunks > 0 ? (max_chunks + win - 1) / win : 1;
   auto window_params = [&](int w) {
     PrefillParams pw = p;
     pw.win0 = w * win;

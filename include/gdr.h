@@ -76,7 +76,8 @@ GDR_API const char *gdr_status_string(int status);
 /* ABI version of this header, bumped whenever a signature or what a call does
  * changes (2: the conv fused into gdr_chunk_prefill,
  * gdr_chunk_prefill_fused_workspace_size; 3: gdr_decode_step_slots; 4:
- * gdr_chunk_prefill_slots). */
+ * gdr_chunk_prefill_slots; 5: gdr_chunk_prefill_schedule and the
+ * pipelined window schedule). */
 GDR_API int gdr_abi_version(void);
 
 /*
@@ -211,6 +212,22 @@ GDR_API int gdr_chunk_prefill(const void *q, const void *k, const void *v, int64
  */
 GDR_API size_t gdr_chunk_prefill_workspace_size(int n_seqs, int hv, int window_chunks,
                                                 int has_final_state);
+
+/*
+ * The window schedule gdr_chunk_prefill (and gdr_chunk_prefill_slots,
+ * has_final_state = 0) follows for these sequences and this workspace on the
+ * current device, outside stream capture: *windows receives the number of
+ * windows (each one launch of the operand kernel and one of the state kernel;
+ * 1 when no sequence has a token) and *pipelined 1 when window w + 1 is built
+ * beside window w's state walk (the two-buffer schedule described under
+ * gdr_chunk_prefill), else 0.  Host only; it may query the device's SM
+ * count.  Returns GDR_ERR_NULL for a NULL pointer, GDR_ERR_SHAPE for hv <= 0,
+ * a negative n_seqs or has_final_state not 0 or 1, GDR_ERR_CU_SEQLENS for
+ * bad offsets, GDR_ERR_WORKSPACE when not one chunk of every sequence fits.
+ */
+GDR_API int gdr_chunk_prefill_schedule(const int32_t *cu_seqlens_host, int n_seqs, int hv,
+                                       size_t workspace_bytes, int has_final_state, int *windows,
+                                       int *pipelined);
 
 /*
  * Bytes of device workspace gdr_chunk_prefill needs with the conv fused

@@ -44,7 +44,7 @@ def test_status_strings(L):
     for code in range(1, 10):
         assert G.status_string(code).startswith("GDR_ERR_")
     assert "UNKNOWN" in G.status_string(12345)
-    assert L.gdr_abi_version() == 4
+    assert L.gdr_abi_version() == 5
 
 
 @pytest.mark.parametrize("lengths", [[0], [1], [64], [65, 0, 128, 1, 63], [5000, 3, 64 * 7 + 1],
@@ -169,6 +169,30 @@ def test_wait_self_test_rejects_bad_arguments(L):
     assert L.gdr_debug_wait_timeout(0, 0, FAKE, None) == 2           # no bound
     assert L.gdr_debug_wait_timeout(0, 1 << 40, FAKE, None) == 2     # bound above 2^31
     assert L.gdr_debug_wait_timeout(0, 10, None, None) == 1          # no result word
+
+
+def test_prefill_schedule_on_host(L):
+    """Windows of a call as the workspace shrinks (no pipelining below 33 chunks, so no device
+    query), and argument rejection."""
+    f = L.gdr_chunk_prefill_schedule
+    f.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int, ctypes.c_int, ctypes.c_size_t, ctypes.c_int,
+                  ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    cu, cup = _cu([300, 64, 1])                # 5, 1, 1 chunks
+    w, pl = ctypes.c_int(-1), ctypes.c_int(-1)
+    for chunks, final, want in ((5, 1, 1), (2, 1, 3), (1, 1, 5), (3, 0, 2)):
+        ws = L.gdr_chunk_prefill_workspace_size(3, 48, chunks, final)
+        assert f(cup, 3, 48, ws, final, ctypes.byref(w), ctypes.byref(pl)) == 0
+        assert (w.value, pl.value) == (want, 0), chunks
+    assert f(cup, 3, 48, L.gdr_chunk_prefill_workspace_size(3, 48, 1, 1) - 1, 1, ctypes.byref(w),
+             ctypes.byref(pl)) == 6
+    assert f(cup, 3, 48, 1 << 30, 1, None, ctypes.byref(pl)) == 1
+    assert f(cup, 3, 0, 1 << 30, 1, ctypes.byref(w), ctypes.byref(pl)) == 2
+    assert f(cup, 3, 48, 1 << 30, 2, ctypes.byref(w), ctypes.byref(pl)) == 2
+    bad, badp = _cu([3])
+    bad[1] = -1
+    assert f(badp, 1, 48, 1 << 30, 1, ctypes.byref(w), ctypes.byref(pl)) == 4
+    empty, emptyp = _cu([0, 0])
+    assert f(emptyp, 2, 48, 0, 1, ctypes.byref(w), ctypes.byref(pl)) == 0 and w.value == 1
 
 
 def test_prefill_slots_rejects_bad_arguments_on_host(L):

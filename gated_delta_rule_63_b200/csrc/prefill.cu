@@ -110,8 +110,8 @@ static_assert(C_SMEM <= 232448, "chain shared memory exceeds 227 KB");
 static_assert((C_QW_KB | C_OFF_K | C_OFF_MQ | C_STAGE | C_OFF_H | C_OFF_U) % 1024 == 0,
               "swizzled tiles need 1 KB alignment");
 constexpr uint32_t C_TM_COLS = 512;
-constexpr uint32_t C_COL_P = 0;      // [W_hi; Q] [H_hi | H_lo]: lanes 0..63 W rows, 64..127 Q rows
-constexpr uint32_t C_COL_P2 = 128;   // [W_lo; W_hi] H_hi: lanes 0..63 hold W_lo H_hi
+constexpr uint32_t C_COL_P = 0;      // [W_hi; Q] [H_hi | H_lo]: lanes 64..127 hold Q H0 (the W rows go unread)
+constexpr uint32_t C_COL_PW = 128;   // M = 64: W_hi [H_hi | H_lo] + W_lo [H_hi | -], W row 16 q + i in lane 32 q + i
 constexpr uint32_t C_COL_H = 256;    // K^T [U'_hi | U'_lo], lanes = dk
 constexpr uint32_t C_COL_O = 384;    // [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi, lanes 64..127
 
@@ -733,8 +733,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // H (128 dk rows x 64 dv columns) stays in registers of warps 0..7: warp w
 // holds rows 32 (w & 3) .. + 31 (its TMEM lane quarter), columns
 // 32 (w >> 2) .. + 31.  Per chunk:
-//   P  = [W_hi; Q] [H_hi | H_lo],  P2 = [W_lo; W_hi] H_hi          tensor cores
-//   U  = Ut - W H0,  U' = U e^(gamma_L - gamma) / |k|                warps 0, 1, 4, 5 (lanes 0..63)
+//   PW = W_hi [H_hi | H_lo] + W_lo [H_hi | -]   (M = 64)             tensor cores
+//   P  = [W_hi; Q] [H_hi | H_lo]   (for Q H0, after PW)               tensor cores
+//   U  = Ut - W H0,  U' = U e^(gamma_L - gamma) / |k|                warps 0..7
+//   (an M = 64 product puts 16 W rows on each of the four TMEM lane quarters, so the U
+//   phase runs on all four SM sub-partitions, 16 rows x 32 columns a warp)
 //   H' = K^T [U'_hi | U'_lo]                                         tensor cores
 //   H  = e^gamma_L H + H'                                            warps 0..7
 //   O  = [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi              tensor cores
@@ -749,8 +752,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // the next chunk's first products run.
 // The handoffs (mbarrier: who completes it -> what it allows):
 //   full_qw, full_k, full_mq (per stage): a chunk's copies landed -> its products may read them
-//   bar_p:   P and P2 done (commit)     -> U warps read W H0, output warps read Q H0
-//   u_ready: U, U' tiles written (4 W-row warps) -> K^T U' and O may be issued
+//   bar_pw:  PW done (commit)           -> every state warp reads W H0 for the U phase
+//   bar_p:   P done (commit)            -> output warps read Q H0; the [Q | W] stage is free
+//   u_ready: U, U' tiles written (8 warps) -> K^T U' and O may be issued
 //   bar_h:   K^T U' done (commit)       -> every state warp updates its part of H
 //   h_ready: H tiles written (8 warps)  -> the next chunk's P (which overwrites P's region)
 //   bar_o:   O done (commit)            -> output warps read it; the U tiles may be rewritten
@@ -796,8 +800,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   const uint32_t full_qw = bars, full_k = bars + 16, full_mq = bars + 32;   // + 8 * stage
   const uint32_t bar_p = bars + 48, bar_h = bars + 56, bar_o = bars + 64;  // products complete
   const uint32_t o_free = bars + 72, h_ready = bars + 80, u_ready = bars + 88, bar_drain = bars + 96;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 104);
-  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C_OFF_BAR + 108);
+  const uint32_t bar_pw = bars + 104;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 112);
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C_OFF_BAR + 116);
   const bool ctrl = warp == kCtrlWarp;
 
   if (warp == 0) {
@@ -833,9 +838,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     iss_mq = cw + 1;
   };
   if (ctrl && lane == 0) {
-    // full x 6, products x 3, o_free (4 output warps), h_ready (8 warps), u_ready (4 state warps), drain
-    const uint32_t counts[13] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 8, 4, 1};
-    for (int i = 0; i < 13; ++i) mbar_init(bars + 8 * i, counts[i]);
+    // full x 6, products x 3, o_free (4 output warps), h_ready (8 warps), u_ready (8 warps), drain, PW
+    const uint32_t counts[14] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 8, 8, 1, 1};
+    for (int i = 0; i < 14; ++i) mbar_init(bars + 8 * i, counts[i]);
     if (kNorm) {   // the other slice's 64 row sums: 256 transaction bytes per chunk
       mbar_init(sbase + C_OFF_PBAR, 1);
       mbar_init(sbase + C_OFF_PBAR + 8, 1);
@@ -911,7 +916,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       const int s = cw & 1;
       const uint32_t par = (cw >> 1) & 1, ph = cw & 1;
       const uint32_t st = sbase + s * C_STAGE;
-      // ---- P = [Q; W_hi] [H_hi | H_lo] (N = 128), P2 = [W_hi; W_lo] H_hi (N = 64) ----------
+      // ---- PW = W_hi [H_hi | H_lo] + W_lo [H_hi | -] (M = 64), then P = [W_hi; Q] [H_hi | H_lo] ----
       PTIME_T(1 + cw, 25, 32 * kCtrlWarp);
       if (chain_wait(full_qw + 8 * s, par, abort_flag, p.err)) wt_qw = cw + 1;
       PTIME_T(1 + cw, 28, 32 * kCtrlWarp);
@@ -919,17 +924,24 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       PTIME_T(1 + cw, 11, 32 * kCtrlWarp);
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t id1 = idesc_bf16(128, 128, false, true), id2 = idesc_bf16(128, 64, false, true);
+        const uint32_t idw1 = idesc_bf16(64, 128, false, true), idw2 = idesc_bf16(64, 64, false, true);
+        const uint32_t id1 = idesc_bf16(128, 128, false, true);
         const uint64_t bh = sdesc(sbase + C_OFF_H, BLK128, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // A = rows [W_hi; Q]
+        for (int kk = 0; kk < 8; ++kk) {   // A = rows W_hi
           const uint32_t aoff = (kk >> 2) * C_QW_KB + 64 * 128 + (kk & 3) * 32;
-          mma_bf16(tmem + C_COL_P, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id1, kk > 0);
+          mma_bf16(tmem + C_COL_PW, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), idw1, kk > 0);
         }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // A = rows [W_lo; W_hi]
+        for (int kk = 0; kk < 8; ++kk) {   // A = rows W_lo, into the H_hi half
           const uint32_t aoff = (kk >> 2) * C_QW_KB + (kk & 3) * 32;
-          mma_bf16(tmem + C_COL_P2, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id2, kk > 0);
+          mma_bf16(tmem + C_COL_PW, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), idw2, 1);
+        }
+        mma_commit(bar_pw);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {   // A = rows [W_hi; Q]: Q H0 in lanes 64..127
+          const uint32_t aoff = (kk >> 2) * C_QW_KB + 64 * 128 + (kk & 3) * 32;
+          mma_bf16(tmem + C_COL_P, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id1, kk > 0);
         }
         mma_commit(bar_p);
       }
@@ -1001,71 +1013,76 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     __syncwarp();
     if (lane == 0) mbar_arrive(h_ready);
 
-    // per-chunk data read into registers one chunk ahead: Ut (state rows) and scalars
-    float ut[32];
+    // U phase (every state warp): W row ru = 16 q4 + (lane & 15) of the M = 64 product,
+    // dv columns cu .. cu + 15 of this slice (16x32bx2 TMEM loads)
+    const int ru = 16 * q4 + (lane & 15), cu = 32 * ch + 16 * (lane >> 4);
+    // per-chunk data read into registers one chunk ahead: Ut (row ru) and scalars
+    float ut[16];
     auto load_ut = [&](int cw) {
       const float4 *src = reinterpret_cast<const float4 *>(ws_record(p, n, h, cw) + WS_UT +
-                                                           (static_cast<size_t>(slice) * 64 + r) * 256);
+                                                           (static_cast<size_t>(slice) * 64 + ru) * 256);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float4 v4 = src[(8 * ch + j) ^ (r & 7)];
+      for (int j = 0; j < 4; ++j) {
+        const float4 v4 = src[((cu >> 2) + j) ^ (ru & 7)];
         ut[4 * j] = v4.x; ut[4 * j + 1] = v4.y; ut[4 * j + 2] = v4.z; ut[4 * j + 3] = v4.w;
       }
     };
-    float nx_g = 0.0f, nx_s = 0.0f, nx_gL = 0.0f;   // gamma_r, 1/|k_r| or 1/|q_r|, gamma_(L-1)
+    // gamma and 1/|k| of row ru, gamma and 1/|q| of output row r, gamma_(L-1)
+    float nx_gu = 0.0f, nx_ku = 0.0f, nx_g = 0.0f, nx_s = 0.0f, nx_gL = 0.0f;
     auto load_sc = [&](int cw) {
       const float *sc = reinterpret_cast<const float *>(ws_record(p, n, h, cw) + WS_SC);
-      nx_g = sc[r];
-      nx_s = wrow ? sc[128 + r] : sc[64 + r];
+      nx_gu = sc[ru];
+      nx_ku = sc[128 + ru];
+      if (!wrow) {
+        nx_g = sc[r];
+        nx_s = sc[64 + r];
+      }
       nx_gL = sc[63];
     };
     if (nw > 0) {
       load_sc(0);
-      if (wrow) load_ut(0);
+      load_ut(0);
     }
 
     float oreg[32];   // e^gamma / |q| Q H0 part of o (output rows)
     for (int cw = 0; cw < nw; ++cw) {
       const uint32_t ph = cw & 1;
       const int t0 = t0_of(cw), L = min(C, seq_end - t0);
-      const float g_r = nx_g, sb = nx_s, gL = nx_gL;
+      const float g_u = nx_gu, k_u = nx_ku, g_r = nx_g, sb = nx_s, gL = nx_gL;
       if (cw + 1 < nw) load_sc(cw + 1);
       PTIME(1 + cw, 0);
 
-      if (wrow) {
-        // ---- U = Ut - W H0 and U' = U e^(gamma_L - gamma) / |k| (state rows) ----------------
-        chain_wait(bar_p, ph, abort_flag, p.err);
+      {
+        // ---- U = Ut - W H0 and U' = U e^(gamma_L - gamma) / |k| (W row ru, 16 columns) ------
+        chain_wait(bar_pw, ph, abort_flag, p.err);
         PTIME_T(1 + cw, 22, 64);
         if (cw > 0) chain_wait(bar_o, ph ^ 1, abort_flag, p.err);   // the last O product read U
         __syncwarp();
         tc_fence_after();
         PTIME_T(1 + cw, 23, 64);
-        const float ed = __expf(gL - g_r) * sb;
+        const float ed = __expf(gL - g_u) * k_u;
+        const uint32_t tw = tmem + (static_cast<uint32_t>(32 * q4) << 16) + C_COL_PW + 32 * ch;
+        float pab[16], pb[16];
+        tmem_ld16x2(tw, pab);        // W_hi H_hi + W_lo H_hi
+        tmem_ld16x2(tw + 64, pb);    // W_hi H_lo
+        tmem_wait_ld();
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float pa[16], pb[16], pc[16];
-          tmem_ld16(tl + C_COL_P + 16 * hh, pa);
-          tmem_ld16(tl + C_COL_P + 64 + 16 * hh, pb);
-          tmem_ld16(tl + C_COL_P2 + 16 * hh, pc);
-          tmem_wait_ld();
+        for (int c4 = 0; c4 < 2; ++c4) {
+          float u[8], us[8];
 #pragma unroll
-          for (int c4 = 0; c4 < 2; ++c4) {
-            float u[8], us[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int j = 8 * c4 + e;
-              u[e] = ((ut[16 * hh + j] - pa[j]) - pb[j]) - pc[j];
-              us[e] = u[e] * ed;
-            }
-            const uint32_t off = sw128(r, 4 * ch + 2 * hh + c4);
-            uint4 hi, lo;
-            split8x2(u, hi, lo);
-            st_shared16(sbase + C_OFF_U + off, hi);
-            st_shared16(sbase + C_OFF_U + BLK64 + off, lo);
-            split8x2(us, hi, lo);
-            st_shared16(sbase + C_OFF_U + 2 * BLK64 + off, hi);
-            st_shared16(sbase + C_OFF_U + 3 * BLK64 + off, lo);
+          for (int e = 0; e < 8; ++e) {
+            const int j = 8 * c4 + e;
+            u[e] = (ut[j] - pab[j]) - pb[j];
+            us[e] = u[e] * ed;
           }
+          const uint32_t off = sw128(ru, (cu >> 3) + c4);
+          uint4 hi, lo;
+          split8x2(u, hi, lo);
+          st_shared16(sbase + C_OFF_U + off, hi);
+          st_shared16(sbase + C_OFF_U + BLK64 + off, lo);
+          split8x2(us, hi, lo);
+          st_shared16(sbase + C_OFF_U + 2 * BLK64 + off, hi);
+          st_shared16(sbase + C_OFF_U + 3 * BLK64 + off, lo);
         }
         PTIME_T(1 + cw, 24, 64);
         fence_proxy_async();
@@ -1074,7 +1091,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (lane == 0) mbar_arrive(u_ready);
         PTIME_T(1 + cw, 12, 64);
         if (cw + 1 < nw) load_ut(cw + 1);
-      } else {
+      }
+      if (!wrow) {
         // ---- Q H0 part of the output (output rows) ------------------------------------------
         chain_wait(bar_p, ph, abort_flag, p.err);
         __syncwarp();

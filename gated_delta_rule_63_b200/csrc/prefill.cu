@@ -88,8 +88,9 @@ static_assert(3 * (P_SMEM + 1024) <= 228 * 1024, "three prep CTAs per SM");
 constexpr uint32_t P_TM_COLS = 128;                  // [K K^T ; Q K^T] (64 cols), then W, then Ut
 
 // ---- chain kernel ------------------------------------------------------------
-constexpr int kChainThreads = 288;                    // warps 0..7 state and output, warp 8 control
+constexpr int kChainThreads = 320;                    // warps 0..7 state and output, 8 products, 9 copies
 constexpr int kCtrlWarp = 8;
+constexpr int kCopyWarp = 9;
 // stage: per k-block the rows [W_lo 0..63 | W_hi 64..127 | Q 128..191] (A operands
 // [W_lo; W_hi] and [W_hi; Q]), then K (two dk blocks), then [Mq_lo; Mq_hi]
 constexpr uint32_t C_QW_KB = 192 * 128;
@@ -99,10 +100,10 @@ constexpr uint32_t C_STAGE = C_OFF_MQ + 2 * BLK64;   // 80 KiB
 constexpr uint32_t BLK128 = 128 * 128;
 constexpr uint32_t C_OFF_H = 2 * C_STAGE;            // [H_hi | H_lo], each [128 dk][64 dv]
 constexpr uint32_t C_OFF_U = C_OFF_H + 2 * BLK128;   // [U_hi | U_lo | U'_hi | U'_lo], each [64 tok][64 dv]
-constexpr uint32_t C_OFF_BAR = C_OFF_U + 4 * BLK64;  // 13 mbarriers, tmem base, abort flag
+constexpr uint32_t C_OFF_BAR = C_OFF_U + 4 * BLK64;  // 20 mbarriers, tmem base, abort flag
 // fused gated norm: per-row partial sums of squares of this CTA's two column halves
 // [parity 2][half 2][64], the other dv slice's row sums [parity 2][64], two mbarriers
-constexpr uint32_t C_OFF_NORM = C_OFF_BAR + 128;
+constexpr uint32_t C_OFF_NORM = C_OFF_BAR + 192;
 constexpr uint32_t C_OFF_PEER = C_OFF_NORM + 2 * 2 * 64 * 4;
 constexpr uint32_t C_OFF_PBAR = C_OFF_PEER + 2 * 64 * 4;
 constexpr uint32_t C_SMEM = C_OFF_PBAR + 16 + 1024;
@@ -744,14 +745,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 //   o  = scale (e^gamma / |q| Q H0 + O)                              warps 2, 3, 6, 7 (lanes 64..127)
 // N = 128 products stack the hi and lo parts of one operand side by side, so
 // each fp32 product takes two MMA groups instead of three.  Warp 8 issues every
-// product and every copy and does nothing else; the roles meet only on
-// mbarriers (no CTA-wide barrier inside the chunk loop).  Operands arrive two
-// chunks ahead in three groups ([Q | W_hi | W_lo], K, Mq), each refilled as
-// soon as the products reading it are complete; Ut and the chunk scalars are
-// read into registers a chunk ahead; the output of a chunk is finished while
-// the next chunk's first products run.
+// product, warp 9 every copy; the roles meet only on mbarriers (no CTA-wide
+// barrier inside the chunk loop).  Operands arrive two chunks ahead in three
+// groups ([Q | W_hi | W_lo], K, Mq) in two stages; warp 8 commits a stage's
+// "empty" mbarrier after the last product that reads it, and warp 9 refills it
+// then.  Ut and the chunk scalars are read into registers a chunk ahead; the
+// output of a chunk is finished while the next chunk's first products run.
 // The handoffs (mbarrier: who completes it -> what it allows):
 //   full_qw, full_k, full_mq (per stage): a chunk's copies landed -> its products may read them
+//   empty_qw, empty_k, empty_mq (per stage): the products reading the stage are done (commit)
+//            -> warp 9 loads the chunk two ahead into it
 //   bar_pw:  PW done (commit)           -> every state warp reads W H0 for the U phase
 //   bar_p:   P done (commit)            -> output warps read Q H0; the [Q | W] stage is free
 //   u_ready: U, U' tiles written (8 warps) -> K^T U' and O may be issued
@@ -801,17 +804,18 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   const uint32_t bar_p = bars + 48, bar_h = bars + 56, bar_o = bars + 64;  // products complete
   const uint32_t o_free = bars + 72, h_ready = bars + 80, u_ready = bars + 88, bar_drain = bars + 96;
   const uint32_t bar_pw = bars + 104;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 112);
-  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C_OFF_BAR + 116);
-  const bool ctrl = warp == kCtrlWarp;
+  const uint32_t empty_qw = bars + 112, empty_k = bars + 128, empty_mq = bars + 144;   // + 8 * stage
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 160);
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C_OFF_BAR + 164);
+  const bool ctrl = warp == kCtrlWarp, copier = warp == kCopyWarp, state = warp < kCtrlWarp;
 
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_holder), C_TM_COLS);
     tmem_relinquish();
   }
   auto t0_of = [&](int cw) { return seq_start + (p.win0 + cw) * C; };
-  // copies of chunk cw into stage cw & 1 (lane 0 of the control warp); issued counts per group
-  int iss_qw = 0, iss_k = 0, iss_mq = 0, wt_qw = 0, wt_k = 0, wt_mq = 0;
+  // copies of chunk cw into stage cw & 1 (lane 0 of the copy warp); issued counts per group
+  int iss_qw = 0, iss_k = 0, iss_mq = 0;
   auto load_qw = [&](int cw) {
     const uint32_t st = sbase + (cw & 1) * C_STAGE, fb = full_qw + 8 * (cw & 1);
     const uint8_t *rec = ws_record(p, n, h, cw);
@@ -838,22 +842,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     iss_mq = cw + 1;
   };
   if (ctrl && lane == 0) {
-    // full x 6, products x 3, o_free (4 output warps), h_ready (8 warps), u_ready (8 warps), drain, PW
-    const uint32_t counts[14] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 8, 8, 1, 1};
-    for (int i = 0; i < 14; ++i) mbar_init(bars + 8 * i, counts[i]);
+    // full x 6, products x 3, o_free (4 output warps), h_ready (8 warps), u_ready (8 warps), drain, PW,
+    // empty x 6
+    const uint32_t counts[20] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 8, 8, 1, 1, 1, 1, 1, 1, 1, 1};
+    for (int i = 0; i < 20; ++i) mbar_init(bars + 8 * i, counts[i]);
     if (kNorm) {   // the other slice's 64 row sums: 256 transaction bytes per chunk
       mbar_init(sbase + C_OFF_PBAR, 1);
       mbar_init(sbase + C_OFF_PBAR + 8, 1);
     }
     *abort_flag = 0u;
     fence_mbar_init();
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    for (int cw = 0; cw < 2 && cw < nw; ++cw) {
-      load_qw(cw);
-      load_k(cw);
-      load_mq(cw);
-    }
   }
   const int q4 = warp & 3, ch = (warp >> 2) & 1;     // lane quarter, column half
   const int row = 32 * q4 + lane;                    // TMEM lane / dk row of the state
@@ -881,7 +879,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   const size_t crow = (static_cast<size_t>(n) * p.hv + h) * D * D + static_cast<size_t>(row) * D + slice * N + 32 * ch;
   const size_t in_row = (p.slot && state_in == p.carry) ? crow : srow;
   const size_t out_row = (p.slot && state_out == p.carry) ? crow : srow;
-  if (!ctrl) {
+  if (state) {
     if (state_in) {
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {
@@ -918,7 +916,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       const uint32_t st = sbase + s * C_STAGE;
       // ---- PW = W_hi [H_hi | H_lo] + W_lo [H_hi | -] (M = 64), then P = [W_hi; Q] [H_hi | H_lo] ----
       PTIME_T(1 + cw, 25, 32 * kCtrlWarp);
-      if (chain_wait(full_qw + 8 * s, par, abort_flag, p.err)) wt_qw = cw + 1;
+      chain_wait(full_qw + 8 * s, par, abort_flag, p.err);
       PTIME_T(1 + cw, 28, 32 * kCtrlWarp);
       chain_wait(h_ready, ph, abort_flag, p.err);    // H tiles of this chunk; P of the last one read
       PTIME_T(1 + cw, 11, 32 * kCtrlWarp);
@@ -944,20 +942,14 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           mma_bf16(tmem + C_COL_P, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id1, kk > 0);
         }
         mma_commit(bar_p);
+        mma_commit(empty_qw + 8 * s);   // the [Q | W] stage is read
       }
-      // chunk cw + 1's K goes to the stage of chunk cw - 1, whose K^T U' is complete (every
-      // warp passed it before h_ready); issued here, after P, to keep P off the copy issue
-      if (lane == 0 && cw >= 1 && cw + 1 < nw) load_k(cw + 1);
       __syncwarp();
       PTIME_T(1 + cw, 1, 32 * kCtrlWarp);
-      chain_wait(bar_p, ph, abort_flag, p.err);
-      PTIME_T(1 + cw, 2, 32 * kCtrlWarp);
-      if (lane == 0 && cw + 2 < nw) load_qw(cw + 2);   // P has read this stage's [Q | W]
-      __syncwarp();
       // ---- H' = K^T [U'_hi | U'_lo] ----------------------------------------------------------
       chain_wait(u_ready, ph, abort_flag, p.err);
       PTIME_T(1 + cw, 3, 32 * kCtrlWarp);
-      if (chain_wait(full_k + 8 * s, par, abort_flag, p.err)) wt_k = cw + 1;
+      chain_wait(full_k + 8 * s, par, abort_flag, p.err);
       PTIME_T(1 + cw, 8, 32 * kCtrlWarp);
       tc_fence_after();
       if (lane == 0) {
@@ -972,13 +964,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       __syncwarp();
       PTIME_T(1 + cw, 4, 32 * kCtrlWarp);
       // ---- O = [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi (rows in lanes 64..127) ----------
-      if (cw > 0) {
-        chain_wait(o_free, ph ^ 1, abort_flag, p.err);   // the previous O is read ...
-        PTIME_T(1 + cw, 13, 32 * kCtrlWarp);
-        if (lane == 0 && cw + 1 < nw) load_mq(cw + 1);   // ... and its Mq stage is free
-        __syncwarp();
-      }
-      if (chain_wait(full_mq + 8 * s, par, abort_flag, p.err)) wt_mq = cw + 1;
+      if (cw > 0) chain_wait(o_free, ph ^ 1, abort_flag, p.err);   // the previous O is read
+      PTIME_T(1 + cw, 13, 32 * kCtrlWarp);
+      chain_wait(full_mq + 8 * s, par, abort_flag, p.err);
       PTIME_T(1 + cw, 14, 32 * kCtrlWarp);
       tc_fence_after();
       if (lane == 0) {
@@ -991,18 +979,39 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ - BLK64 + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO2, 1);
         mma_commit(bar_o);
+        mma_commit(empty_k + 8 * s);    // K (K^T U' and the unused rows of O) and Mq are read
+        mma_commit(empty_mq + 8 * s);
       }
       __syncwarp();
       PTIME_T(1 + cw, 9, 32 * kCtrlWarp);
     }
-    if (lane == 0) {
-      // every product completes before tensor memory is released; after a
-      // timeout, copies may still be landing in shared memory: let them finish
+    if (lane == 0) {   // every product completes before tensor memory is released
       mma_commit(bar_drain);
       mbar_wait(bar_drain, 0, p.err, 1u << 20);
-      for (int c = wt_qw; c < iss_qw; ++c) mbar_wait(full_qw + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
-      for (int c = wt_k; c < iss_k; ++c) mbar_wait(full_k + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
-      for (int c = wt_mq; c < iss_mq; ++c) mbar_wait(full_mq + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
+    }
+    __syncwarp();
+  } else if (copier) {
+    // ============================= copy warp =============================
+    // chunk c goes into stage c & 1 once the products of chunk c - 2 have read it
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      bool go = true;
+      for (int c = 0; c < nw && go; ++c) {
+        const int s = c & 1;
+        const uint32_t par = ((c - 2) >> 1) & 1;
+        if (c >= 2) go = chain_wait(empty_qw + 8 * s, par, abort_flag, p.err);
+        if (go) load_qw(c);
+        if (go && c >= 2) go = chain_wait(empty_k + 8 * s, par, abort_flag, p.err);
+        if (go) load_k(c);
+        if (go && c >= 2) go = chain_wait(empty_mq + 8 * s, par, abort_flag, p.err);
+        if (go) load_mq(c);
+      }
+      // after a timeout the consumers stop waiting: the last copies land before the CTA
+      // leaves (every earlier copy into a stage was consumed before the stage was refilled)
+      for (int c = max(0, iss_qw - 2); c < iss_qw; ++c) mbar_wait(full_qw + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
+      for (int c = max(0, iss_k - 2); c < iss_k; ++c) mbar_wait(full_k + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
+      for (int c = max(0, iss_mq - 2); c < iss_mq; ++c) mbar_wait(full_mq + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
     }
     __syncwarp();
   } else {
@@ -1218,7 +1227,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   if (kNorm) cluster_sync_all();   // no remote arrivals target a CTA that has left
   tc_fence_before();
   __syncthreads();
-  if (!ctrl && state_out && *abort_flag == 0u) {
+  if (state && state_out && *abort_flag == 0u) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4)
       *reinterpret_cast<float4 *>(state_out + out_row + j) = make_float4(hreg[j], hreg[j + 1], hreg[j + 2], hreg[j + 3]);

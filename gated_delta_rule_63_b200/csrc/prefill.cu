@@ -100,10 +100,10 @@ constexpr uint32_t C_STAGE = C_OFF_MQ + 2 * BLK64;   // 80 KiB
 constexpr uint32_t BLK128 = 128 * 128;
 constexpr uint32_t C_OFF_H = 2 * C_STAGE;            // [H_hi | H_lo], each [128 dk][64 dv]
 constexpr uint32_t C_OFF_U = C_OFF_H + 2 * BLK128;   // [U_hi | U_lo | U'_hi | U'_lo], each [64 tok][64 dv]
-constexpr uint32_t C_OFF_BAR = C_OFF_U + 4 * BLK64;  // 20 mbarriers, tmem base, abort flag
+constexpr uint32_t C_OFF_BAR = C_OFF_U + 4 * BLK64;  // 15 mbarriers, tmem base, abort flag
 // fused gated norm: per-row partial sums of squares of this CTA's two column halves
 // [parity 2][half 2][64], the other dv slice's row sums [parity 2][64], two mbarriers
-constexpr uint32_t C_OFF_NORM = C_OFF_BAR + 192;
+constexpr uint32_t C_OFF_NORM = C_OFF_BAR + 128;
 constexpr uint32_t C_OFF_PEER = C_OFF_NORM + 2 * 2 * 64 * 4;
 constexpr uint32_t C_OFF_PBAR = C_OFF_PEER + 2 * 64 * 4;
 constexpr uint32_t C_SMEM = C_OFF_PBAR + 16 + 1024;
@@ -744,17 +744,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 //   O  = [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi              tensor cores
 //   o  = scale (e^gamma / |q| Q H0 + O)                              warps 2, 3, 6, 7 (lanes 64..127)
 // N = 128 products stack the hi and lo parts of one operand side by side, so
-// each fp32 product takes two MMA groups instead of three.  Warp 8 issues every
-// product, warp 9 every copy; the roles meet only on mbarriers (no CTA-wide
+// each fp32 product takes two MMA groups instead of three.  Warp 8 issues the
+// products on the state's critical path (PW, K^T U'); warp 9 issues the output's
+// products (P after PW, O after K^T U', so neither delays the chain in the tensor
+// pipe) and every operand copy.  The roles meet only on mbarriers (no CTA-wide
 // barrier inside the chunk loop).  Operands arrive two chunks ahead in three
-// groups ([Q | W_hi | W_lo], K, Mq) in two stages; warp 8 commits a stage's
-// "empty" mbarrier after the last product that reads it, and warp 9 refills it
-// then.  Ut and the chunk scalars are read into registers a chunk ahead; the
-// output of a chunk is finished while the next chunk's first products run.
+// groups ([Q | W_hi | W_lo], K, Mq) in two stages; warp 9 refills a stage once
+// the chunk's O, its last product, is done.  Ut and the chunk scalars are read
+// into registers a chunk ahead; the output of a chunk is finished while the
+// next chunk's first products run.
 // The handoffs (mbarrier: who completes it -> what it allows):
 //   full_qw, full_k, full_mq (per stage): a chunk's copies landed -> its products may read them
-//   empty_qw, empty_k, empty_mq (per stage): the products reading the stage are done (commit)
-//            -> warp 9 loads the chunk two ahead into it
 //   bar_pw:  PW done (commit)           -> every state warp reads W H0 for the U phase
 //   bar_p:   P done (commit)            -> output warps read Q H0; the [Q | W] stage is free
 //   u_ready: U, U' tiles written (8 warps) -> K^T U' and O may be issued
@@ -803,10 +803,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   const uint32_t full_qw = bars, full_k = bars + 16, full_mq = bars + 32;   // + 8 * stage
   const uint32_t bar_p = bars + 48, bar_h = bars + 56, bar_o = bars + 64;  // products complete
   const uint32_t o_free = bars + 72, h_ready = bars + 80, u_ready = bars + 88, bar_drain = bars + 96;
-  const uint32_t bar_pw = bars + 104;
-  const uint32_t empty_qw = bars + 112, empty_k = bars + 128, empty_mq = bars + 144;   // + 8 * stage
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 160);
-  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C_OFF_BAR + 164);
+  const uint32_t bar_pw = bars + 104, bar_drain2 = bars + 112;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C_OFF_BAR + 120);
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C_OFF_BAR + 124);
   const bool ctrl = warp == kCtrlWarp, copier = warp == kCopyWarp, state = warp < kCtrlWarp;
 
   if (warp == 0) {
@@ -843,9 +842,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   };
   if (ctrl && lane == 0) {
     // full x 6, products x 3, o_free (4 output warps), h_ready (8 warps), u_ready (8 warps), drain, PW,
-    // empty x 6
-    const uint32_t counts[20] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 8, 8, 1, 1, 1, 1, 1, 1, 1, 1};
-    for (int i = 0; i < 20; ++i) mbar_init(bars + 8 * i, counts[i]);
+    // the copy warp's drain
+    const uint32_t counts[15] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 8, 8, 1, 1, 1};
+    for (int i = 0; i < 15; ++i) mbar_init(bars + 8 * i, counts[i]);
     if (kNorm) {   // the other slice's 64 row sums: 256 transaction bytes per chunk
       mbar_init(sbase + C_OFF_PBAR, 1);
       mbar_init(sbase + C_OFF_PBAR + 8, 1);
@@ -909,21 +908,20 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   if (kNorm) cluster_sync_all();   // both CTAs' barriers exist before either arrives remotely
 
   if (ctrl) {
-    // =========================== control warp ===========================
+    // ============= control warp: the products on the state's critical path =============
     for (int cw = 0; cw < nw; ++cw) {
       const int s = cw & 1;
       const uint32_t par = (cw >> 1) & 1, ph = cw & 1;
       const uint32_t st = sbase + s * C_STAGE;
-      // ---- PW = W_hi [H_hi | H_lo] + W_lo [H_hi | -] (M = 64), then P = [W_hi; Q] [H_hi | H_lo] ----
+      // ---- PW = W_hi [H_hi | H_lo] + W_lo [H_hi | -] (M = 64) ----------------------------------
       PTIME_T(1 + cw, 25, 32 * kCtrlWarp);
       chain_wait(full_qw + 8 * s, par, abort_flag, p.err);
       PTIME_T(1 + cw, 28, 32 * kCtrlWarp);
-      chain_wait(h_ready, ph, abort_flag, p.err);    // H tiles of this chunk; P of the last one read
+      chain_wait(h_ready, ph, abort_flag, p.err);    // H tiles of this chunk; the last PW and P read
       PTIME_T(1 + cw, 11, 32 * kCtrlWarp);
       tc_fence_after();
       if (lane == 0) {
         const uint32_t idw1 = idesc_bf16(64, 128, false, true), idw2 = idesc_bf16(64, 64, false, true);
-        const uint32_t id1 = idesc_bf16(128, 128, false, true);
         const uint64_t bh = sdesc(sbase + C_OFF_H, BLK128, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // A = rows W_hi
@@ -936,13 +934,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           mma_bf16(tmem + C_COL_PW, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), idw2, 1);
         }
         mma_commit(bar_pw);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // A = rows [W_hi; Q]: Q H0 in lanes 64..127
-          const uint32_t aoff = (kk >> 2) * C_QW_KB + 64 * 128 + (kk & 3) * 32;
-          mma_bf16(tmem + C_COL_P, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id1, kk > 0);
-        }
-        mma_commit(bar_p);
-        mma_commit(empty_qw + 8 * s);   // the [Q | W] stage is read
       }
       __syncwarp();
       PTIME_T(1 + cw, 1, 32 * kCtrlWarp);
@@ -963,52 +954,74 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       }
       __syncwarp();
       PTIME_T(1 + cw, 4, 32 * kCtrlWarp);
-      // ---- O = [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi (rows in lanes 64..127) ----------
-      if (cw > 0) chain_wait(o_free, ph ^ 1, abort_flag, p.err);   // the previous O is read
-      PTIME_T(1 + cw, 13, 32 * kCtrlWarp);
-      chain_wait(full_mq + 8 * s, par, abort_flag, p.err);
-      PTIME_T(1 + cw, 14, 32 * kCtrlWarp);
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t idO1 = idesc_bf16(128, 128, false, true), idO2 = idesc_bf16(128, 64, false, true);
-        const uint64_t bo = sdesc(sbase + C_OFF_U, BLK64, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO1, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ - BLK64 + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO2, 1);
-        mma_commit(bar_o);
-        mma_commit(empty_k + 8 * s);    // K (K^T U' and the unused rows of O) and Mq are read
-        mma_commit(empty_mq + 8 * s);
-      }
-      __syncwarp();
-      PTIME_T(1 + cw, 9, 32 * kCtrlWarp);
     }
-    if (lane == 0) {   // every product completes before tensor memory is released
+    if (lane == 0) {   // its products complete before tensor memory is released
       mma_commit(bar_drain);
       mbar_wait(bar_drain, 0, p.err, 1u << 20);
     }
     __syncwarp();
   } else if (copier) {
-    // ============================= copy warp =============================
-    // chunk c goes into stage c & 1 once the products of chunk c - 2 have read it
+    // ====== copy warp: the other products (Q H0, O) and every operand copy ======
+    // Each wait here is on work this warp issued or on a handoff that needs it, so no
+    // mbarrier can run a phase ahead of the wait.  P goes to the tensor pipe once PW is
+    // done and O once K^T U' is done, so neither delays a product of the state chain.
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      bool go = true;
-      for (int c = 0; c < nw && go; ++c) {
-        const int s = c & 1;
-        const uint32_t par = ((c - 2) >> 1) & 1;
-        if (c >= 2) go = chain_wait(empty_qw + 8 * s, par, abort_flag, p.err);
-        if (go) load_qw(c);
-        if (go && c >= 2) go = chain_wait(empty_k + 8 * s, par, abort_flag, p.err);
-        if (go) load_k(c);
-        if (go && c >= 2) go = chain_wait(empty_mq + 8 * s, par, abort_flag, p.err);
-        if (go) load_mq(c);
+      for (int c = 0; c < 2 && c < nw; ++c) {
+        load_qw(c);
+        load_k(c);
+        load_mq(c);
       }
-      // after a timeout the consumers stop waiting: the last copies land before the CTA
-      // leaves (every earlier copy into a stage was consumed before the stage was refilled)
+      for (int cw = 0; cw < nw; ++cw) {
+        const int s = cw & 1;
+        const uint32_t par = (cw >> 1) & 1, ph = cw & 1;
+        const uint32_t st = sbase + s * C_STAGE;
+        // ---- P = [W_hi; Q] [H_hi | H_lo]: Q H0 in lanes 64..127 -------------------------------
+        if (!chain_wait(bar_pw, ph, abort_flag, p.err)) break;
+        if (!chain_wait(full_qw + 8 * s, par, abort_flag, p.err)) break;   // (landed: PW read it)
+        tc_fence_after();
+        {
+          const uint32_t id1 = idesc_bf16(128, 128, false, true);
+          const uint64_t bh = sdesc(sbase + C_OFF_H, BLK128, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff = (kk >> 2) * C_QW_KB + 64 * 128 + (kk & 3) * 32;
+            mma_bf16(tmem + C_COL_P, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id1, kk > 0);
+          }
+          mma_commit(bar_p);
+        }
+        // ---- O = [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi (rows in lanes 64..127) --------
+        if (!chain_wait(bar_h, ph, abort_flag, p.err)) break;             // U tiles written, K^T U' first
+        if (cw > 0 && !chain_wait(o_free, ph ^ 1, abort_flag, p.err)) break;   // the previous O is read
+        if (!chain_wait(full_mq + 8 * s, par, abort_flag, p.err)) break;
+        tc_fence_after();
+        {
+          const uint32_t idO1 = idesc_bf16(128, 128, false, true), idO2 = idesc_bf16(128, 64, false, true);
+          const uint64_t bo = sdesc(sbase + C_OFF_U, BLK64, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO1, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ - BLK64 + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO2,
+                     1);
+          mma_commit(bar_o);
+        }
+        // ---- stage s takes chunk cw + 2 once every product of chunk cw has read it (PW,
+        // waited above; P and O, this thread's, complete with bar_o) -----------------------------
+        if (cw + 2 < nw) {
+          if (!chain_wait(bar_o, ph, abort_flag, p.err)) break;
+          load_qw(cw + 2);
+          load_k(cw + 2);
+          load_mq(cw + 2);
+        }
+      }
+      // its products complete before tensor memory is released; after a timeout the
+      // consumers stop waiting: the last copies land before the CTA leaves (every earlier
+      // copy into a stage was consumed before the stage was refilled)
+      mma_commit(bar_drain2);
+      mbar_wait(bar_drain2, 0, p.err, 1u << 20);
       for (int c = max(0, iss_qw - 2); c < iss_qw; ++c) mbar_wait(full_qw + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
       for (int c = max(0, iss_k - 2); c < iss_k; ++c) mbar_wait(full_k + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
       for (int c = max(0, iss_mq - 2); c < iss_mq; ++c) mbar_wait(full_mq + 8 * (c & 1), (c >> 1) & 1, p.err, 1u << 16);
@@ -1140,6 +1153,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             hreg[16 * hh + 2 * j] = hn.x;
             hreg[16 * hh + 2 * j + 1] = hn.y;
           }
+        }
+        // P (the copy warp's product, not covered by bar_h) reads the H tiles too: the output
+        // warps waited for it before reading Q H0
+        if (wrow) {
+          chain_wait(bar_p, ph, abort_flag, p.err);
+          __syncwarp();
         }
         write_h();
       }

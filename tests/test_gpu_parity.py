@@ -671,3 +671,62 @@ def test_prefill_varlen8_full_path_sampled_heads():
         for key in ("o", "y"):
             assert rel_l2(got[key][s:e], want[key][s:e]) <= TOL_BF16, (key, n)
         assert rel_l2(got_h[n], want_h[n]) <= TOL_STATE, n
+
+
+# ---------------------------------------------------------------------------
+# head sharding: the layer split over GPUs by heads needs no exchange
+# ---------------------------------------------------------------------------
+
+def _shard_channels(C_hk, C_hv, hk, hv, shard, n_shards):
+    """Channel indices of one head shard in the [q | k | v] layout: its key heads' q and k
+    channels and its value heads' v channels (contiguous head groups)."""
+    ks, vs = hk // n_shards, hv // n_shards
+    q = np.arange(shard * ks * 128, (shard + 1) * ks * 128)
+    k = C_hk + q
+    v = 2 * C_hk + np.arange(shard * vs * 128, (shard + 1) * vs * 128)
+    return np.concatenate([q, k, v]), slice(shard * ks, (shard + 1) * ks), slice(shard * vs, (shard + 1) * vs)
+
+
+def test_head_sharded_layer_equals_the_full_layer():
+    """Two head shards (8 key / 24 value heads each, as a 2-GPU split of the layer would hold
+    them) run through the same entry points on their slices of the inputs give the full
+    layer's o, final states and conv states bit for bit: heads never exchange data inside the
+    layer, so sharding by heads is a split of the inputs and nothing else (here both shards run
+    on one GPU, one after the other)."""
+    hk, hv = GI.HK, GI.HV
+    n = 2
+    # prefill: several windows, varlen, initial states
+    inp = GI.make_core_inputs(98, [300, 64, 129], prenorm_qk=False, h0_std=0.02)
+    full_o, full_h = None, None
+    def run(q, k, v, a, b, Al, db, h0):
+        hT = torch.empty_like(h0)
+        o = G.chunk_prefill(q, k, v, a, b, Al, db, dev_i32(inp.cu_seqlens), inp.cu_seqlens, h0=h0, hT=hT)
+        torch.cuda.synchronize()
+        return host_bits(o), hT.cpu().numpy()
+    full_o, full_h = run(dev_bf16(inp.q), dev_bf16(inp.k), dev_bf16(inp.v), dev_bf16(inp.a), dev_bf16(inp.b),
+                         dev_f32(inp.A_log), dev_f32(inp.dt_bias), dev_f32(inp.h0))
+    for s in range(n):
+        _, ks, vs = _shard_channels(hk * 128, hv * 128, hk, hv, s, n)
+        o, h = run(dev_bf16(np.ascontiguousarray(inp.q[:, ks])), dev_bf16(np.ascontiguousarray(inp.k[:, ks])),
+                   dev_bf16(np.ascontiguousarray(inp.v[:, vs])), dev_bf16(np.ascontiguousarray(inp.a[:, vs])),
+                   dev_bf16(np.ascontiguousarray(inp.b[:, vs])), dev_f32(inp.A_log[vs]), dev_f32(inp.dt_bias[vs]),
+                   dev_f32(np.ascontiguousarray(inp.h0[:, vs])))
+        assert np.array_equal(o, full_o[:, vs]), s
+        assert np.array_equal(h, full_h[:, vs]), s
+    assert G.get_device_error() == 0
+
+    # decode: conv step, norms, gates and the state update on the shard's channels and heads
+    dec = GI.make_decode_inputs(99, 4, 2)
+    f_outs, f_st, f_cs = run_gpu_decode(dec, 2, keep=(0, 1))
+    for s in range(n):
+        ch, ks, vs = _shard_channels(hk * 128, hv * 128, hk, hv, s, n)
+        part = GI.DecodeInputs(np.ascontiguousarray(dec.x[:, :, ch]), np.ascontiguousarray(dec.a[:, :, vs]),
+                               np.ascontiguousarray(dec.b[:, :, vs]), np.ascontiguousarray(dec.conv_w[ch]),
+                               np.ascontiguousarray(dec.conv_state[:, :, ch]),
+                               np.ascontiguousarray(dec.state[:, vs]), dec.A_log[vs], dec.dt_bias[vs],
+                               hk // n, hv // n, scale=dec.scale)
+        outs, st, cs = run_gpu_decode(part, 2, keep=(0, 1))
+        for step in (0, 1):
+            assert np.array_equal(outs[step], f_outs[step][:, vs]), (s, step)
+        assert np.array_equal(st, f_st[:, vs]), s
+        assert np.array_equal(cs, f_cs[:, :, ch]), s

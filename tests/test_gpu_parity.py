@@ -371,6 +371,8 @@ def test_prefill_pipelined_windows_equal_one_window(final_state):
     for window in (None, 32):
         hT = torch.full((1, hv, 128, 128), float("nan"), device="cuda") if final_state else None
         ws = G.prefill_workspace(inp.cu_seqlens, hv, "cuda", window=window, has_final_state=final_state)
+        assert G.prefill_schedule(inp.cu_seqlens, hv, ws.numel(), final_state) == ((1, False) if window is None
+                                                                                     else (3, True))
         o = torch.full((T, hv, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
         G.chunk_prefill(*args, h0=h0, hT=hT, o=o, scale=inp.scale, workspace=ws)
         torch.cuda.synchronize()
@@ -399,6 +401,19 @@ def test_prefill_pipelined_windows_equal_one_window(final_state):
     assert np.array_equal(host_bits(o), outs[0][0])
     if final_state:
         assert np.array_equal(hT.cpu().numpy(), outs[0][1])
+        # the pooled form on the same schedule: entry 2 of a 3-entry pool holds h0 and receives
+        # the final state, in place across the pipelined windows
+        pool = torch.zeros((3, hv, 128, 128), device="cuda")
+        pool[2] = h0[0]
+        ws = G.prefill_workspace(inp.cu_seqlens, hv, "cuda", window=32, has_final_state=False)
+        assert G.prefill_schedule(inp.cu_seqlens, hv, ws.numel(), has_final_state=False) == (3, True)
+        o = G.chunk_prefill_slots(*args, pool, dev_i32(np.array([2], np.int32)), init_from_pool=True,
+                                  scale=inp.scale, workspace=ws)
+        torch.cuda.synchronize()
+        assert G.get_device_error() == 0
+        assert np.array_equal(host_bits(o), outs[0][0])
+        assert np.array_equal(pool[2:].cpu().numpy(), outs[0][1])
+        assert not pool[:2].cpu().numpy().any()
 
 
 @pytest.mark.parametrize("case", ["no_decay", "instant_decay", "no_write", "full_write"])

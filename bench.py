@@ -228,6 +228,7 @@ def bench_ours(args, rank, world, device):
                     if args.part == "all" else None)
         other = bench_long_and_varlen(torch, G, device) if args.part == "all" else None
         mixed = bench_mixed(torch, G, device, args) if args.part == "all" else None
+        proj = bench_projections(torch, G, device, flush) if args.part == "all" else None
     if world > 1:
         torch.distributed.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -264,9 +265,10 @@ def bench_ours(args, rank, world, device):
         "long_context": other["long_context"] if other else None,
         "varlen8": other["varlen8"] if other else None,
         "mixed_serving": mixed,
+        "projections": proj,
         "e2e": e2e,
         # conv, prep, chain, norm per step, in the step pass and the prefill-timing pass
-        "gpu_launches": 8 * args.steps + sum(r["launches"] for r in (dec_res, slot_res, other, mixed) if r),
+        "gpu_launches": 8 * args.steps + sum(r["launches"] for r in (dec_res, slot_res, other, mixed, proj) if r),
         "clocks": clk.summary(),
     }
     return res
@@ -417,6 +419,47 @@ def bench_mixed(torch, G, device, args, steps=20):
                                           "achieved": dbytes / (dms * 1e-3) / 1e9, "peak": hbm_peak,
                                           "unit": "GB/s", "frac": dbytes / (dms * 1e-3) / 1e9 / hbm_peak}},
             "steps": steps, "launches": (3 + steps) * launches}
+
+
+def bench_projections(torch, G, device, flush, reps=10):
+    """The layer's two projections at T = 4096 (in: 4096 x 5120 -> 16 480 outputs, q|k|v, z, a,
+    b; out: 4096 x 6144 -> 5120) on their seeded inputs: gdr_linear and, beside it, torch.matmul
+    (cuBLAS) on the same tensors; CUDA events on the launching stream, L2 flushed before each
+    call, median of `reps` after 3 untimed calls."""
+    _, tc_peak, _ = measured_peaks()
+    out = {}
+    for name, (x, w) in (("in_proj", GI.workload_in_proj_T4096()), ("out_proj", GI.workload_out_proj_T4096())):
+        xd, wd = to_dev(torch, x, device), to_dev(torch, w, device)
+        M, K = x.shape
+        N = w.shape[0]
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        y2 = torch.empty_like(y)
+        wt = wd.t()
+
+        def timed(fn):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            ts = []
+            for i in range(reps):
+                flush.fill_(float(i))
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            return statistics.median(ts)
+        ms = timed(lambda: G.linear(xd, wd, y))
+        ms_cublas = timed(lambda: torch.matmul(xd, wt, out=y2))
+        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        out[name] = {"shape": {"M": M, "N": N, "K": K}, "ms": ms, "tflops": tf,
+                     "roofline": {"kernel": "gdr_linear", "bound": "tensor", "achieved": tf, "peak": tc_peak,
+                                  "unit": "TFLOP/s", "frac": tf / tc_peak},
+                     "cublas_ms": ms_cublas, "cublas_tflops": 2.0 * M * N * K / (ms_cublas * 1e-3) / 1e12}
+        del xd, wd, y, y2, wt
+    out["launches"] = 2 * (3 + reps)
+    return out
 
 
 def n_windows(G, cu_host, hv, ws, has_final_state=True):

@@ -16,7 +16,7 @@ import numpy as np
 
 __all__ = [
     "GdrError", "lib", "status_string", "prepare_chunks", "causal_conv", "chunk_prefill",
-    "chunk_prefill_noalloc", "chunk_prefill_slots", "prefill_schedule", "prefill_workspace", "prefill_fused_workspace", "prefill_window",
+    "chunk_prefill_noalloc", "chunk_prefill_slots", "prefill_schedule", "prefill_workspace", "linear", "prefill_fused_workspace", "prefill_window",
     "decode_step", "decode_step_slots", "gated_rmsnorm", "get_device_error", "debug_wait_timeout",
     "HEAD_DIM", "CHUNK",
 ]
@@ -89,11 +89,12 @@ def lib(path: Optional[str] = None):
     L.gdr_chunk_prefill_slots.argtypes = [_vp, _vp, _vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp, _vp,
                                           ctypes.c_float, ctypes.c_int, ctypes.c_int, _vp, _ip, ctypes.c_int,
                                           _vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, ctypes.c_size_t, _vp]
+    L.gdr_linear.argtypes = [_vp, _vp, _vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _vp]
     L.gdr_chunk_prefill_schedule.argtypes = [_ip, ctypes.c_int, ctypes.c_int, ctypes.c_size_t, ctypes.c_int,
                                              ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     for fn in ("gdr_prepare_chunks", "gdr_causal_conv", "gdr_chunk_prefill", "gdr_decode_step",
                "gdr_decode_step_slots", "gdr_gated_rmsnorm", "gdr_get_device_error",
-               "gdr_debug_wait_timeout", "gdr_chunk_prefill_slots", "gdr_chunk_prefill_schedule"):
+               "gdr_debug_wait_timeout", "gdr_chunk_prefill_slots", "gdr_chunk_prefill_schedule", "gdr_linear"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
     return L
@@ -404,6 +405,25 @@ def decode_step_slots(x, conv_w, conv_state_pool, a, b, A_log, dt_bias, state_po
             float(scale), int(hk), int(hv), _ptr(state_pool, f32, "state_pool"), n_slots,
             _ptr(slot, torch.int32, "slot"), _ptr(o, bf, "o"), int(B), _stream(stream, dev)))
     return o
+
+
+def linear(x, w, y=None, stream=None):
+    """y = x w^T: x [M, K], w [N, K] bf16 CUDA tensors (dense rows) -> y [M, N] bf16."""
+    torch = _torch()
+    bf = torch.bfloat16
+    if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[1]:
+        raise ValueError("linear: x [M, K] and w [N, K] with the same K")
+    M, K = x.shape
+    N = w.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=bf, device=x.device)
+    if tuple(y.shape) != (M, N):
+        raise ValueError("linear: y must be [M, N]")
+    dev = _device_of(x, w, y)
+    with torch.cuda.device(dev):
+        _check("gdr_linear", lib().gdr_linear(_ptr(x, bf, "x"), _ptr(w, bf, "w"), _ptr(y, bf, "y"), int(M), int(N),
+                                              int(K), _stream(stream, dev)))
+    return y
 
 
 def gated_rmsnorm(o, z, w=None, eps: float = 1e-6, y=None, stream=None):

@@ -14,7 +14,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["gdr_host.cu", "conv.cu", "rmsnorm.cu", "decode.cu", "prefill.cu", "prefill_noalloc.cu", "diag.cu"]
+SOURCES = ["gdr_host.cu", "conv.cu", "rmsnorm.cu", "decode.cu", "prefill.cu", "prefill_noalloc.cu", "diag.cu",
+           "linear.cu"]
 LIB = os.path.join(HERE, "libgdr.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -76,7 +76,7 @@ const char *gdr_status_string(int status) {
   }
 }
 
-int gdr_abi_version(void) { return 5; }
+int gdr_abi_version(void) { return 6; }
 
 const char *gdr_last_error_string(void) { return gdr::t_last_error_ptr(); }
 
@@ -197,6 +197,20 @@ int gdr_decode_step_slots(const void *x, const void *conv_w, void *conv_state_po
 size_t gdr_chunk_prefill_workspace_size(int n_seqs, int hv, int window_chunks, int has_final_state) {
   if (n_seqs <= 0 || hv <= 0 || window_chunks <= 0) return 0;
   return chunk_prefill_workspace_bytes(n_seqs, hv, window_chunks, has_final_state == 0);
+}
+
+int gdr_linear(const void *x, const void *w, void *y, int64_t M, int64_t N, int64_t K, void *stream) {
+  clear_last_error();
+  if (M < 0 || N <= 0 || K <= 0 || M > (int64_t{1} << 31) || N > (int64_t{1} << 24) || K > (int64_t{1} << 31))
+    return GDR_ERR_SHAPE;
+  if (N % 8 != 0 || K % 8 != 0) return GDR_ERR_SHAPE;   // rows of whole 16-byte chunks
+  if (M == 0) return GDR_OK;
+  if (!x || !w || !y) return GDR_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return GDR_ERR_ALIGN;
+  const size_t yb = static_cast<size_t>(M) * N * 2;
+  if (overlaps(y, yb, x, static_cast<size_t>(M) * K * 2) || overlaps(y, yb, w, static_cast<size_t>(N) * K * 2))
+    return GDR_ERR_ALIAS;
+  return launch_linear(x, w, y, M, N, K, static_cast<cudaStream_t>(stream));
 }
 
 int gdr_chunk_prefill_schedule(const int32_t *cu_host, int n_seqs, int hv, size_t workspace_bytes,

@@ -89,6 +89,8 @@ int launch_chunk_prefill(const void *q, const void *k, const void *v, int64_t qk
                          float eps, void *y, void *workspace, size_t ws_bytes, cudaStream_t s,
                          const PrefillPool *pool = nullptr);
 size_t chunk_prefill_workspace_bytes(int n_seqs, int hv, int window_chunks, bool need_carry);
+// y[M][N] = x[M][K] W[N][K]^T in bf16 with fp32 accumulation (linear.cu)
+int launch_linear(const void *x, const void *w, void *y, int64_t M, int64_t N, int64_t K, cudaStream_t s);
 // window schedule of a prefill call on the current device (windows, chunks per window,
 // whether the next window's prep runs beside the current chain); GDR_ERR_WORKSPACE when
 // not even one chunk per sequence fits

@@ -389,3 +389,31 @@ def workload_mixed_serving(seed=5, n_new=4, rows=64, n_slots=128):
     lengths = varlen_lengths(seed, n_new, 256, 4096)
     return MixedServing(make_core_inputs(seed + 1000, lengths, prenorm_qk=False), new_slot,
                         decode_slot, n_slots)
+
+
+# ---------------------------------------------------------------------------
+# the layer's projections (hidden 5120 -> q|k|v 10 240, z 6144, a, b 48 each; 6144 -> 5120)
+# ---------------------------------------------------------------------------
+
+HIDDEN = 5120
+IN_PROJ_N = 2 * HK * DK + HV * DV + HV * DV + 2 * HV   # q|k|v, z, a, b: 16 480 outputs
+OUT_PROJ_K = HV * DV                                    # the gated norm's output, 6144
+
+
+def make_linear_inputs(seed: int, M: int, N: int, K: int):
+    """Activations x [M, K] ~ N(0, 1) and a weight w [N, K] ~ N(0, 1/K) (a projection at
+    initialisation scale), both bf16 bits.  Draw order: x, w."""
+    rng = _rng(seed)
+    x = _normal_bf16(rng, (M, K))
+    w = _normal_bf16(rng, (N, K), std=1.0 / np.sqrt(K))
+    return x, w
+
+
+def workload_in_proj_T4096(seed=6):
+    """The input projection of the T = 4096 prefill: 4096 tokens x 5120 -> 16 480."""
+    return make_linear_inputs(seed, 4096, IN_PROJ_N, HIDDEN)
+
+
+def workload_out_proj_T4096(seed=7):
+    """The output projection of the T = 4096 prefill: 4096 tokens x 6144 -> 5120."""
+    return make_linear_inputs(seed, 4096, HIDDEN, OUT_PROJ_K)

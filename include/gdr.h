@@ -77,7 +77,7 @@ GDR_API const char *gdr_status_string(int status);
  * changes (2: the conv fused into gdr_chunk_prefill,
  * gdr_chunk_prefill_fused_workspace_size; 3: gdr_decode_step_slots; 4:
  * gdr_chunk_prefill_slots; 5: gdr_chunk_prefill_schedule and the
- * pipelined window schedule). */
+ * pipelined window schedule; 6: gdr_linear). */
 GDR_API int gdr_abi_version(void);
 
 /*
@@ -366,6 +366,22 @@ GDR_API int gdr_chunk_prefill_slots(const void *q, const void *k, const void *v,
                                     const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int n_seqs,
                                     float *state_pool, int n_slots, const int32_t *slot, int init_from_pool,
                                     void *o, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdr_linear -- a projection of the layer: y = x W^T in bf16 with fp32
+ * accumulation, on the tensor cores ("33B 只做 18 层 ...", §2 parameter table:
+ * the hidden state of 5120 is projected to q|k|v (10 240), z (6144), a and b
+ * (48 each), and the gated norm's output (6144) back to 5120).
+ *   x: bf16 [M][K] row-major (rows of the activations, e.g. tokens x hidden)
+ *   w: bf16 [N][K] row-major (the weight as stored for out = in W^T)
+ *   y: bf16 [M][N] row-major, written; must not overlap x or w (GDR_ERR_ALIAS)
+ * y[m][n] = round_bf16(sum_k x[m][k] w[n][k]), the sum in fp32.  N and K must
+ * be multiples of 8 (rows of whole 16-byte chunks) and M, N, K positive with
+ * N <= 2^24 (GDR_ERR_SHAPE); M == 0 is a no-op.  Pointers 16-byte aligned
+ * (GDR_ERR_ALIGN).  Asynchronous on `stream`; a bounded wait that runs out
+ * sets GDR_ERR_TIMEOUT in the device error word and leaves y incomplete.
+ */
+GDR_API int gdr_linear(const void *x, const void *w, void *y, int64_t M, int64_t N, int64_t K, void *stream);
 
 /*
  * gdr_gated_rmsnorm -- gated RMSNorm over rows of d values

@@ -238,6 +238,13 @@ def core_path(inp, heads=None, nthreads=None, chunked=False):
     return round_bf16(o), o, hT
 
 
+def linear(x_bits, w_bits):
+    """One of the layer's projections ("33B 只做 18 层 ...", §2 parameter table: hidden 5120 to
+    q|k|v, z, a, b and 6144 back to 5120): y = x W^T of the bf16 inputs x [M, K] and W [N, K],
+    in fp64, rounded to bf16.  Returns bf16 bits [M, N]."""
+    return round_bf16(bf16_to_f64(x_bits) @ bf16_to_f64(w_bits).T)
+
+
 def split_qkv(y, hk, hv, dk, dv):
     T = y.shape[0]
     q = y[:, : hk * dk].reshape(T, hk, dk)

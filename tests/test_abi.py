@@ -44,7 +44,7 @@ def test_status_strings(L):
     for code in range(1, 10):
         assert G.status_string(code).startswith("GDR_ERR_")
     assert "UNKNOWN" in G.status_string(12345)
-    assert L.gdr_abi_version() == 5
+    assert L.gdr_abi_version() == 6
 
 
 @pytest.mark.parametrize("lengths", [[0], [1], [64], [65, 0, 128, 1, 63], [5000, 3, 64 * 7 + 1],
@@ -169,6 +169,20 @@ def test_wait_self_test_rejects_bad_arguments(L):
     assert L.gdr_debug_wait_timeout(0, 0, FAKE, None) == 2           # no bound
     assert L.gdr_debug_wait_timeout(0, 1 << 40, FAKE, None) == 2     # bound above 2^31
     assert L.gdr_debug_wait_timeout(0, 10, None, None) == 1          # no result word
+
+
+def test_linear_rejects_bad_arguments_on_host(L):
+    f = L.gdr_linear
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 3 + [ctypes.c_void_p]
+    Y = FAKE + (1 << 30)
+    assert f(FAKE, FAKE, None, 4, 8, 8, None) == 1                  # no output
+    assert f(FAKE, FAKE, Y, 4, 12, 8, None) == 2                    # N not a multiple of 8
+    assert f(FAKE, FAKE, Y, 4, 8, 12, None) == 2                    # K not a multiple of 8
+    assert f(FAKE, FAKE, Y, -1, 8, 8, None) == 2
+    assert f(FAKE, FAKE, Y, 4, 0, 8, None) == 2
+    assert f(FAKE, FAKE, Y, 0, 8, 8, None) == 0                     # no rows: nothing to do
+    assert f(ODD, FAKE, Y, 4, 8, 8, None) == 3
+    assert f(FAKE, FAKE, FAKE + 32, 4, 8, 8, None) == 9             # y overlaps x
 
 
 def test_prefill_schedule_on_host(L):

@@ -745,3 +745,59 @@ def test_head_sharded_layer_equals_the_full_layer():
             assert np.array_equal(outs[step], f_outs[step][:, vs]), (s, step)
         assert np.array_equal(st, f_st[:, vs]), s
         assert np.array_equal(cs, f_cs[:, :, ch]), s
+
+
+# ---------------------------------------------------------------------------
+# the layer's projections
+# ---------------------------------------------------------------------------
+
+def _ulp_diff(a_bits, b_bits):
+    """Distance in bf16 units in the last place between two arrays of finite bf16 bits."""
+    def key(u):
+        u = u.astype(np.int32)
+        return np.where(u & 0x8000, 0x8000 - u, u)   # order-preserving map of the bit patterns
+    return np.abs(key(a_bits) - key(b_bits))
+
+
+def _check_linear(got, ref, x, w):
+    """Element by element within the bound of the arithmetic: the GPU sums K products in fp32
+    (error at most K 2^-24 sum_k |x_k w_k|, the usual bound for recursive summation) and both
+    sides round to bf16 (together at most one ulp of the larger value); and rel-L2 <= 1e-3."""
+    g, r = bits_f64(got), bits_f64(ref)
+    K = x.shape[1]
+    mag = np.abs(O.bf16_to_f64(x)) @ np.abs(O.bf16_to_f64(w)).T
+    big = np.maximum(np.abs(g), np.abs(r))
+    ulp = np.exp2(np.floor(np.log2(np.maximum(big, 1e-300))) - 7)   # bf16: 8 significant bits
+    assert np.all(np.abs(g - r) <= ulp + K * 2.0 ** -24 * mag)
+    assert rel_l2(g, r) <= 1e-3
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 600, 512), (128, 48, 5120), (1, 8, 8), (257, 264, 136), (129, 256, 64)])
+def test_linear_matches_oracle(M, N, K):
+    """y = x W^T against the fp64 product rounded to bf16, element by element: ragged tiles in M
+    (tile 128), N (tile 256) and K (step 64) and the a/b projection's N = 48.  The GPU sums in
+    fp32, so an output may round to a neighbouring bf16 value (rarely; further only where the
+    sum cancels to far below its terms)."""
+    x, w = GI.make_linear_inputs(M + 7 * N + 13 * K, M, N, K)
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    G.linear(dev_bf16(x), dev_bf16(w), y)
+    torch.cuda.synchronize()
+    assert G.get_device_error() == 0
+    got, ref = host_bits(y), O.linear(x, w)
+    _check_linear(got, ref, x, w)
+    assert np.mean(_ulp_diff(got, ref) > 0) < 0.02
+
+
+@pytest.mark.parametrize("which", ["in_proj", "out_proj"])
+def test_linear_projections_full_size_sampled_rows(which):
+    """The two projections of the T = 4096 prefill at full size (4096 x 5120 -> 16 480 and
+    4096 x 6144 -> 5120), 40 rows (including the first and last) against the oracle."""
+    x, w = GI.workload_in_proj_T4096() if which == "in_proj" else GI.workload_out_proj_T4096()
+    M, N = x.shape[0], w.shape[0]
+    y = G.linear(dev_bf16(x), dev_bf16(w))
+    torch.cuda.synchronize()
+    assert G.get_device_error() == 0
+    rows = np.unique(np.concatenate([[0, M - 1], np.random.default_rng(8).choice(M, 38, replace=False)]))
+    got = y[torch.from_numpy(rows).cuda()].view(torch.int16).cpu().numpy().view(np.uint16)
+    ref = O.linear(x[rows], w)
+    _check_linear(got, ref, x[rows], w)

@@ -613,3 +613,24 @@ def test_full_path_norm_reads_the_bf16_output():
     out = O.full_path(inp)
     y = O.round_bf16(O.gated_rmsnorm(O.bf16_to_f64(out["o"]), O.bf16_to_f64(inp.z), inp.norm_w, inp.eps))
     assert np.array_equal(out["y"], y)
+
+
+def test_linear_is_the_product_written_out():
+    """The projection oracle against explicit sums on a tiny case, including a column where the
+    bf16 rounding of the sum is decided by the last term (so a dropped term or a transposed
+    operand changes bits)."""
+    r = np.random.default_rng(3)
+    x = GI.f32_to_bf16_bits(r.standard_normal((3, 5)).astype(np.float32))
+    w = GI.f32_to_bf16_bits(r.standard_normal((4, 5)).astype(np.float32))
+    xf, wf = O.bf16_to_f64(x), O.bf16_to_f64(w)
+    want = np.zeros((3, 4))
+    for m in range(3):
+        for n in range(4):
+            acc = 0.0
+            for k in range(5):
+                acc += xf[m, k] * wf[n, k]
+            want[m, n] = acc
+    assert np.array_equal(O.linear(x, w), O.round_bf16(want))
+    # x = e_0, W = rows of distinct values: y picks column 0 of W, exactly
+    e = GI.f32_to_bf16_bits(np.eye(2, 5, dtype=np.float32))
+    assert np.array_equal(O.linear(e, w), w[:, :2].T)

@@ -2,7 +2,7 @@
 """Benchmark of the gated delta-rule layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--part all|prefill|decode] [--decode-steps S] [--decode-slots]
+                    [--part all|prefill|decode|proj] [--decode-steps S] [--decode-slots]
                     [--no-cpu-baseline]
 
 A step of the default workload is one pass of the prefill path of one layer
@@ -14,8 +14,9 @@ slot-indexed form (64 rows on a pool of 128 cached states) under
 "decode_slots".  Inputs are seeded
 synthetic tensors (gdr_inputs) with the layer's shapes; there are no weights.
 
-`--part prefill` / `--part decode` run one of the two paths alone (for
-profiling); the default `all` is the benchmark.
+`--part prefill` / `--part decode` / `--part proj` run one path alone (the
+projections: `gdr_linear` beside cuBLAS) for profiling; the default `all` is the
+benchmark.
 
 Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs its own
 replica of the workload (the path has no cross-GPU exchange) and the value is
@@ -759,7 +760,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--part", choices=["all", "prefill", "decode"], default="all")
+    ap.add_argument("--part", choices=["all", "prefill", "decode", "proj"], default="all")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--decode-slots", action="store_true",
                     help="with --part decode: the slot-indexed form on a pool of 128 cached states")
@@ -790,6 +791,15 @@ def main():
         for line in bench_sweep(torch, G, device):
             if rank == 0:
                 print(json.dumps(line), flush=True)
+        return
+    if args.part == "proj":
+        torch.cuda.set_device(device)
+        import gated_delta_rule_63_b200 as G
+        G.lib()
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+        res = bench_projections(torch, G, device, flush, reps=max(3, args.steps))
+        if rank == 0:
+            print(json.dumps(res), flush=True)
         return
     if args.part == "decode":
         torch.cuda.set_device(device)

@@ -801,3 +801,60 @@ def test_linear_projections_full_size_sampled_rows(which):
     got = y[torch.from_numpy(rows).cuda()].view(torch.int16).cpu().numpy().view(np.uint16)
     ref = O.linear(x[rows], w)
     _check_linear(got, ref, x[rows], w)
+
+
+def _layer_ours(h, w_in, conv_w, A_log, dt_bias, w_out, cu, hk, hv):
+    """Our kernels end to end: projection -> conv -> recurrence -> gated norm -> projection
+    (the normed output and the output projection's result, both bf16 bits)."""
+    T = h.shape[0]
+    c = 2 * hk * 128 + hv * 128
+    yi = G.linear(dev_bf16(h), dev_bf16(w_in))
+    x = yi[:, :c].contiguous()
+    z = yi[:, c:c + hv * 128].contiguous().view(T, hv, 128)
+    a = yi[:, c + hv * 128:c + hv * 128 + hv].contiguous()
+    b = yi[:, c + hv * 128 + hv:].contiguous()
+    conv_y = torch.empty_like(x)
+    G.causal_conv(x, dev_bf16(conv_w), dev_i32(cu), cu, None, None, conv_y)
+    q = conv_y[:, :hk * 128].view(T, hk, 128)
+    k = conv_y[:, hk * 128:2 * hk * 128].view(T, hk, 128)
+    v = conv_y[:, 2 * hk * 128:].view(T, hv, 128)
+    o = G.chunk_prefill(q, k, v, a, b, dev_f32(A_log), dev_f32(dt_bias), dev_i32(cu), cu)
+    y = G.gated_rmsnorm(o, z, None, 1e-6)
+    out = G.linear(y.view(T, hv * 128), dev_bf16(np.ascontiguousarray(w_out)))
+    torch.cuda.synchronize()
+    return host_bits(y).reshape(T, hv * 128), host_bits(out)
+
+
+def test_layer_with_projections_sharded_by_heads():
+    """The whole layer with its projections through our kernels, unsharded and as two head
+    shards (gated_delta_rule_63_b200.shard: 8 key / 24 value heads each, the shards run one
+    after the other on this GPU): each shard's normed output equals the unsharded one's columns
+    bit for bit; the sum of the shards' out-projection partials (the all-reduce of a two-GPU
+    run) matches the unsharded output, and both match the fp64 oracle of the whole layer."""
+    from gated_delta_rule_63_b200.shard import head_shard
+    import tests.test_head_shard as TH
+    h, w_in, w_out, conv_w, A_log, dt_bias = TH._layer_inputs()
+    cu = GI.cu_seqlens_from_lengths(TH.LENGTHS)
+    y_full, out_full = _layer_ours(h, w_in, conv_w, A_log, dt_bias, w_out, cu, 16, 48)
+    assert G.get_device_error() == 0
+    summed, bound = np.zeros(out_full.shape), np.zeros(out_full.shape)
+    wf = bits_f64(w_out)
+    for r in range(2):
+        s = head_shard(r, 2)
+        y, part = _layer_ours(h, w_in[s.in_rows], conv_w[s.conv_channels], A_log[s.heads], dt_bias[s.heads],
+                              w_out[:, s.out_cols], cu, s.hk, s.hv)
+        assert np.array_equal(y, y_full[:, s.out_cols]), r
+        summed += bits_f64(part)
+        # each partial: fp32 sum of 3072 products, rounded to bf16
+        mag = np.abs(bits_f64(y)) @ np.abs(wf[:, s.out_cols]).T
+        bound += 2.0 ** -8 * np.abs(bits_f64(part)) + 3072 * 2.0 ** -24 * mag
+    # the partials sum to the exact product of the (shared) normed output and the weight, within
+    # their roundings; so does the unsharded output, rounded once
+    exact = bits_f64(y_full) @ wf.T
+    assert np.all(np.abs(summed - exact) <= bound + 1e-30)
+    full_mag = np.abs(bits_f64(y_full)) @ np.abs(wf).T
+    assert np.all(np.abs(bits_f64(out_full) - exact) <= 2.0 ** -8 * np.abs(exact) + 6144 * 2.0 ** -24 * full_mag)
+    ref_y = TH._normed(h, w_in, conv_w, A_log, dt_bias, 16, 48)
+    assert rel_l2(bits_f64(y_full), bits_f64(ref_y)) <= TOL_BF16
+    ref_out = O.linear(ref_y, w_out)
+    assert rel_l2(bits_f64(out_full), bits_f64(ref_out)) <= TOL_BF16

@@ -980,6 +980,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // ---- P = [W_hi; Q] [H_hi | H_lo]: Q H0 in lanes 64..127 -------------------------------
         if (!chain_wait(bar_pw, ph, abort_flag, p.err)) break;
         if (!chain_wait(full_qw + 8 * s, par, abort_flag, p.err)) break;   // (landed: PW read it)
+        PTIME_T(1 + cw, 31, 32 * kCopyWarp);
         tc_fence_after();
         {
           const uint32_t id1 = idesc_bf16(128, 128, false, true);
@@ -991,10 +992,14 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           }
           mma_commit(bar_p);
         }
+        PTIME_T(1 + cw, 26, 32 * kCopyWarp);
         // ---- O = [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi (rows in lanes 64..127) --------
         if (!chain_wait(bar_h, ph, abort_flag, p.err)) break;             // U tiles written, K^T U' first
+        PTIME_T(1 + cw, 27, 32 * kCopyWarp);
         if (cw > 0 && !chain_wait(o_free, ph ^ 1, abort_flag, p.err)) break;   // the previous O is read
+        PTIME_T(1 + cw, 9, 32 * kCopyWarp);
         if (!chain_wait(full_mq + 8 * s, par, abort_flag, p.err)) break;
+        PTIME_T(1 + cw, 10, 32 * kCopyWarp);
         tc_fence_after();
         {
           const uint32_t idO1 = idesc_bf16(128, 128, false, true), idO2 = idesc_bf16(128, 64, false, true);
@@ -1008,13 +1013,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                      1);
           mma_commit(bar_o);
         }
+        PTIME_T(1 + cw, 13, 32 * kCopyWarp);
         // ---- stage s takes chunk cw + 2 once every product of chunk cw has read it (PW,
         // waited above; P and O, this thread's, complete with bar_o) -----------------------------
         if (cw + 2 < nw) {
           if (!chain_wait(bar_o, ph, abort_flag, p.err)) break;
+          PTIME_T(1 + cw, 14, 32 * kCopyWarp);
           load_qw(cw + 2);
           load_k(cw + 2);
           load_mq(cw + 2);
+          PTIME_T(1 + cw, 15, 32 * kCopyWarp);
         }
       }
       // its products complete before tensor memory is released; after a timeout the
@@ -1184,6 +1192,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             mbar_arrive_expect_tx(sbase + C_OFF_PBAR + 8 * (cw & 1), 64 * 4);
         }
         chain_wait(bar_o, ph, abort_flag, p.err);
+        PTIME_T(1 + cw, 2, 64);
         __syncwarp();
         tc_fence_after();
 #pragma unroll

@@ -50,6 +50,32 @@ struct ConvParams {
   int *err;
 };
 
+// SiLU of a pair of values, x / (1 + e^-x), with e^-x = 2^(-x log2 e) from the MUFU's base-2
+// exponential and the quotient from its reciprocal; the multiplies and the add run two-wide.
+// Very negative x gives an infinite exponential, a zero reciprocal and a signed zero, the limit.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float2 silu2(float2 x) {
+  constexpr float kNegLog2e = -1.4426950408889634f;   // -log2(e)
+  const float2 t = __fmul2_rn(x, make_float2(kNegLog2e, kNegLog2e));
+  const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)), make_float2(1.0f, 1.0f));
+  return __fmul2_rn(x, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+// 8 bf16 (one 16-byte vector) as four pairs of floats
+__device__ __forceinline__ void unpack8x2(const uint4 &u, float2 *f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+
 // sequence containing token t: largest n with cu[n] <= t (skipping empty ones)
 __device__ int seq_of(const int32_t *cu, int n_seqs, int t) {
   int lo = 0, hi = n_seqs - 1;
@@ -115,34 +141,42 @@ causal_conv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
     const uint32_t tbuf = sbase + buf * kBufBytes + cg * 16;
     const bool ok = mbar_wait(bar0 + 8 * buf, parity, p.err);
     if (ok && c0 < C && tb < p.total) {
-      float w[4][8];
+      float2 w[4][4];   // tap j, channel pair cp
       {   // w is [C][4]: channels c0..c0+7 occupy 32 contiguous bf16
         const uint4 *wp = reinterpret_cast<const uint4 *>(p.w + static_cast<size_t>(c0) * 4);
         float tmp[32];
 #pragma unroll
         for (int i = 0; i < 4; ++i) unpack8(__ldg(wp + i), tmp + 8 * i);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
+        for (int cp = 0; cp < 4; ++cp)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) w[j][ch] = tmp[ch * 4 + j];
+          for (int j = 0; j < 4; ++j) w[j][cp] = make_float2(tmp[8 * cp + j], tmp[8 * cp + 4 + j]);
       }
+      // sum_j w_j x_j in tap order (a product, then three fused multiply-adds), then SiLU
+      auto conv2 = [&](const float2 &x0, const float2 &x1, const float2 &x2, const float2 &x3, int cp) {
+        float2 acc = __fmul2_rn(w[0][cp], x0);
+        acc = __ffma2_rn(w[1][cp], x1, acc);
+        acc = __ffma2_rn(w[2][cp], x2, acc);
+        acc = __ffma2_rn(w[3][cp], x3, acc);
+        return silu2(acc);
+      };
       auto row = [&](int t) { return ld_shared16(tbuf + (t - row0) * kRowBytes); };   // token t's 8 inputs
       int n = seq_of(p.cu, p.n_seqs, tb);
       int seq_start = __ldg(p.cu + n), seq_end = __ldg(p.cu + n + 1);
       if (tb - 3 >= seq_start && tb + 8 < seq_end) {
         // ---- inside one sequence, not its last token: no state, no boundary ----
-        float xw[4][8];
+        float2 xw[4][4];   // sliding window of 4 token rows, channel pairs
 #pragma unroll
-        for (int j = 0; j < 3; ++j) unpack8(row(tb - 3 + j), xw[j]);
+        for (int j = 0; j < 3; ++j) unpack8x2(row(tb - 3 + j), xw[j]);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          unpack8(row(tb + i), xw[(i + 3) & 3]);
+          unpack8x2(row(tb + i), xw[(i + 3) & 3]);
           float out[8];
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const float acc = w[0][ch] * xw[i & 3][ch] + w[1][ch] * xw[(i + 1) & 3][ch] +
-                              w[2][ch] * xw[(i + 2) & 3][ch] + w[3][ch] * xw[(i + 3) & 3][ch];
-            out[ch] = silu_fast(acc);
+          for (int cp = 0; cp < 4; ++cp) {
+            const float2 y2 = conv2(xw[i & 3][cp], xw[(i + 1) & 3][cp], xw[(i + 2) & 3][cp], xw[(i + 3) & 3][cp], cp);
+            out[2 * cp] = y2.x;
+            out[2 * cp + 1] = y2.y;
           }
           *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(tb + i) * C + c0) = pack8x2(out);
         }
@@ -164,19 +198,16 @@ causal_conv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                   p.cs_in + (static_cast<size_t>(n) * 3 + (3 - (seq_start - pos))) * C + c0);
             return make_uint4(0, 0, 0, 0);
           };
-          float acc[8];
+          float2 xv[4][4];
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) acc[ch] = 0.0f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float xv[8];
-            unpack8(tap(t - 3 + j), xv);
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) acc[ch] += w[j][ch] * xv[ch];
-          }
+          for (int j = 0; j < 4; ++j) unpack8x2(tap(t - 3 + j), xv[j]);
           float out[8];
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) out[ch] = silu_fast(acc[ch]);
+          for (int cp = 0; cp < 4; ++cp) {
+            const float2 y2 = conv2(xv[0][cp], xv[1][cp], xv[2][cp], xv[3][cp], cp);
+            out[2 * cp] = y2.x;
+            out[2 * cp + 1] = y2.y;
+          }
           *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(t) * C + c0) = pack8x2(out);
           if (t == seq_end - 1 && p.cs_out) {   // last token: the last three inputs are the new conv state
 #pragma unroll

@@ -111,10 +111,10 @@ static_assert(C_SMEM <= 232448, "chain shared memory exceeds 227 KB");
 static_assert((C_QW_KB | C_OFF_K | C_OFF_MQ | C_STAGE | C_OFF_H | C_OFF_U) % 1024 == 0,
               "swizzled tiles need 1 KB alignment");
 constexpr uint32_t C_TM_COLS = 512;
-constexpr uint32_t C_COL_P = 0;      // [W_hi; Q] [H_hi | H_lo]: lanes 64..127 hold Q H0 (the W rows go unread)
+constexpr uint32_t C_COL_P = 0;      // M = 64: Q [H_hi | H_lo], Q row 16 q + i in lane 32 q + i
 constexpr uint32_t C_COL_PW = 128;   // M = 64: W_hi [H_hi | H_lo] + W_lo [H_hi | -], W row 16 q + i in lane 32 q + i
 constexpr uint32_t C_COL_H = 256;    // K^T [U'_hi | U'_lo], lanes = dk
-constexpr uint32_t C_COL_O = 384;    // [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi, lanes 64..127
+constexpr uint32_t C_COL_O = 384;    // M = 64: Mq_hi [U_hi | U_lo] + Mq_lo [U_hi | -], row 16 q + i in lane 32 q + i
 
 #ifdef GDR_PREFILL_TIMING
 // diagnostic build: step timestamps; prep CTA (0,0,0) in row 0, chain CTA
@@ -735,14 +735,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // holds rows 32 (w & 3) .. + 31 (its TMEM lane quarter), columns
 // 32 (w >> 2) .. + 31.  Per chunk:
 //   PW = W_hi [H_hi | H_lo] + W_lo [H_hi | -]   (M = 64)             tensor cores
-//   P  = [W_hi; Q] [H_hi | H_lo]   (for Q H0, after PW)               tensor cores
+//   P  = Q [H_hi | H_lo]   (M = 64, for Q H0, after PW)               tensor cores
 //   U  = Ut - W H0,  U' = U e^(gamma_L - gamma) / |k|                warps 0..7
 //   (an M = 64 product puts 16 W rows on each of the four TMEM lane quarters, so the U
 //   phase runs on all four SM sub-partitions, 16 rows x 32 columns a warp)
 //   H' = K^T [U'_hi | U'_lo]                                         tensor cores
 //   H  = e^gamma_L H + H'                                            warps 0..7
-//   O  = [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi              tensor cores
-//   o  = scale (e^gamma / |q| Q H0 + O)                              warps 2, 3, 6, 7 (lanes 64..127)
+//   O  = Mq_hi [U_hi | U_lo] + Mq_lo [U_hi | -]   (M = 64)           tensor cores
+//   o  = scale (e^gamma / |q| Q H0 + O)                              warps 0..7
+//   (the output products take the U phase's layout: each warp reads 16 output rows x 32
+//   columns of its lane quarter, so the output and the fused norm run on all four SM
+//   sub-partitions)
 // N = 128 products stack the hi and lo parts of one operand side by side, so
 // each fp32 product takes two MMA groups instead of three.  Warp 8 issues the
 // products on the state's critical path (PW, K^T U'); warp 9 issues the output's
@@ -841,9 +844,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     iss_mq = cw + 1;
   };
   if (ctrl && lane == 0) {
-    // full x 6, products x 3, o_free (4 output warps), h_ready (8 warps), u_ready (8 warps), drain, PW,
+    // full x 6, products x 3, o_free (8 warps), h_ready (8 warps), u_ready (8 warps), drain, PW,
     // the copy warp's drain
-    const uint32_t counts[15] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 4, 8, 8, 1, 1, 1};
+    const uint32_t counts[15] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 8, 8, 8, 1, 1, 1};
     for (int i = 0; i < 15; ++i) mbar_init(bars + 8 * i, counts[i]);
     if (kNorm) {   // the other slice's 64 row sums: 256 transaction bytes per chunk
       mbar_init(sbase + C_OFF_PBAR, 1);
@@ -854,8 +857,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   }
   const int q4 = warp & 3, ch = (warp >> 2) & 1;     // lane quarter, column half
   const int row = 32 * q4 + lane;                    // TMEM lane / dk row of the state
-  const bool wrow = row < 64;                        // W rows (state side) vs Q rows (output side)
-  const int r = row & 63;                            // chunk row
 
   // ---- the state: row `row`, columns 32 ch .. 32 ch + 31 of this dv slice --------------
   float hreg[32];
@@ -977,23 +978,23 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const int s = cw & 1;
         const uint32_t par = (cw >> 1) & 1, ph = cw & 1;
         const uint32_t st = sbase + s * C_STAGE;
-        // ---- P = [W_hi; Q] [H_hi | H_lo]: Q H0 in lanes 64..127 -------------------------------
+        // ---- P = Q [H_hi | H_lo] (M = 64): Q H0, row 16 q + i in lane 32 q + i ------------------
         if (!chain_wait(bar_pw, ph, abort_flag, p.err)) break;
         if (!chain_wait(full_qw + 8 * s, par, abort_flag, p.err)) break;   // (landed: PW read it)
         PTIME_T(1 + cw, 31, 32 * kCopyWarp);
         tc_fence_after();
         {
-          const uint32_t id1 = idesc_bf16(128, 128, false, true);
+          const uint32_t id1 = idesc_bf16(64, 128, false, true);
           const uint64_t bh = sdesc(sbase + C_OFF_H, BLK128, 1024);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff = (kk >> 2) * C_QW_KB + 64 * 128 + (kk & 3) * 32;
+          for (int kk = 0; kk < 8; ++kk) {   // A = the Q rows 128..191 of the k-block
+            const uint32_t aoff = (kk >> 2) * C_QW_KB + 128 * 128 + (kk & 3) * 32;
             mma_bf16(tmem + C_COL_P, sdesc(st + aoff, 16, 1024), bh + ((kk * 2048) >> 4), id1, kk > 0);
           }
           mma_commit(bar_p);
         }
         PTIME_T(1 + cw, 26, 32 * kCopyWarp);
-        // ---- O = [Mq_lo; Mq_hi] [U_hi | U_lo] + [K; Mq_lo] U_hi (rows in lanes 64..127) --------
+        // ---- O = Mq_hi [U_hi | U_lo] + Mq_lo [U_hi | -] (M = 64, rows as in P) -------------------
         if (!chain_wait(bar_h, ph, abort_flag, p.err)) break;             // U tiles written, K^T U' first
         PTIME_T(1 + cw, 27, 32 * kCopyWarp);
         if (cw > 0 && !chain_wait(o_free, ph ^ 1, abort_flag, p.err)) break;   // the previous O is read
@@ -1002,15 +1003,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         PTIME_T(1 + cw, 10, 32 * kCopyWarp);
         tc_fence_after();
         {
-          const uint32_t idO1 = idesc_bf16(128, 128, false, true), idO2 = idesc_bf16(128, 64, false, true);
+          const uint32_t idO1 = idesc_bf16(64, 128, false, true), idO2 = idesc_bf16(64, 64, false, true);
           const uint64_t bo = sdesc(sbase + C_OFF_U, BLK64, 1024);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO1, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)   // A = Mq_hi
+            mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + BLK64 + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO1,
+                     kk > 0);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ - BLK64 + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO2,
-                     1);
+          for (int kk = 0; kk < 4; ++kk)   // A = Mq_lo, into the U_hi half
+            mma_bf16(tmem + C_COL_O, sdesc(st + C_OFF_MQ + kk * 32, 16, 1024), bo + ((kk * 2048) >> 4), idO2, 1);
           mma_commit(bar_o);
         }
         PTIME_T(1 + cw, 13, 32 * kCopyWarp);
@@ -1043,8 +1044,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     __syncwarp();
     if (lane == 0) mbar_arrive(h_ready);
 
-    // U phase (every state warp): W row ru = 16 q4 + (lane & 15) of the M = 64 product,
-    // dv columns cu .. cu + 15 of this slice (16x32bx2 TMEM loads)
+    // U phase and output (every state warp): chunk row ru = 16 q4 + (lane & 15) of the M = 64
+    // products (W rows for U, Q rows for o), dv columns cu .. cu + 15 of this slice (16x32bx2
+    // TMEM loads)
     const int ru = 16 * q4 + (lane & 15), cu = 32 * ch + 16 * (lane >> 4);
     // per-chunk data read into registers one chunk ahead: Ut (row ru) and scalars
     float ut[16];
@@ -1057,16 +1059,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         ut[4 * j] = v4.x; ut[4 * j + 1] = v4.y; ut[4 * j + 2] = v4.z; ut[4 * j + 3] = v4.w;
       }
     };
-    // gamma and 1/|k| of row ru, gamma and 1/|q| of output row r, gamma_(L-1)
-    float nx_gu = 0.0f, nx_ku = 0.0f, nx_g = 0.0f, nx_s = 0.0f, nx_gL = 0.0f;
+    // gamma, 1/|q| and 1/|k| of row ru, gamma_(L-1)
+    float nx_gu = 0.0f, nx_ku = 0.0f, nx_s = 0.0f, nx_gL = 0.0f;
     auto load_sc = [&](int cw) {
       const float *sc = reinterpret_cast<const float *>(ws_record(p, n, h, cw) + WS_SC);
       nx_gu = sc[ru];
+      nx_s = sc[64 + ru];
       nx_ku = sc[128 + ru];
-      if (!wrow) {
-        nx_g = sc[r];
-        nx_s = sc[64 + r];
-      }
       nx_gL = sc[63];
     };
     if (nw > 0) {
@@ -1074,11 +1073,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       load_ut(0);
     }
 
-    float oreg[32];   // e^gamma / |q| Q H0 part of o (output rows)
+    float oreg[16];   // o of row ru, columns cu .. cu + 15
     for (int cw = 0; cw < nw; ++cw) {
       const uint32_t ph = cw & 1;
       const int t0 = t0_of(cw), L = min(C, seq_end - t0);
-      const float g_u = nx_gu, k_u = nx_ku, g_r = nx_g, sb = nx_s, gL = nx_gL;
+      const float g_u = nx_gu, k_u = nx_ku, sb = nx_s, gL = nx_gL;
       if (cw + 1 < nw) load_sc(cw + 1);
       PTIME(1 + cw, 0);
 
@@ -1122,21 +1121,19 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         PTIME_T(1 + cw, 12, 64);
         if (cw + 1 < nw) load_ut(cw + 1);
       }
-      if (!wrow) {
-        // ---- Q H0 part of the output (output rows) ------------------------------------------
+      {
+        // ---- Q H0 part of the output (row ru); P read the H tiles, which write_h overwrites ---
         chain_wait(bar_p, ph, abort_flag, p.err);
         __syncwarp();
         tc_fence_after();
-        const float f = p.scale * __expf(g_r) * sb;
+        const float f = p.scale * __expf(g_u) * sb;
+        const uint32_t tp = tmem + (static_cast<uint32_t>(32 * q4) << 16) + C_COL_P + 32 * ch;
+        float pa[16], pb[16];
+        tmem_ld16x2(tp, pa);        // Q H_hi
+        tmem_ld16x2(tp + 64, pb);   // Q H_lo
+        tmem_wait_ld();
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float pa[16], pb[16];
-          tmem_ld16(tl + C_COL_P + 16 * hh, pa);
-          tmem_ld16(tl + C_COL_P + 64 + 16 * hh, pb);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) oreg[16 * hh + j] = (pa[j] + pb[j]) * f;
-        }
+        for (int j = 0; j < 16; ++j) oreg[j] = (pa[j] + pb[j]) * f;
       }
 
       // ---- H <- e^gamma_L H + K^T U' ------------------------------------------------------------
@@ -1162,12 +1159,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             hreg[16 * hh + 2 * j + 1] = hn.y;
           }
         }
-        // P (the copy warp's product, not covered by bar_h) reads the H tiles too: the output
-        // warps waited for it before reading Q H0
-        if (wrow) {
-          chain_wait(bar_p, ph, abort_flag, p.err);
-          __syncwarp();
-        }
         write_h();
       }
       PTIME(1 + cw, 18);
@@ -1180,73 +1171,76 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       PTIME_T(1 + cw, 20, 64);
       PTIME_T(1 + cw, 21, 224);
 
-      // ---- output rows: o = scale (e^gamma / |q| Q H0 + O), overlapping the next chunk ---------
-      if (!wrow) {
-        uint4 zr[kNorm ? 4 : 1];   // the norm's gate, this thread's 32 columns of row r
-        const size_t orow = (static_cast<size_t>(t0 + r) * p.hv + h) * D + slice * N + 32 * ch;
+      // ---- output: o = scale (e^gamma / |q| Q H0 + O), row ru, overlapping the next chunk ------
+      {
+        uint4 zr[kNorm ? 2 : 1];   // the norm's gate, this thread's 16 columns of row ru
+        const size_t orow = (static_cast<size_t>(t0 + ru) * p.hv + h) * D + slice * N + cu;
         if (kNorm) {
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4)
-            zr[c4] = r < L ? __ldg(reinterpret_cast<const uint4 *>(p.z + orow) + c4) : make_uint4(0, 0, 0, 0);
-          if (tid == 64)   // this chunk's 64 row sums from the other slice: 256 bytes
+          for (int c2 = 0; c2 < 2; ++c2)
+            zr[c2] = ru < L ? __ldg(reinterpret_cast<const uint4 *>(p.z + orow) + c2) : make_uint4(0, 0, 0, 0);
+          if (tid == 0)   // this chunk's 64 row sums from the other slice: 256 bytes
             mbar_arrive_expect_tx(sbase + C_OFF_PBAR + 8 * (cw & 1), 64 * 4);
         }
         chain_wait(bar_o, ph, abort_flag, p.err);
         PTIME_T(1 + cw, 2, 64);
         __syncwarp();
         tc_fence_after();
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+        {
+          const uint32_t to = tmem + (static_cast<uint32_t>(32 * q4) << 16) + C_COL_O + 32 * ch;
           float oa[16], ob[16];
-          tmem_ld16(tl + C_COL_O + 16 * hh, oa);
-          tmem_ld16(tl + C_COL_O + 64 + 16 * hh, ob);
+          tmem_ld16x2(to, oa);        // Mq_hi U_hi + Mq_lo U_hi
+          tmem_ld16x2(to + 64, ob);   // Mq_hi U_lo
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) oreg[16 * hh + j] += p.scale * (oa[j] + ob[j]);
+          for (int j = 0; j < 16; ++j) oreg[j] += p.scale * (oa[j] + ob[j]);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(o_free);
         if (kNorm) {
-          // fused gated RMSNorm: the row's 128 values are split over this thread, the thread of
-          // the other column half and the two threads of the other dv slice (cluster peer)
+          // fused gated RMSNorm: the row's 128 values are split over this thread (16), its
+          // partner 16 lanes away (16), the two threads of the other column half (32) and the
+          // four threads of the other dv slice (64, cluster peer)
           const uint32_t pb = cw & 1;
           float ss = 0.0f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             oreg[j] = round_bf16(oreg[j]);   // the norm reads the bf16 o
             ss += oreg[j] * oreg[j];
           }
+          ss += __shfl_xor_sync(0xffffffffu, ss, 16);
           float *s_ss = reinterpret_cast<float *>(smem + C_OFF_NORM) + pb * 128;
-          s_ss[ch * 64 + r] = ss;
-          named_sync(1, 128);   // the four output warps
-          const float own = s_ss[r] + s_ss[64 + r];
-          const uint32_t peer_slot = smem_u32(smem + C_OFF_PEER) + (pb * 64 + r) * 4;
-          if (ch == 0) st_async_remote(map_peer(peer_slot, peer), own, map_peer(sbase + C_OFF_PBAR + 8 * pb, peer));
+          if (lane < 16) s_ss[ch * 64 + ru] = ss;
+          named_sync(1, 256);   // the eight state warps
+          const float own = s_ss[ru] + s_ss[64 + ru];
+          const uint32_t peer_slot = smem_u32(smem + C_OFF_PEER) + (pb * 64 + ru) * 4;
+          if (ch == 0 && lane < 16)
+            st_async_remote(map_peer(peer_slot, peer), own, map_peer(sbase + C_OFF_PBAR + 8 * pb, peer));
           PTIME_T(1 + cw, 29, 64);
           float total = own;
           if (chain_wait_cluster(sbase + C_OFF_PBAR + 8 * pb, (cw >> 1) & 1, abort_flag, p.err))
-            total += reinterpret_cast<const float *>(smem + C_OFF_PEER)[pb * 64 + r];
+            total += reinterpret_cast<const float *>(smem + C_OFF_PEER)[pb * 64 + ru];
           PTIME_T(1 + cw, 30, 64);
           const float inv = 1.0f / sqrtf(total * (1.0f / 128.0f) + p.eps);
-          if (r < L) {
-            const int col0 = slice * N + 32 * ch;
+          if (ru < L) {
+            const int col0 = slice * N + cu;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c2 = 0; c2 < 2; ++c2) {
               float zf[8], yv[8];
-              unpack8(zr[c4], zf);
+              unpack8(zr[c2], zf);
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
-                const float wv = p.norm_w ? __ldg(p.norm_w + col0 + 8 * c4 + e) : 1.0f;
-                yv[e] = oreg[8 * c4 + e] * inv * wv * silu_fast(zf[e]);
+                const float wv = p.norm_w ? __ldg(p.norm_w + col0 + 8 * c2 + e) : 1.0f;
+                yv[e] = oreg[8 * c2 + e] * inv * wv * silu_fast(zf[e]);
               }
-              *reinterpret_cast<uint4 *>(p.y + orow + 8 * c4) = pack8x2(yv);
-              if (p.o) *reinterpret_cast<uint4 *>(p.o + orow + 8 * c4) = pack8x2(oreg + 8 * c4);
+              *reinterpret_cast<uint4 *>(p.y + orow + 8 * c2) = pack8x2(yv);
+              if (p.o) *reinterpret_cast<uint4 *>(p.o + orow + 8 * c2) = pack8x2(oreg + 8 * c2);
             }
           }
-        } else if (r < L) {
+        } else if (ru < L) {
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) *reinterpret_cast<uint4 *>(p.o + orow + 8 * c4) = pack8x2(oreg + 8 * c4);
+          for (int c2 = 0; c2 < 2; ++c2) *reinterpret_cast<uint4 *>(p.o + orow + 8 * c2) = pack8x2(oreg + 8 * c2);
         }
         PTIME_T(1 + cw, 7, 64);
       }

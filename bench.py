@@ -53,9 +53,9 @@ B_FUSED = CX * 2 + 2 * GI.HV * 2 + 2 * GI.HV * GI.DV * 2 # x, a, b, z read + y w
 STATE_BYTES = GI.HV * GI.DK * GI.DV * 4                  # one sequence's fp32 state
 
 # DRAM bytes (read + written) per launch from one ncu capture of the current kernels:
-# prefill = prep + state chain on full_T4096 (283.9 + 327.6 MB), decode = one B=64 step
+# prefill = prep + state chain on full_T4096 (283.9 + 327.8 MB), decode = one B=64 step
 # (a replayed launch, partly served from L2), and the same step in the slot-indexed form
-TRAFFIC_PREFILL = 611_426_304
+TRAFFIC_PREFILL = 611_689_472
 TRAFFIC_DECODE = 355_618_304
 TRAFFIC_DECODE_SLOTS = 354_019_840
 

@@ -91,8 +91,8 @@ constexpr uint32_t P_TM_COLS = 128;                  // [K K^T ; Q K^T] (64 cols
 constexpr int kChainThreads = 320;                    // warps 0..7 state and output, 8 products, 9 copies
 constexpr int kCtrlWarp = 8;
 constexpr int kCopyWarp = 9;
-// stage: per k-block the rows [W_lo 0..63 | W_hi 64..127 | Q 128..191] (A operands
-// [W_lo; W_hi] and [W_hi; Q]), then K (two dk blocks), then [Mq_lo; Mq_hi]
+// stage: per k-block the rows [W_lo 0..63 | W_hi 64..127 | Q 128..191] (the M = 64 A
+// operands of W H0 and Q H0), then K (two dk blocks), then [Mq_lo; Mq_hi]
 constexpr uint32_t C_QW_KB = 192 * 128;
 constexpr uint32_t C_OFF_K = 2 * C_QW_KB;
 constexpr uint32_t C_OFF_MQ = C_OFF_K + 2 * BLK64;
@@ -759,12 +759,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // The handoffs (mbarrier: who completes it -> what it allows):
 //   full_qw, full_k, full_mq (per stage): a chunk's copies landed -> its products may read them
 //   bar_pw:  PW done (commit)           -> every state warp reads W H0 for the U phase
-//   bar_p:   P done (commit)            -> output warps read Q H0; the [Q | W] stage is free
+//   bar_p:   P done (commit)            -> every state warp reads Q H0, then may rewrite the H tiles
 //   u_ready: U, U' tiles written (8 warps) -> K^T U' and O may be issued
 //   bar_h:   K^T U' done (commit)       -> every state warp updates its part of H
-//   h_ready: H tiles written (8 warps)  -> the next chunk's P (which overwrites P's region)
-//   bar_o:   O done (commit)            -> output warps read it; the U tiles may be rewritten
-//   o_free:  O read (4 output warps)    -> the next O may be issued, the Mq stage refilled
+//   h_ready: H tiles written (8 warps)  -> the next chunk's PW (then its P, which overwrites P's region)
+//   bar_o:   O done (commit)            -> every state warp reads it; the U tiles may be rewritten
+//   o_free:  O read (8 warps)           -> the next O may be issued, the Mq stage refilled
 
 // the same for an mbarrier that another CTA of the cluster arrives on; it polls
 // (with a short back-off) instead of sleeping in try_wait
